@@ -1,0 +1,110 @@
+"""Seeded synthetic inputs shared by the tests and the bench.
+
+This module only draws random numbers (numpy PCG64 ``default_rng(seed)``) and
+rounds activations to bf16; it holds none of the quantiser's arithmetic.  The
+shapes, distributions and seeds stand in for the workloads the pages describe
+(Llama / SmolLM linear layers on the "glq 0.1.1" PyPI page, DiT linear layers in
+the EntroPack news item); no real weights exist in this environment, so every
+matrix here is random with the stated distribution.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import numpy as np
+
+# Per-bpw target RMS of the transformed, scaled weights (scale = rms(W) / SIGMA_T).
+# Frozen from a sweep of the oracle's reconstruction MSE on Gaussian rows
+# (oracle/sigma_sweep.py prints the sweep); the scale is an input of the
+# quantiser, so these numbers affect quality only, never parity.
+SIGMA_T = {2: 1.00, 3: 1.00, 4: 0.90}
+
+
+def gaussian_weights(N: int, K: int, std: float, seed) -> np.ndarray:
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((N, K), dtype=np.float64) * std).astype(np.float32)
+
+
+def student_t_outlier_weights(N: int, K: int, seed: int, std: float = 0.02, nu: float = 4.0,
+                              outlier_frac: float = 0.01, outlier_mult: float = 8.0) -> np.ndarray:
+    """Student-t (nu) rows scaled to the given std, then round(frac*K) seeded columns x mult."""
+    rng = np.random.default_rng(seed)
+    W = rng.standard_t(nu, size=(N, K)) * (std / np.sqrt(nu / (nu - 2.0)))
+    n_out = int(round(outlier_frac * K))
+    cols = rng.choice(K, size=n_out, replace=False)
+    W[:, cols] *= outlier_mult
+    return W.astype(np.float32)
+
+
+def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round fp32 to bf16 (round to nearest even), returned as uint16 bit patterns."""
+    b = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    b = (b + 0x7FFF + ((b >> 16) & 1)) >> 16
+    return b.astype(np.uint16)
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def activations_bf16(M: int, K: int, seed: int) -> np.ndarray:
+    """X ~ N(0, 1) rounded to bf16; uint16 bit patterns [M, K]."""
+    rng = np.random.default_rng(seed)
+    return f32_to_bf16_bits(rng.standard_normal((M, K), dtype=np.float64).astype(np.float32))
+
+
+def suggest_scale(W: np.ndarray, bpw: int) -> float:
+    """One global scale per layer: rms(W) in binary64 divided by SIGMA_T[bpw]."""
+    rms = float(np.sqrt(np.mean(np.square(W.astype(np.float64)))))
+    return float(np.float32(rms / SIGMA_T[bpw]))
+
+
+@dataclass
+class Layer:
+    name: str
+    N: int
+    K: int
+    bpw: int
+    w_seed: object                  # int, or (layer, matrix) pair seeding one numpy stream
+    rht_seed: int
+    std: float = 0.02
+    dist: str = "gaussian"          # or "student_t_outliers"
+
+    def weights(self) -> np.ndarray:
+        if self.dist == "gaussian":
+            return gaussian_weights(self.N, self.K, self.std, self.w_seed)
+        return student_t_outlier_weights(self.N, self.K, self.w_seed, std=self.std)
+
+
+@dataclass
+class Workload:
+    name: str
+    layers: list
+    M: list = field(default_factory=list)   # activation rows (tokens); empty = encode/decode only
+    x_seed: int = 0
+
+
+def workloads() -> dict:
+    """The five synthetic workloads (sizes, seeds, distributions, bits per weight)."""
+    w = {}
+    w["single_256"] = Workload("single_256", [Layer("w", 256, 256, 2, 0, 0)], M=[16], x_seed=1)
+    w["llama_4096_b4"] = Workload("llama_4096_b4", [Layer("w", 4096, 4096, 4, 2, 2)],
+                                  M=[1, 4, 16], x_seed=3)
+    w["mlp_up_14336_b3"] = Workload("mlp_up_14336_b3",
+                                    [Layer("up", 14336, 4096, 3, 4, 4, std=0.015)],
+                                    M=[4096], x_seed=5)
+    dit = [Layer("qkv", 9216, 3072, 4, 6, 6, dist="student_t_outliers"),
+           Layer("out", 3072, 3072, 4, 7, 7, dist="student_t_outliers"),
+           Layer("up", 12288, 3072, 4, 8, 8, dist="student_t_outliers"),
+           Layer("down", 3072, 12288, 4, 9, 9, dist="student_t_outliers")]
+    w["dit_3072_b4"] = Workload("dit_3072_b4", dit, M=[4096], x_seed=10)
+    shapes = [("q", 4096, 4096), ("k", 1024, 4096), ("v", 1024, 4096), ("o", 4096, 4096),
+              ("gate", 14336, 4096), ("up", 14336, 4096), ("down", 4096, 14336)]
+    for bpw in (2, 3, 4):
+        layers = []
+        for layer in range(32):
+            for mid, (nm, N, K) in enumerate(shapes):
+                layers.append(Layer("L%d.%s" % (layer, nm), N, K, bpw, (100 + layer, mid),
+                                    1000 * layer + mid))
+        w["llama3_8b_x32_b%d" % bpw] = Workload("llama3_8b_x32_b%d" % bpw, layers)
+    return w
