@@ -1,1 +1,236 @@
-"""E8 lattice-codebook weights decoded on the GPU and fed into a bf16 GEMM (B200, sm_100a)."""
+"""E8 lattice-codebook weights decoded on a B200 and fed into a bf16 GEMM.
+
+Thin ctypes binding over ``libe8.so`` (C ABI in ``include/e8.h``).  The
+functions carry the C names and only marshal arguments: tensors become device
+pointers, the current torch CUDA stream becomes the ``stream`` argument, and
+nonzero status codes raise :class:`E8Error`.  Every step of the computation
+runs in the library's CUDA kernels; if the library is missing this module
+raises instead of computing anything another way.
+
+Method: page "glq 0.1.1" on PyPI, "How it works" (E8 codebook of 65536 vectors
+from the first 7 shells, 16-bit index per 8 weights plus an 8/16-bit residual
+index at 3/4 bpw, randomized Hadamard transform, Euclidean nearest codebook
+vector) and the "Bit widths" table (one global scale per layer).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "_lib", "libe8.so")
+
+E8_OK, E8_EINVAL, E8_EWORKSPACE, E8_EDEVICE, E8_ECUDA, E8_ETIMEOUT, E8_ENOMEM = range(7)
+E8_GEMM_AUTO, E8_GEMM_ACT_RHT, E8_GEMM_DECODED_W, E8_GEMM_ACT_RHT_SMEM, E8_GEMM_SIMT = range(5)
+E8_OP_ENCODE = 100
+
+# every symbol include/e8.h declares
+EXPORTED = ("e8_codebook_build", "e8_codebook_free", "e8_codebook_export", "e8_rht_forward",
+            "e8_encode", "e8_decode_to_bf16", "e8_act_rht", "e8_gemm", "e8_gemm_auto_mode",
+            "e8_workspace_bytes", "e8_sync_status", "e8_debug_wait_timeout", "e8_status_str",
+            "e8_version")
+
+_lib = None
+
+
+class E8Error(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__("%s failed: %s (%d)" % (where, status_str(code), code))
+
+
+def load_library(path: str = LIB_PATH):
+    """Loads libe8.so and declares argument types.  Raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError("libe8.so not built (%s); run `python -m decode_gemm_e8_b200.build`" % path)
+    lib = ctypes.CDLL(path)
+    c = ctypes
+    P, I64, U64 = c.c_void_p, c.c_int64, c.c_uint64
+    sig = {
+        "e8_codebook_build": ([c.POINTER(c.c_void_p), c.c_int], c.c_int),
+        "e8_codebook_free": ([P], None),
+        "e8_codebook_export": ([P, P], c.c_int),
+        "e8_rht_forward": ([P, P, I64, I64, U64, c.c_float, P, P], c.c_int),
+        "e8_encode": ([P, P, I64, I64, c.c_int, U64, c.c_float, P, P, P, c.c_size_t, P], c.c_int),
+        "e8_decode_to_bf16": ([P, P, P, I64, I64, c.c_int, U64, c.c_float, P, P], c.c_int),
+        "e8_act_rht": ([P, I64, I64, U64, P, I64, P], c.c_int),
+        "e8_gemm": ([P, P, I64, P, P, I64, I64, c.c_int, U64, c.c_float, P, c.c_int, P,
+                     c.c_size_t, P], c.c_int),
+        "e8_gemm_auto_mode": ([I64, I64, I64, c.c_int], c.c_int),
+        "e8_workspace_bytes": ([c.c_int, I64, I64, I64, c.c_int], c.c_size_t),
+        "e8_sync_status": ([P, P], c.c_int),
+        "e8_debug_wait_timeout": ([P, c.c_int, P], c.c_int),
+        "e8_status_str": ([c.c_int], c.c_char_p),
+        "e8_version": ([], c.c_int),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = res
+    _lib = lib
+    return lib
+
+
+def status_str(code: int) -> str:
+    return load_library().e8_status_str(int(code)).decode()
+
+
+def _check(rc: int, where: str):
+    if rc != E8_OK:
+        raise E8Error(rc, where)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+class Codebook:
+    """Device-resident canonical codebook tables (``e8_codebook_build``)."""
+
+    def __init__(self, device: int = 0):
+        lib = load_library()
+        h = ctypes.c_void_p()
+        _check(lib.e8_codebook_build(ctypes.byref(h), int(device)), "e8_codebook_build")
+        self._h = h
+        self.device = int(device)
+
+    @property
+    def handle(self):
+        return self._h
+
+    def free(self):
+        if getattr(self, "_h", None):
+            load_library().e8_codebook_free(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.free()
+        except Exception:
+            pass
+
+
+def e8_codebook_build(device: int = 0) -> Codebook:
+    return Codebook(device)
+
+
+def e8_codebook_free(cb: Codebook) -> None:
+    cb.free()
+
+
+def e8_codebook_export(cb: Codebook):
+    """The 65536 codebook vectors as an int8 numpy array [65536, 8] of doubled coordinates."""
+    import numpy as np
+    out = np.zeros((65536, 8), dtype=np.int8)
+    _check(load_library().e8_codebook_export(cb.handle, ctypes.c_void_p(out.ctypes.data)),
+           "e8_codebook_export")
+    return out
+
+
+def e8_rht_forward(cb: Codebook, W, rht_seed: int, scale: float, U=None, stream=None):
+    import torch
+    N, K = W.shape
+    if U is None:
+        U = torch.empty_like(W)
+    _check(load_library().e8_rht_forward(cb.handle, _ptr(W), N, K, int(rht_seed) & (2**64 - 1),
+                                         float(scale), _ptr(U), _stream(stream)),
+           "e8_rht_forward")
+    return U
+
+
+def e8_workspace_bytes(op: int, M: int, N: int, K: int, bpw: int) -> int:
+    return int(load_library().e8_workspace_bytes(int(op), int(M), int(N), int(K), int(bpw)))
+
+
+def e8_gemm_auto_mode(M: int, N: int, K: int, bpw: int) -> int:
+    return int(load_library().e8_gemm_auto_mode(int(M), int(N), int(K), int(bpw)))
+
+
+def _workspace(nbytes: int, device, workspace=None):
+    import torch
+    if workspace is not None:
+        return workspace
+    return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device=device)
+
+
+def e8_encode(cb: Codebook, W, bpw: int, rht_seed: int, scale: float, idx1=None, idx2=None,
+              workspace=None, stream=None):
+    """W fp32 [N, K] (CUDA) -> (idx1 uint16 [N, K/8], idx2 uint8/uint16 [N, K/8] or None)."""
+    import torch
+    N, K = W.shape
+    dev = W.device
+    if idx1 is None:
+        idx1 = torch.empty((N, K // 8), dtype=torch.uint16, device=dev)
+    if idx2 is None and bpw > 2:
+        idx2 = torch.empty((N, K // 8), dtype=torch.uint8 if bpw == 3 else torch.uint16, device=dev)
+    need = e8_workspace_bytes(E8_OP_ENCODE, 0, N, K, bpw)
+    ws = _workspace(need, dev, workspace)
+    _check(load_library().e8_encode(cb.handle, _ptr(W), N, K, int(bpw), int(rht_seed) & (2**64 - 1),
+                                    float(scale), _ptr(idx1), _ptr(idx2), _ptr(ws), ws.numel(),
+                                    _stream(stream)), "e8_encode")
+    return idx1, idx2
+
+
+def e8_decode_to_bf16(cb: Codebook, idx1, idx2, N: int, K: int, bpw: int, rht_seed: int,
+                      scale: float, out=None, stream=None):
+    """Decoded weights, torch.bfloat16 [N, K] on the device of idx1."""
+    import torch
+    if out is None:
+        out = torch.empty((N, K), dtype=torch.bfloat16, device=idx1.device)
+    _check(load_library().e8_decode_to_bf16(cb.handle, _ptr(idx1), _ptr(idx2), N, K, int(bpw),
+                                            int(rht_seed) & (2**64 - 1), float(scale), _ptr(out),
+                                            _stream(stream)), "e8_decode_to_bf16")
+    return out
+
+
+def e8_act_rht(X, rht_seed: int, rows: int | None = None, out=None, stream=None):
+    """X bf16 [M, K] -> Xt bf16 [rows, K] (hi rows, lo rows, zero padding)."""
+    import torch
+    M, K = X.shape
+    rows = 2 * M if rows is None else int(rows)
+    if out is None:
+        out = torch.empty((rows, K), dtype=torch.bfloat16, device=X.device)
+    _check(load_library().e8_act_rht(_ptr(X), M, K, int(rht_seed) & (2**64 - 1), _ptr(out), rows,
+                                     _stream(stream)), "e8_act_rht")
+    return out
+
+
+def e8_gemm(cb: Codebook, X, idx1, idx2, N: int, K: int, bpw: int, rht_seed: int, scale: float,
+            mode: int = E8_GEMM_AUTO, Y=None, workspace=None, stream=None):
+    """Y fp32 [M, N] = X bf16 [M, K] times the decoded weights transposed."""
+    import torch
+    M = X.shape[0]
+    dev = X.device
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float32, device=dev)
+    need = e8_workspace_bytes(mode, M, N, K, bpw)
+    ws = _workspace(need, dev, workspace)
+    _check(load_library().e8_gemm(cb.handle, _ptr(X), M, _ptr(idx1), _ptr(idx2), N, K, int(bpw),
+                                  int(rht_seed) & (2**64 - 1), float(scale), _ptr(Y), int(mode),
+                                  _ptr(ws), ws.numel(), _stream(stream)), "e8_gemm")
+    return Y
+
+
+def e8_sync_status(cb: Codebook, stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the device status as a status code."""
+    return int(load_library().e8_sync_status(cb.handle, _stream(stream)))
+
+
+def e8_debug_wait_timeout(cb: Codebook, wait_ms: int, stream=None) -> None:
+    _check(load_library().e8_debug_wait_timeout(cb.handle, int(wait_ms), _stream(stream)),
+           "e8_debug_wait_timeout")
+
+
+def e8_version() -> int:
+    return int(load_library().e8_version())

@@ -1,0 +1,102 @@
+// Activation-side transform for the small-batch GEMM.
+//
+// With w_n = alpha D H z_n per Hadamard block (H symmetric, "glq 0.1.1",
+// "How it works", item 2), every output is
+//     y[m][n] = sum_k x_mk w_nk = alpha * sum_k (H D x_m)_k z_nk,
+// so the GEMM can run on the integer codebook vectors z (exact in bf16) once
+// the activations are transformed.  The transformed row xt = FWHT(D x) is
+// split into two bf16 parts, hi = bf16(xt) and lo = bf16(xt - hi), so that the
+// bf16 tensor-core product keeps about 16 significant bits of xt.
+#include "e8_common.cuh"
+#include "e8_internal.h"
+
+namespace e8 {
+
+__global__ void __launch_bounds__(256) k_act_rht(const uint16_t* __restrict__ X, int64_t M,
+                                                 int64_t K, int nh, int elems_per_cta,
+                                                 uint64_t seed, uint16_t* __restrict__ Xt) {
+  extern __shared__ __align__(16) float s_x[];
+  const int64_t total = M * K;
+  const int64_t base = (int64_t)blockIdx.x * elems_per_cta;
+  const int E = (int)(int64_t)min((long long)elems_per_cta, (long long)(total - base));
+  const int ngroups = E >> 3;
+  for (int g = threadIdx.x; g < ngroups; g += blockDim.x) {
+    int64_t e0 = base + 8 * (int64_t)g;
+    int64_t k0 = e0 % K;
+    uint4 raw = __ldg(reinterpret_cast<const uint4*>(X + e0));
+    uint32_t r[4] = {raw.x, raw.y, raw.z, raw.w};
+    float y[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      y[2 * i] = bf16_lo_to_f32(r[i]);
+      y[2 * i + 1] = bf16_hi_to_f32(r[i]);
+    }
+    uint64_t word = splitmix64_output(seed, (uint64_t)(k0 >> 6));
+    uint32_t bits = (uint32_t)(word >> (k0 & 63));
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      y[i] = __uint_as_float(__float_as_uint(y[i]) ^ (((bits >> i) & 1u) << 31));
+#pragma unroll
+    for (int h = 1; h < 8; h <<= 1) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if ((i & h) == 0) {
+          float a = y[i], c = y[i + h];
+          y[i] = a + c;
+          y[i + h] = a - c;
+        }
+      }
+    }
+    float4* dst = reinterpret_cast<float4*>(s_x + 8 * g);
+    dst[0] = make_float4(y[0], y[1], y[2], y[3]);
+    dst[1] = make_float4(y[4], y[5], y[6], y[7]);
+  }
+  const int half = E >> 1;
+  for (int h = 8; h < nh; h <<= 1) {
+    __syncthreads();
+    for (int b = threadIdx.x; b < half; b += blockDim.x) {
+      int i = (b / h) * (2 * h) + (b % h);
+      float a = s_x[i], c = s_x[i + h];
+      s_x[i] = a + c;
+      s_x[i + h] = a - c;
+    }
+  }
+  __syncthreads();
+  for (int g = threadIdx.x; g < ngroups; g += blockDim.x) {
+    int64_t e0 = base + 8 * (int64_t)g;
+    int64_t m = e0 / K, k0 = e0 % K;
+    const float4* src = reinterpret_cast<const float4*>(s_x + 8 * g);
+    float4 lo4 = src[0], hi4 = src[1];
+    float y[8] = {lo4.x, lo4.y, lo4.z, lo4.w, hi4.x, hi4.y, hi4.z, hi4.w};
+    uint32_t hw[4], lw[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      hw[i] = pack_bf16x2(y[2 * i], y[2 * i + 1]);
+      float r0 = y[2 * i] - bf16_lo_to_f32(hw[i]);
+      float r1 = y[2 * i + 1] - bf16_hi_to_f32(hw[i]);
+      lw[i] = pack_bf16x2(r0, r1);
+    }
+    *reinterpret_cast<uint4*>(Xt + m * K + k0) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    *reinterpret_cast<uint4*>(Xt + (M + m) * K + k0) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+  }
+}
+
+cudaError_t launch_act_rht(const uint16_t* X, int64_t M, int64_t K, uint64_t seed, uint16_t* Xt,
+                           int64_t rows, cudaStream_t st) {
+  const int nh = (int)hadamard_block(K);
+  const int epc = nh < 2048 ? 2048 : nh;
+  const int64_t total = M * K;
+  const int64_t ctas = (total + epc - 1) / epc;
+  const size_t smem = (size_t)epc * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(k_act_rht, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  if (rows > 2 * M) {
+    e = cudaMemsetAsync(Xt + 2 * M * K, 0, (size_t)(rows - 2 * M) * K * sizeof(uint16_t), st);
+    if (e != cudaSuccess) return e;
+  }
+  k_act_rht<<<(unsigned)ctas, 256, smem, st>>>(X, M, K, nh, epc, seed, Xt);
+  return cudaGetLastError();
+}
+
+}  // namespace e8

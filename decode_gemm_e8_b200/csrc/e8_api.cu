@@ -1,0 +1,333 @@
+// C ABI of libe8 (declared in include/e8.h): argument checks, workspace
+// carving, scale constants, kernel launches.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "e8.h"
+#include "e8_common.cuh"
+#include "e8_codebook.cuh"
+#include "e8_internal.h"
+
+struct e8_codebook {
+  int device;
+  int sm_count;
+  int8_t* vecs;
+  uint32_t* table;
+  uint32_t* hkeys;
+  uint32_t* hvals;
+  uint32_t* status;
+  int max_probe;
+};
+
+namespace {
+
+constexpr int64_t kMaxNh = 32768;
+constexpr size_t kTableAlloc = 131088;  // 32769 u32 padded to a multiple of 16 bytes
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_device(const e8_codebook* cb) {
+  if (!cb) return E8_EINVAL;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return E8_ECUDA;
+  return dev == cb->device ? E8_OK : E8_EDEVICE;
+}
+
+// K: positive multiple of 8 whose Hadamard block is at most 32768.
+bool valid_k(int64_t K) {
+  if (K < 8 || (K % 8) != 0) return false;
+  return e8::hadamard_block(K) <= kMaxNh;
+}
+
+bool valid_bpw(int bpw) { return bpw >= 2 && bpw <= 4; }
+
+int m_of(int bpw) { return bpw == 2 ? 2 : (bpw == 3 ? 4 : 8); }
+
+float gamma_of(float scale, int64_t nh) {
+  return (float)(1.0 / ((double)scale * std::sqrt((double)nh)));
+}
+
+float alpha_of(float scale, int64_t nh, int bpw) {
+  return (float)((double)scale / ((double)m_of(bpw) * std::sqrt((double)nh)));
+}
+
+e8::DeviceCodebook dev_view(const e8_codebook* cb) {
+  e8::DeviceCodebook d;
+  d.vecs = cb->vecs;
+  d.table = cb->table;
+  d.hkeys = cb->hkeys;
+  d.hvals = cb->hvals;
+  d.status = cb->status;
+  return d;
+}
+
+int rows_b_for(int64_t M) {
+  int64_t r = 2 * M;
+  r = (r + 15) / 16 * 16;
+  return (int)r;
+}
+
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? E8_OK : E8_ECUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int e8_version(void) { return 100; }
+
+const char* e8_status_str(int s) {
+  switch (s) {
+    case E8_OK: return "ok";
+    case E8_EINVAL: return "invalid argument";
+    case E8_EWORKSPACE: return "workspace too small";
+    case E8_EDEVICE: return "unsupported or wrong device";
+    case E8_ECUDA: return "CUDA error";
+    case E8_ETIMEOUT: return "device wait timed out";
+    case E8_ENOMEM: return "out of device memory";
+    default: return "unknown status";
+  }
+}
+
+int e8_codebook_build(e8_codebook** out, int device) {
+  if (!out) return E8_EINVAL;
+  *out = nullptr;
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) return E8_EDEVICE;
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, device) != cudaSuccess) return E8_ECUDA;
+  if (prop.major != 10) return E8_EDEVICE;
+  int prev = -1;
+  cudaGetDevice(&prev);
+  if (cudaSetDevice(device) != cudaSuccess) return E8_ECUDA;
+  e8_codebook* cb = new e8_codebook();
+  cb->device = device;
+  cb->sm_count = prop.multiProcessorCount;
+  int rc = E8_OK;
+  auto fail = [&](int code) {
+    cudaFree(cb->vecs);
+    cudaFree(cb->table);
+    cudaFree(cb->hkeys);
+    cudaFree(cb->hvals);
+    cudaFree(cb->status);
+    delete cb;
+    if (prev >= 0) cudaSetDevice(prev);
+    return code;
+  };
+  if (cudaMalloc(&cb->vecs, (size_t)e8::kCbSize * 8) != cudaSuccess) return fail(E8_ENOMEM);
+  if (cudaMalloc(&cb->table, kTableAlloc) != cudaSuccess) return fail(E8_ENOMEM);
+  if (cudaMalloc(&cb->hkeys, e8::kHashSlots * sizeof(uint32_t)) != cudaSuccess)
+    return fail(E8_ENOMEM);
+  if (cudaMalloc(&cb->hvals, e8::kHashSlots * sizeof(uint32_t)) != cudaSuccess)
+    return fail(E8_ENOMEM);
+  if (cudaMalloc(&cb->status, 16) != cudaSuccess) return fail(E8_ENOMEM);
+  cudaStream_t st;
+  if (cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking) != cudaSuccess) return fail(E8_ECUDA);
+  cudaMemsetAsync(cb->status, 0, 16, st);
+  cudaMemsetAsync(cb->table, 0, kTableAlloc, st);
+  int reps = e8::build_codebook_tables(cb->vecs, cb->table, cb->hkeys, cb->hvals, &cb->max_probe,
+                                       st);
+  cudaStreamDestroy(st);
+  // the E8 shells of squared norm 2..12 hold 117360 vectors, half of them
+  // positive representatives
+  if (reps != 58680) rc = E8_ECUDA;
+  if (rc != E8_OK) return fail(rc);
+  if (prev >= 0) cudaSetDevice(prev);
+  *out = cb;
+  return E8_OK;
+}
+
+void e8_codebook_free(e8_codebook* cb) {
+  if (!cb) return;
+  int prev = -1;
+  cudaGetDevice(&prev);
+  cudaSetDevice(cb->device);
+  cudaFree(cb->vecs);
+  cudaFree(cb->table);
+  cudaFree(cb->hkeys);
+  cudaFree(cb->hvals);
+  cudaFree(cb->status);
+  if (prev >= 0) cudaSetDevice(prev);
+  delete cb;
+}
+
+int e8_codebook_export(const e8_codebook* cb, int8_t* host_vecs) {
+  if (!cb || !host_vecs) return E8_EINVAL;
+  int prev = -1;
+  cudaGetDevice(&prev);
+  cudaSetDevice(cb->device);
+  cudaError_t e = cudaMemcpy(host_vecs, cb->vecs, (size_t)e8::kCbSize * 8, cudaMemcpyDeviceToHost);
+  if (prev >= 0) cudaSetDevice(prev);
+  return cuda_status(e);
+}
+
+int e8_rht_forward(const e8_codebook* cb, const float* W, int64_t N, int64_t K,
+                   uint64_t rht_seed, float scale, float* U, void* stream) {
+  int rc = check_device(cb);
+  if (rc != E8_OK) return rc;
+  if (N < 0 || !valid_k(K) || !(scale > 0.0f) || !std::isfinite(scale)) return E8_EINVAL;
+  if (N == 0) return E8_OK;
+  if (!W || !U || !aligned16(W) || !aligned16(U) || W == U) return E8_EINVAL;
+  const int64_t nh = e8::hadamard_block(K);
+  cudaError_t e = e8::launch_encode(dev_view(cb), W, N, K, 2, rht_seed, gamma_of(scale, nh),
+                                    nullptr, nullptr, nullptr, nullptr, 0, U, 0, cb->sm_count,
+                                    (cudaStream_t)stream);
+  return cuda_status(e);
+}
+
+size_t e8_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int bpw) {
+  if (!valid_bpw(bpw) || N < 0 || M < 0 || !valid_k(K)) return 0;
+  const size_t G = (size_t)N * (size_t)(K / 8);
+  switch (op) {
+    case E8_OP_ENCODE:
+      return 256 + G * sizeof(e8::WorkItem);
+    case E8_GEMM_AUTO:
+      return e8_workspace_bytes(e8_gemm_auto_mode(M, N, K, bpw), M, N, K, bpw);
+    case E8_GEMM_ACT_RHT:
+    case E8_GEMM_ACT_RHT_SMEM:
+      return round256((size_t)rows_b_for(M) * (size_t)K * 2);
+    case E8_GEMM_DECODED_W:
+    case E8_GEMM_SIMT:
+      return round256((size_t)N * (size_t)K * 2);
+    default:
+      return 0;
+  }
+}
+
+int e8_gemm_auto_mode(int64_t M, int64_t N, int64_t K, int bpw) {
+  (void)N;
+  (void)bpw;
+  if (M <= 64 && (K % 128) == 0) return E8_GEMM_ACT_RHT;
+  return E8_GEMM_DECODED_W;
+}
+
+int e8_encode(const e8_codebook* cb, const float* W, int64_t N, int64_t K, int bpw,
+              uint64_t rht_seed, float scale, uint16_t* idx1, void* idx2, void* workspace,
+              size_t ws_bytes, void* stream) {
+  int rc = check_device(cb);
+  if (rc != E8_OK) return rc;
+  if (N < 0 || !valid_k(K) || !valid_bpw(bpw) || !(scale > 0.0f) || !std::isfinite(scale))
+    return E8_EINVAL;
+  if ((bpw == 2) != (idx2 == nullptr)) return E8_EINVAL;
+  if (N == 0) return E8_OK;
+  if (!W || !idx1 || !aligned16(W) || !aligned16(idx1) || (idx2 && !aligned16(idx2)))
+    return E8_EINVAL;
+  const size_t need = e8_workspace_bytes(E8_OP_ENCODE, 0, N, K, bpw);
+  if (!workspace || !aligned16(workspace) || ws_bytes < need) return E8_EWORKSPACE;
+  const int64_t nh = e8::hadamard_block(K);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* count = reinterpret_cast<uint32_t*>(ws);
+  e8::WorkItem* items = reinterpret_cast<e8::WorkItem*>(ws + 256);
+  const uint64_t cap = (uint64_t)N * (uint64_t)(K / 8);
+  cudaError_t e = e8::launch_encode(dev_view(cb), W, N, K, bpw, rht_seed, gamma_of(scale, nh),
+                                    idx1, idx2, items, count, cap, nullptr, 1, cb->sm_count,
+                                    (cudaStream_t)stream);
+  return cuda_status(e);
+}
+
+int e8_decode_to_bf16(const e8_codebook* cb, const uint16_t* idx1, const void* idx2, int64_t N,
+                      int64_t K, int bpw, uint64_t rht_seed, float scale, uint16_t* W_dec,
+                      void* stream) {
+  int rc = check_device(cb);
+  if (rc != E8_OK) return rc;
+  if (N < 0 || !valid_k(K) || !valid_bpw(bpw) || !(scale > 0.0f) || !std::isfinite(scale))
+    return E8_EINVAL;
+  if ((bpw == 2) != (idx2 == nullptr)) return E8_EINVAL;
+  if (N == 0) return E8_OK;
+  if (!idx1 || !W_dec || !aligned16(idx1) || !aligned16(W_dec) || (idx2 && !aligned16(idx2)))
+    return E8_EINVAL;
+  const int64_t nh = e8::hadamard_block(K);
+  cudaError_t e = e8::launch_decode(dev_view(cb), idx1, idx2, N, K, bpw, rht_seed,
+                                    alpha_of(scale, nh, bpw), W_dec, (cudaStream_t)stream);
+  return cuda_status(e);
+}
+
+int e8_act_rht(const uint16_t* X, int64_t M, int64_t K, uint64_t rht_seed, uint16_t* Xt,
+               int64_t rows, void* stream) {
+  if (M < 0 || !valid_k(K) || rows < 2 * M) return E8_EINVAL;
+  if (M == 0) return E8_OK;
+  if (!X || !Xt || !aligned16(X) || !aligned16(Xt)) return E8_EINVAL;
+  return cuda_status(e8::launch_act_rht(X, M, K, rht_seed, Xt, rows, (cudaStream_t)stream));
+}
+
+int e8_gemm(const e8_codebook* cb, const uint16_t* X, int64_t M, const uint16_t* idx1,
+            const void* idx2, int64_t N, int64_t K, int bpw, uint64_t rht_seed, float scale,
+            float* Y, int mode, void* workspace, size_t ws_bytes, void* stream) {
+  int rc = check_device(cb);
+  if (rc != E8_OK) return rc;
+  if (M < 0 || N < 0 || !valid_k(K) || !valid_bpw(bpw) || !(scale > 0.0f) ||
+      !std::isfinite(scale))
+    return E8_EINVAL;
+  if ((bpw == 2) != (idx2 == nullptr)) return E8_EINVAL;
+  if (mode == E8_GEMM_AUTO) mode = e8_gemm_auto_mode(M, N, K, bpw);
+  if (mode < E8_GEMM_ACT_RHT || mode > E8_GEMM_SIMT) return E8_EINVAL;
+  const bool act = mode == E8_GEMM_ACT_RHT || mode == E8_GEMM_ACT_RHT_SMEM;
+  if (act && (M > 64 || (K % 128) != 0)) return E8_EINVAL;
+  if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return E8_EINVAL;
+  if (M == 0 || N == 0) return E8_OK;
+  if (!X || !idx1 || !Y || !aligned16(X) || !aligned16(idx1) || !aligned16(Y) ||
+      (idx2 && !aligned16(idx2)))
+    return E8_EINVAL;
+  const size_t need = e8_workspace_bytes(mode, M, N, K, bpw);
+  if (!workspace || !aligned16(workspace) || ws_bytes < need) return E8_EWORKSPACE;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int64_t nh = e8::hadamard_block(K);
+  const float alpha = alpha_of(scale, nh, bpw);
+  const e8::DeviceCodebook d = dev_view(cb);
+  cudaError_t e;
+  if (act) {
+    const int rows_b = rows_b_for(M);
+    uint16_t* Xt = static_cast<uint16_t*>(workspace);
+    e = e8::launch_act_rht(X, M, K, rht_seed, Xt, rows_b, st);
+    if (e != cudaSuccess) return E8_ECUDA;
+    e8::ActGemmArgs a;
+    a.Xt = Xt;
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.rows_b = rows_b;
+    a.idx1 = idx1;
+    a.idx2 = idx2;
+    a.bpw = bpw;
+    a.alpha = alpha;
+    a.Y = Y;
+    a.variant = mode == E8_GEMM_ACT_RHT ? 1 : 0;
+    e = e8::launch_act_gemm(d, a, cb->sm_count, st);
+    return cuda_status(e);
+  }
+  uint16_t* Wd = static_cast<uint16_t*>(workspace);
+  e = e8::launch_decode(d, idx1, idx2, N, K, bpw, rht_seed, alpha, Wd, st);
+  if (e != cudaSuccess) return E8_ECUDA;
+  if (mode == E8_GEMM_SIMT)
+    e = e8::launch_simt_gemm(X, M, Wd, N, K, Y, st);
+  else
+    e = e8::launch_dense_gemm(X, M, Wd, N, K, Y, cb->status, cb->sm_count, st);
+  return cuda_status(e);
+}
+
+int e8_sync_status(const e8_codebook* cb, void* stream) {
+  int rc = check_device(cb);
+  if (rc != E8_OK) return rc;
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return E8_ECUDA;
+  uint32_t s = 0;
+  if (cudaMemcpy(&s, cb->status, sizeof(s), cudaMemcpyDeviceToHost) != cudaSuccess) return E8_ECUDA;
+  if (s != 0 && cudaMemset(cb->status, 0, sizeof(s)) != cudaSuccess) return E8_ECUDA;
+  if (s & (e8::kDevTimeoutFull | e8::kDevTimeoutEmpty | e8::kDevTimeoutMma | e8::kDevTimeoutCluster))
+    return E8_ETIMEOUT;
+  if (s & e8::kDevWorklistOverflow) return E8_EWORKSPACE;
+  return E8_OK;
+}
+
+int e8_debug_wait_timeout(const e8_codebook* cb, int wait_ms, void* stream) {
+  int rc = check_device(cb);
+  if (rc != E8_OK) return rc;
+  if (wait_ms < 1 || wait_ms > 5000) return E8_EINVAL;
+  return cuda_status(e8::launch_wait_never_signalled(cb->status, (uint64_t)wait_ms * 1000000ull,
+                                                     (cudaStream_t)stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,66 @@
+// Declarations shared between the kernel translation units and the C ABI layer.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "e8_codebook.cuh"
+
+namespace e8 {
+
+// One group that the encoder's fast path could not decide exactly.
+struct WorkItem {
+  float u[8];      // transformed, scaled weights of the group
+  int64_t group;   // global group index (row * K/8 + column / 8)
+  uint32_t mask;   // bit 0: stage 1 undecided, bit 1: stage 2 undecided
+  uint32_t pad;
+};
+static_assert(sizeof(WorkItem) == 48, "WorkItem layout");
+
+int build_codebook_tables(int8_t* d_vecs, uint32_t* d_table, uint32_t* d_hkeys, uint32_t* d_hvals,
+                          int* h_max_probe, cudaStream_t st);
+
+int encode_elems_per_cta(int nh);
+cudaError_t launch_encode(const DeviceCodebook& cb, const float* W, int64_t N, int64_t K, int bpw,
+                          uint64_t seed, float gamma, uint16_t* idx1, void* idx2,
+                          WorkItem* work, uint32_t* work_count, uint64_t work_cap, float* U,
+                          int do_quantise, int sm_count, cudaStream_t st);
+
+cudaError_t launch_decode(const DeviceCodebook& cb, const uint16_t* idx1, const void* idx2,
+                          int64_t N, int64_t K, int bpw, uint64_t seed, float alpha,
+                          uint16_t* Wdec, cudaStream_t st);
+
+// X [M][K] bf16 -> Xt [rows][K] bf16: rows [0, M) hi parts, [M, 2M) lo parts of
+// FWHT(D x), rows [2M, rows) zero.
+cudaError_t launch_act_rht(const uint16_t* X, int64_t M, int64_t K, uint64_t seed, uint16_t* Xt,
+                           int64_t rows, cudaStream_t st);
+
+// Fused decode + GEMM with the transform moved onto the activations:
+// Y[m][n] = alpha * sum_k Xt[m][k] Z[n][k] (hi + lo rows), Z decoded on chip.
+struct ActGemmArgs {
+  const uint16_t* Xt;   // [rows_b][K], rows_b = padded 2M
+  int64_t M, N, K;
+  int rows_b;           // MMA N dimension (16..256, multiple of 16)
+  const uint16_t* idx1;
+  const void* idx2;
+  int bpw;
+  float alpha;
+  float* Y;             // [M][N] fp32
+  int variant;          // 0: decoded operand in shared memory, 1: in tensor memory
+};
+cudaError_t launch_act_gemm(const DeviceCodebook& cb, const ActGemmArgs& a, int sm_count,
+                            cudaStream_t st);
+
+// Dense Y[M][N] fp32 = X[M][K] bf16 * W[N][K]^T bf16 on tcgen05.
+cudaError_t launch_dense_gemm(const uint16_t* X, int64_t M, const uint16_t* W, int64_t N,
+                              int64_t K, float* Y, uint32_t* status, int sm_count,
+                              cudaStream_t st);
+
+// Reference-quality CUDA-core GEMM used by the simt mode (diagnostics).
+cudaError_t launch_simt_gemm(const uint16_t* X, int64_t M, const uint16_t* W, int64_t N,
+                             int64_t K, float* Y, cudaStream_t st);
+
+// Failure-detection check: a bounded wait on a barrier nobody signals.
+cudaError_t launch_wait_never_signalled(uint32_t* status, uint64_t limit_ns, cudaStream_t st);
+
+}  // namespace e8

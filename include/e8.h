@@ -1,0 +1,169 @@
+/*
+ * libe8 -- E8 lattice-codebook weights decoded on a B200 (sm_100a) GPU and
+ * fed into a bf16 tensor-core GEMM, plus the data-parallel encoder.
+ *
+ * The method is the one described on the PyPI page of "glq 0.1.1"
+ * (section "How it works" and the "Bit widths" table):
+ *   - a codebook of 65536 vectors of the E8 lattice taken from its first seven
+ *     shells (squared norms 0, 2, ..., 12); each group of 8 consecutive weights
+ *     of a row is replaced by a 16-bit codebook index (2 bits per weight);
+ *   - for 3 and 4 bits per weight a second-stage residual codebook adds an
+ *     8-bit or a 16-bit index per group;
+ *   - before quantisation every weight row is passed through a randomized
+ *     Hadamard transform (random sign flips, then a fast Walsh-Hadamard
+ *     transform), and each group is mapped to its Euclidean nearest codebook
+ *     vector;
+ *   - one global scale per layer, no per-group scales, so the storage is
+ *     exactly bpw * N * K / 8 bytes plus the scale (and the transform seed).
+ *
+ * Conventions fixed by this library where the page is silent:
+ *   - weights W are [N][K] row-major (output rows, input columns); groups and
+ *     the transform run along K; the Hadamard block n_h is the largest power
+ *     of two dividing K (block-diagonal transform when K is not a power of
+ *     two); n_h must not exceed 32768;
+ *   - codebook order: origin first, then shells by increasing norm; inside a
+ *     shell the vectors whose first nonzero coordinate is positive, sorted
+ *     lexicographically on their coordinates, each followed by its negation;
+ *     cut at 65536 entries;
+ *   - residual codebook: the first 256 entries at scale 1/2 (3 bpw) or the
+ *     whole codebook at scale 1/4 (4 bpw), chosen greedily after stage 1;
+ *   - nearest means exact Euclidean distance on the fp32 transformed weights,
+ *     ties resolved to the smallest index;
+ *   - sign vector: SplitMix64 stream seeded with rht_seed, output word j gives
+ *     the signs of columns 64j..64j+63 (bit set = negate);
+ *   - forward transform: u = fl32(FWHT(D w) * gamma) in fp32, stages
+ *     h = 1, 2, 4, ..., butterfly (a, b) -> (a + b, a - b),
+ *     gamma = fl32(1 / (scale * sqrt(n_h)));
+ *   - decoded weight: w = bf16_rne(d * fl32(t * alpha)), t = FWHT(z) computed
+ *     exactly on the integer group vectors z = m (c1 + beta c2), m = 2, 4, 8
+ *     for 2, 3, 4 bpw, alpha = fl32(scale / (m * sqrt(n_h))).
+ *
+ * General rules for every call below:
+ *   - all pointers are device pointers unless a parameter says "host";
+ *     device pointers must be 16-byte aligned;
+ *   - the caller owns every buffer; only e8_codebook_build allocates (device
+ *     tables, freed by e8_codebook_free);
+ *   - calls are asynchronous on `stream` (a cudaStream_t, NULL = legacy
+ *     default stream) and never synchronise, except e8_codebook_build,
+ *     e8_codebook_export and e8_sync_status, which are synchronous;
+ *   - the current CUDA device must be the device the codebook was built on;
+ *   - N == 0 or M == 0 is a valid empty call that launches nothing;
+ *   - argument errors are reported before anything is launched.
+ */
+#ifndef E8_H
+#define E8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes. */
+#define E8_OK 0          /* success */
+#define E8_EINVAL 1      /* bad argument: null/misaligned pointer, shape, bpw, scale, mode */
+#define E8_EWORKSPACE 2  /* workspace missing or smaller than e8_workspace_bytes() */
+#define E8_EDEVICE 3     /* no sm_100 device, or the current device is not the codebook's */
+#define E8_ECUDA 4       /* a CUDA runtime or driver call failed */
+#define E8_ETIMEOUT 5    /* a kernel gave up on a bounded wait (reported by e8_sync_status) */
+#define E8_ENOMEM 6      /* device allocation failed (e8_codebook_build only) */
+
+/* GEMM modes (e8_gemm `mode`, and `op` of e8_workspace_bytes). */
+#define E8_GEMM_AUTO 0          /* ACT_RHT for M <= 64 and K % 128 == 0, else DECODED_W */
+#define E8_GEMM_ACT_RHT 1       /* transform on the activations, codes decoded on chip into
+                                   tensor memory, fused tcgen05 GEMM (M <= 64, K % 128 == 0) */
+#define E8_GEMM_DECODED_W 2     /* decode to a bf16 workspace, then a dense tcgen05 GEMM */
+#define E8_GEMM_ACT_RHT_SMEM 3  /* as ACT_RHT, decoded operand staged in shared memory */
+#define E8_GEMM_SIMT 4          /* decode to bf16, CUDA-core fp32 GEMM (diagnostic) */
+#define E8_OP_ENCODE 100        /* e8_workspace_bytes: workspace of e8_encode */
+
+typedef struct e8_codebook e8_codebook;
+
+/* Builds the canonical codebook tables on CUDA device `device` ("How it
+ * works", item 1) and stores an opaque handle in *out.  Synchronous.
+ * Allocates about 1.2 MB of device memory.  Errors: E8_EINVAL (out NULL),
+ * E8_EDEVICE (device missing or not compute capability 10.x), E8_ENOMEM,
+ * E8_ECUDA. */
+int e8_codebook_build(e8_codebook** out, int device);
+
+/* Releases the tables of a codebook built by e8_codebook_build (NULL is a no-op). */
+void e8_codebook_free(e8_codebook* cb);
+
+/* Copies the 65536 codebook vectors, doubled coordinates (2x, all in [-6, 6]),
+ * as int8 [65536][8] into the HOST buffer host_vecs.  Synchronous. */
+int e8_codebook_export(const e8_codebook* cb, int8_t* host_vecs);
+
+/* Forward randomized Hadamard transform of every row ("How it works", item 2):
+ * U = fl32(FWHT_{n_h}(D W) * gamma), W and U fp32 [N][K] (may not alias).
+ * Bit-exact to the sequential definition given at the top of this file. */
+int e8_rht_forward(const e8_codebook* cb, const float* W, int64_t N, int64_t K,
+                   uint64_t rht_seed, float scale, float* U, void* stream);
+
+/* Encoder ("How it works", items 1-2; "Bit widths" table): W fp32 [N][K] ->
+ * idx1 uint16 [N][K/8] and, for bpw 3, idx2 uint8 [N][K/8], for bpw 4 idx2
+ * uint16 [N][K/8] (idx2 must be NULL for bpw 2).  scale > 0 is the layer's
+ * global scale.  Every index equals the exact nearest codebook point of the
+ * transformed, scaled group (smallest index on ties); groups with a
+ * non-finite coordinate get index 0.  workspace: at least
+ * e8_workspace_bytes(E8_OP_ENCODE, 0, N, K, bpw) bytes, contents ignored. */
+int e8_encode(const e8_codebook* cb, const float* W, int64_t N, int64_t K, int bpw,
+              uint64_t rht_seed, float scale, uint16_t* idx1, void* idx2, void* workspace,
+              size_t ws_bytes, void* stream);
+
+/* Decoder: indices -> bf16 weights W_dec [N][K] (raw bf16 bits), the exact
+ * inverse transform followed by the two roundings given at the top of this
+ * file, bit-exact.  Needs no workspace. */
+int e8_decode_to_bf16(const e8_codebook* cb, const uint16_t* idx1, const void* idx2, int64_t N,
+                      int64_t K, int bpw, uint64_t rht_seed, float scale, uint16_t* W_dec,
+                      void* stream);
+
+/* Activation-side transform used by E8_GEMM_ACT_RHT: X bf16 [M][K] ->
+ * Xt bf16 [rows][K] with rows >= 2M; row m holds hi = bf16(FWHT(D x_m)) and
+ * row M + m holds lo = bf16(FWHT(D x_m) - hi); rows 2M..rows-1 are zeroed.
+ * No normalisation is applied (the GEMM multiplies by alpha). */
+int e8_act_rht(const uint16_t* X, int64_t M, int64_t K, uint64_t rht_seed, uint16_t* Xt,
+               int64_t rows, void* stream);
+
+/* GEMM with compressed weights: Y fp32 [M][N] = X bf16 [M][K] * W_dec^T, where
+ * W_dec is what e8_decode_to_bf16 returns for (idx1, idx2, scale, rht_seed).
+ * In the DECODED_W and SIMT modes the product uses W_dec itself; in the
+ * ACT_RHT modes it uses the unrounded decoded weights (relative Frobenius
+ * difference to the W_dec product about 1.7e-3, from the bf16 rounding of
+ * W_dec).  workspace: at least e8_workspace_bytes(mode, M, N, K, bpw) bytes. */
+int e8_gemm(const e8_codebook* cb, const uint16_t* X, int64_t M, const uint16_t* idx1,
+            const void* idx2, int64_t N, int64_t K, int bpw, uint64_t rht_seed, float scale,
+            float* Y, int mode, void* workspace, size_t ws_bytes, void* stream);
+
+/* Mode that E8_GEMM_AUTO selects for these sizes. */
+int e8_gemm_auto_mode(int64_t M, int64_t N, int64_t K, int bpw);
+
+/* Workspace bytes for e8_encode (op = E8_OP_ENCODE) or for e8_gemm in mode
+ * `op`; 0 if the arguments are invalid or nothing is needed. */
+size_t e8_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int bpw);
+
+/* Synchronises `stream`, then reads and clears the codebook's device status
+ * word.  Returns E8_ETIMEOUT if a kernel gave up on a bounded wait since the
+ * last call, E8_EWORKSPACE on an encoder work-list overflow, E8_ECUDA if the
+ * stream reported an error, else E8_OK. */
+int e8_sync_status(const e8_codebook* cb, void* stream);
+
+/* Failure-detection check (diagnostic): launches one thread that waits on a
+ * barrier nothing ever signals, gives up after wait_ms (1..5000) milliseconds
+ * and sets the timeout bit of the codebook's status word, the same way every
+ * pipeline kernel reports a wait that ran out.  The next e8_sync_status then
+ * returns E8_ETIMEOUT; the CUDA context stays usable.  The paper has no
+ * counterpart; this exists to test the library's error reporting. */
+int e8_debug_wait_timeout(const e8_codebook* cb, int wait_ms, void* stream);
+
+/* Human-readable name of a status code (static string). */
+const char* e8_status_str(int status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int e8_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* E8_H */

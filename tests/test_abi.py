@@ -1,0 +1,74 @@
+"""The C-ABI library loads on the CPU host and exports every symbol that
+include/e8.h declares; host-only entry points answer without a GPU."""
+import os
+import re
+
+import pytest
+
+import decode_gemm_e8_b200 as e8
+from decode_gemm_e8_b200 import build as e8build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "e8.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(e8_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    e8build.build()
+    return e8.load_library()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert "e8_gemm" in names and "e8_encode" in names and len(names) >= 12
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(e8.EXPORTED)
+
+
+def test_library_is_sm100a_only():
+    # the build passes exactly one -gencode, for sm_100a
+    assert e8build.ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
+
+
+def test_status_strings_and_version(lib):
+    assert e8.status_str(0) == "ok"
+    assert "timed out" in e8.status_str(5)
+    assert e8.e8_version() >= 100
+
+
+def test_workspace_sizes(lib):
+    N, K = 4096, 4096
+    assert e8.e8_workspace_bytes(e8.E8_OP_ENCODE, 0, N, K, 4) == 256 + 48 * N * K // 8
+    assert e8.e8_workspace_bytes(e8.E8_GEMM_DECODED_W, 4096, N, K, 3) == N * K * 2
+    # hi and lo rows for 16 tokens: 32 rows of K bf16
+    assert e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT, 16, N, K, 4) == 32 * K * 2
+    assert e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT, 1, N, K, 4) == 16 * K * 2
+    assert e8.e8_workspace_bytes(e8.E8_GEMM_AUTO, 16, N, K, 4) == 32 * K * 2
+    assert e8.e8_workspace_bytes(e8.E8_GEMM_AUTO, 4096, N, K, 4) == N * K * 2
+    # invalid arguments give 0
+    assert e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT, 16, N, 100, 4) == 0
+    assert e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT, 16, N, K, 5) == 0
+    assert e8.e8_workspace_bytes(e8.E8_OP_ENCODE, 0, N, 65536, 2) == 0
+
+
+def test_auto_mode(lib):
+    assert e8.e8_gemm_auto_mode(16, 4096, 4096, 4) == e8.E8_GEMM_ACT_RHT
+    assert e8.e8_gemm_auto_mode(64, 4096, 4096, 4) == e8.E8_GEMM_ACT_RHT
+    assert e8.e8_gemm_auto_mode(65, 4096, 4096, 4) == e8.E8_GEMM_DECODED_W
+    assert e8.e8_gemm_auto_mode(16, 4096, 264, 4) == e8.E8_GEMM_DECODED_W
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    saved = e8._lib
+    try:
+        e8._lib = None
+        with pytest.raises(ImportError):
+            e8.load_library(str(tmp_path / "absent.so"))
+    finally:
+        e8._lib = saved

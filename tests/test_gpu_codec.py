@@ -1,0 +1,192 @@
+"""GPU parity of the codebook build, forward transform, encoder and decoder
+against the CPU oracle, through the C ABI.
+
+Bar: bit-exact (integer indices, fp32 transformed weights, bf16 decoded
+weights).  Sizes: full matrices where the oracle's brute force finishes in
+seconds; at the full workload sizes, every group of a seeded sample of rows
+(rows are independent, so the oracle can process just those rows).
+"""
+import numpy as np
+import pytest
+import torch
+
+import decode_gemm_e8_b200 as e8
+from decode_gemm_e8_b200 import synth
+from oracle import oracle as orc
+from tests import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def gcb():
+    gu.dev()
+    from decode_gemm_e8_b200 import build
+    build.build()
+    return e8.Codebook(0)
+
+
+def test_codebook_matches_oracle_byte_for_byte(gcb, cb):
+    got = e8.e8_codebook_export(gcb)
+    assert np.array_equal(got, cb)
+
+
+@pytest.mark.parametrize("N,K,seed", [(3, 256, 0), (5, 3072, 7), (2, 4096, 11), (1, 14336, 3),
+                                      (3, 12288, 5), (7, 8, 1), (2, 32768, 9), (130, 264, 2)])
+def test_rht_forward_bit_exact(gcb, N, K, seed):
+    W = synth.gaussian_weights(N, K, 0.02, seed)
+    s = synth.suggest_scale(W, 4)
+    U = gu.to_np(e8.e8_rht_forward(gcb, gu.to_dev(W), seed + 100, s))
+    ref = orc.rht_forward(W, seed + 100, s)
+    assert np.array_equal(U.view(np.uint32), ref.view(np.uint32))
+
+
+def _encode_both(gcb, W, bpw, rs, s, rows=None):
+    i1, i2 = e8.e8_encode(gcb, gu.to_dev(W), bpw, rs, s)
+    g1 = gu.to_np(i1)
+    g2 = gu.to_np(i2) if i2 is not None else None
+    Wr = W if rows is None else W[rows]
+    r1, r2 = orc.encode(Wr, bpw, rs, s)
+    if rows is not None:
+        g1 = g1[rows]
+        g2 = g2[rows] if g2 is not None else None
+    return g1, g2, r1, r2
+
+
+@pytest.mark.parametrize("bpw", [2, 3, 4])
+def test_encode_single_256_full(gcb, bpw):
+    # the single-layer workload (W 256x256 ~ N(0, 0.02^2), seed 0), every group
+    lay = synth.workloads()["single_256"].layers[0]
+    W = lay.weights()
+    s = synth.suggest_scale(W, bpw)
+    g1, g2, r1, r2 = _encode_both(gcb, W, bpw, lay.rht_seed, s)
+    assert np.array_equal(g1, r1)
+    if bpw > 2:
+        assert g2.dtype == r2.dtype
+        assert np.array_equal(g2, r2)
+
+
+@pytest.mark.parametrize("bpw,sigma_mult", [(2, 1.0), (2, 3.0), (3, 0.5), (4, 1.0), (4, 2.5)])
+def test_encode_many_scales(gcb, bpw, sigma_mult):
+    # overload-heavy (small scale) and granular (large scale) regimes, ragged row count
+    W = synth.gaussian_weights(37, 1024, 0.02, 40 + bpw)
+    s = synth.suggest_scale(W, bpw) / sigma_mult
+    g1, g2, r1, r2 = _encode_both(gcb, W, bpw, 77, s)
+    assert np.array_equal(g1, r1)
+    if bpw > 2:
+        assert np.array_equal(g2, r2)
+
+
+def test_encode_planted_ties_and_lattice_points(gcb, cb):
+    # W whose transformed groups land exactly on codebook points, on midpoints
+    # between lattice neighbours (exact ties) and on deep holes
+    n = 256
+    rng = np.random.default_rng(5)
+    G = 4 * n // 8
+    U = np.zeros((G, 8))
+    roots = cb[1:241].astype(np.float64) / 2
+    for g in range(G):
+        kind = g % 4
+        a = cb[rng.integers(0, 30000)].astype(np.float64) / 2
+        if kind == 0:
+            U[g] = a
+        elif kind == 1:
+            U[g] = a + roots[rng.integers(0, 240)] / 2
+        elif kind == 2:
+            U[g] = np.eye(8)[rng.integers(0, 8)] * (1 if rng.integers(2) else -1)
+        else:
+            U[g] = a / 4
+    U = U.reshape(4, n)
+    # W = s * D H U / sqrt(n) makes u = U up to fp32 rounding; with s = 1/sqrt(n)
+    # gamma = 1 and the transform of small dyadic values is exact in fp32
+    from tests import indep
+    H = indep.sylvester(n).astype(np.float64)
+    d = orc.signs(3, n).astype(np.float64)
+    s = float(np.float32(1.0 / np.sqrt(n)))
+    W = (d[None, :] * (U @ H) / n).astype(np.float32)
+    assert np.array_equal(orc.rht_forward(W, 3, s).astype(np.float64), U)
+    for bpw in (2, 3, 4):
+        g1, g2, r1, r2 = _encode_both(gcb, W, bpw, 3, s)
+        assert np.array_equal(g1, r1)
+        if bpw > 2:
+            assert np.array_equal(g2, r2)
+
+
+def test_encode_zero_and_nonfinite(gcb):
+    W = np.zeros((4, 512), np.float32)
+    W[1, 17] = np.nan
+    W[2, 300] = np.inf
+    i1, i2 = e8.e8_encode(gcb, gu.to_dev(W), 4, 1, 0.01)
+    g1, g2 = gu.to_np(i1), gu.to_np(i2)
+    r1, r2 = orc.encode(W, 4, 1, 0.01)
+    assert np.array_equal(g1, r1) and np.array_equal(g2, r2)
+    assert not g1[0].any() and not g1[3].any()
+
+
+def _sample_rows(N, k, seed):
+    return np.sort(np.random.default_rng(seed).choice(N, size=min(k, N), replace=False))
+
+
+@pytest.mark.parametrize("wl", ["llama_4096_b4", "mlp_up_14336_b3", "dit_3072_b4"])
+def test_encode_full_size_sampled_rows(gcb, wl):
+    for li, lay in enumerate(synth.workloads()[wl].layers):
+        W = lay.weights()
+        s = synth.suggest_scale(W, lay.bpw)
+        rows = _sample_rows(lay.N, 6, 100 + li)
+        g1, g2, r1, r2 = _encode_both(gcb, W, lay.bpw, lay.rht_seed, s, rows)
+        assert np.array_equal(g1, r1), lay.name
+        assert np.array_equal(g2, r2), lay.name
+
+
+@pytest.mark.parametrize("bpw", [2, 3, 4])
+def test_encode_llama3_layer_sampled_rows(gcb, bpw):
+    layers = synth.workloads()["llama3_8b_x32_b%d" % bpw].layers
+    for lay in layers[:7]:          # the seven matrices of decoder layer 0
+        W = lay.weights()
+        s = synth.suggest_scale(W, bpw)
+        rows = _sample_rows(lay.N, 3, lay.rht_seed + 1)
+        g1, g2, r1, r2 = _encode_both(gcb, W, bpw, lay.rht_seed, s, rows)
+        assert np.array_equal(g1, r1), lay.name
+        if bpw > 2:
+            assert np.array_equal(g2, r2), lay.name
+
+
+def _random_codes(N, K, bpw, seed):
+    rng = np.random.default_rng(seed)
+    i1 = rng.integers(0, 65536, (N, K // 8)).astype(np.uint16)
+    i2 = None
+    if bpw == 3:
+        i2 = rng.integers(0, 256, (N, K // 8)).astype(np.uint8)
+    if bpw == 4:
+        i2 = rng.integers(0, 65536, (N, K // 8)).astype(np.uint16)
+    return i1, i2
+
+
+@pytest.mark.parametrize("bpw,N,K", [(2, 256, 256), (3, 33, 3072), (4, 17, 4096), (4, 5, 14336),
+                                     (3, 9, 12288), (2, 3, 32768), (4, 130, 264), (2, 1, 8)])
+def test_decode_bit_exact(gcb, bpw, N, K):
+    i1, i2 = _random_codes(N, K, bpw, N + K + bpw)
+    s = 0.0173
+    out = e8.e8_decode_to_bf16(gcb, gu.to_dev(i1), None if i2 is None else gu.to_dev(i2), N, K,
+                               bpw, 42, s)
+    ref = orc.decode(i1, i2, N, K, bpw, 42, s)
+    assert np.array_equal(gu.to_np(out), ref)
+
+
+@pytest.mark.parametrize("wl", ["llama_4096_b4", "mlp_up_14336_b3"])
+def test_encode_decode_full_size(gcb, wl):
+    lay = synth.workloads()[wl].layers[0]
+    W = lay.weights()
+    s = synth.suggest_scale(W, lay.bpw)
+    i1, i2 = e8.e8_encode(gcb, gu.to_dev(W), lay.bpw, lay.rht_seed, s)
+    out = gu.to_np(e8.e8_decode_to_bf16(gcb, i1, i2, lay.N, lay.K, lay.bpw, lay.rht_seed, s))
+    rows = _sample_rows(lay.N, 16, 9)
+    h1, h2 = gu.to_np(i1), gu.to_np(i2)
+    ref = orc.decode(h1[rows], h2[rows], len(rows), lay.K, lay.bpw, lay.rht_seed, s)
+    assert np.array_equal(out[rows], ref)
+    # reconstruction quality of the whole matrix: relative MSE in the range the
+    # oracle's scale sweep gives for this rate
+    wd = synth.bf16_bits_to_f32(out).astype(np.float64)
+    rel = np.mean((wd - W) ** 2) / np.mean(W.astype(np.float64) ** 2)
+    assert rel < {2: 0.1, 3: 0.035, 4: 0.0095}[lay.bpw]
+    assert e8.e8_sync_status(gcb) == e8.E8_OK
