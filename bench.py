@@ -1,0 +1,521 @@
+"""Benchmark of the E8-codebook decode GEMM on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload (the small-batch decode configuration): one Llama-style linear layer,
+W 4096 x 4096 ~ N(0, 0.02^2) (seed 2) quantised at 4 bits per weight (16-bit
+index + 16-bit residual index per 8 weights, one global scale), activations
+X 16 x 4096 bf16 ~ N(0, 1) (seed 3).  One step is one call of the hot path:
+the activation-side Hadamard transform plus the fused decode + tcgen05 GEMM
+(E8_GEMM_AUTO picks it for 16 tokens).  The compressed weights were produced
+by the GPU encoder beforehand and stay resident; the step rotates over 32
+copies of them (32 x 8.4 MB > 126 MB L2) so every step reads its codes from HBM.
+
+Printed (rank 0, one JSON line): whole-job TFLOP/s (2 M N K per step), decoded
+weights/s, the roofline of the dominant kernel (HBM bound), an end-to-end
+number through the public API with host buffers, the other hot-path rows
+(encode, decode to bf16, 1 and 4 tokens) and the CPU oracle timed on this
+host as a baseline.  Multi-GPU (torchrun): every rank runs its own layer
+(independent weight matrices, no collective on the data path), weak scaling.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "llama_4096_b4"
+M_HEAD = 16
+ROTATE = 32
+GRAPH_STEPS = 1000
+METRIC = "fused E8-decode GEMM TFLOP/s & decoded weights/s, as % of HBM/tensor roofline"
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# ------------------------------------------------------------------ clocks --
+_REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+            0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+            0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+            0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with nvidia-smi while running."""
+
+    def __init__(self, index: int, period_ms: int = 100):
+        self.index, self.period = index, period_ms
+        self.samples = []
+        self.proc = None
+        self.marks = []
+
+    def start(self):
+        cmd = ["nvidia-smi", "-i", str(self.index),
+               "--query-gpu=clocks.sm,clocks.max.sm,clocks_event_reasons.active",
+               "--format=csv,noheader,nounits", "-lms", str(self.period)]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 3:
+                continue
+            try:
+                self.samples.append((time.time(), float(parts[0]), float(parts[1]),
+                                     int(parts[2], 16)))
+            except ValueError:
+                pass
+
+    def mark(self):
+        self.marks.append(time.time())
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0, t1, fallback_t0=None):
+        sel = [s for s in self.samples if t0 <= s[0] <= t1]
+        window = "timed region"
+        if len(sel) < 3 and fallback_t0 is not None:
+            sel = [s for s in self.samples if fallback_t0 <= s[0] <= t1]
+            window = "timed region and the load phase just before it (same workload)"
+        if not sel:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "window": window}
+        mask = 0
+        for s in sel:
+            mask |= s[3]
+        return {"sm_mhz": statistics.median(s[1] for s in sel), "sm_max_mhz": max(s[2] for s in sel),
+                "reasons": sorted(v for k, v in _REASONS.items() if mask & k and k != 0x1),
+                "samples": len(sel), "window": window}
+
+
+# ------------------------------------------------------------- distributed --
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def _max_over_ranks(x: float, ws: int, device):
+    if ws == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# -------------------------------------------------------------- our arm ----
+def _graph_of(fn, n, stream):
+    import torch
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(n):
+            fn(i)
+    return g
+
+
+def _time_graphs(fn, steps, warmup, stream):
+    """Captures fn(i) for i in [0, G) into graphs covering exactly `steps` calls,
+    replays `warmup` untimed calls first, returns elapsed ms of the timed replay."""
+    import torch
+    G = min(GRAPH_STEPS, max(1, steps))
+    full, rem = divmod(steps, G)
+    g_full = _graph_of(fn, G, stream)
+    g_rem = _graph_of(fn, rem, stream) if rem else None
+    torch.cuda.synchronize()
+    wg = _graph_of(fn, min(warmup, G), stream) if warmup > 0 else None
+    if wg is not None:
+        for _ in range(max(1, warmup // max(1, min(warmup, G)))):
+            wg.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(full):
+            g_full.replay()
+        if g_rem is not None:
+            g_rem.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def run_ours(args):
+    import torch
+    import decode_gemm_e8_b200 as e8
+    from decode_gemm_e8_b200 import build, synth
+
+    ws, rank, local = _dist()
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    build.build()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks = _peaks()
+    lay = synth.workloads()[WORKLOAD].layers[0]
+    N, K, bpw = lay.N, lay.K, lay.bpw
+    M = args.M
+    cb = e8.Codebook(local)
+    # every rank quantises its own layer (weak scaling); rank 0 is the seeded workload
+    W = synth.gaussian_weights(N, K, lay.std, lay.w_seed if rank == 0 else (lay.w_seed, rank))
+    s = synth.suggest_scale(W, bpw)
+    rs = lay.rht_seed + 7919 * rank
+    Wd = torch.from_numpy(W).to(dev)
+    i1, i2 = e8.e8_encode(cb, Wd, bpw, rs, s)
+    torch.cuda.synchronize()
+    codes = [(i1, i2)] + [(i1.clone(), i2.clone()) for _ in range(ROTATE - 1)]
+    Xh = synth.activations_bf16(M, K, synth.workloads()[WORKLOAD].x_seed)
+    X = torch.from_numpy(Xh.view(np.int16)).to(dev).view(torch.bfloat16)
+    Y = torch.empty((M, N), dtype=torch.float32, device=dev)
+    mode = e8.e8_gemm_auto_mode(M, N, K, bpw)
+    wsb = torch.empty(max(16, e8.e8_workspace_bytes(mode, M, N, K, bpw)), dtype=torch.uint8,
+                      device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(i, M=M, X=X, Y=Y, wsb=wsb, mode=mode):
+        c1, c2 = codes[i % ROTATE]
+        e8.e8_gemm(cb, X, c1, c2, N, K, bpw, rs, s, mode=mode, Y=Y, workspace=wsb, stream=stream)
+
+    if args.profile:
+        # a few eager steps of the headline kernel pair, for ncu captures
+        for i in range(8):
+            step(i)
+        torch.cuda.synchronize()
+        print("profile steps done", flush=True)
+        cb.free()
+        return
+    sampler = ClockSampler(local)
+    if rank == 0:
+        sampler.start()
+    # load phase right before the timed region, for the clock record only
+    t_load = time.time()
+    if not args.no_load:
+        _time_graphs(step, 20 * GRAPH_STEPS, 0, stream)
+    _barrier(ws)
+    torch.cuda.synchronize()
+    t0 = time.time()
+    ms = _time_graphs(step, args.steps, args.warmup, stream)
+    t1 = time.time()
+    torch.cuda.synchronize()
+    _barrier(ws)
+    ms = _max_over_ranks(ms, ws, dev)
+    clocks = sampler.summary(t0, t1, fallback_t0=t_load) if rank == 0 else None
+
+    flop_step = 2.0 * M * N * K
+    sec = ms / 1e3
+    value = flop_step * args.steps * ws / sec / 1e12
+    step_us = ms * 1e3 / args.steps
+    code_bytes = N * K * bpw // 8
+    alg_bytes = code_bytes + M * K * 2 + M * N * 4
+
+    # dominant kernel alone: fused decode-GEMM on pre-transformed activations
+    rows = e8.e8_gemm_xt_rows(M)
+    Xt = e8.e8_act_rht(X, rs, rows=rows)
+
+    def gemm_only(i, M=M, Xt=Xt, Y=Y):
+        c1, c2 = codes[i % ROTATE]
+        e8.e8_gemm_xt(cb, Xt, M, c1, c2, N, K, bpw, s, Y=Y, stream=stream)
+
+    kern_steps = min(args.steps, 20 * GRAPH_STEPS)
+    k_ms = _time_graphs(gemm_only, kern_steps, args.warmup, stream)
+    k_us = k_ms * 1e3 / kern_steps
+    achieved = alg_bytes / (k_us * 1e-6) / 1e9
+
+    def rht_only(i, X=X, Xt=Xt):
+        e8.e8_act_rht(X, rs, rows=rows, out=Xt, stream=stream)
+
+    r_ms = _time_graphs(rht_only, kern_steps, args.warmup, stream)
+    rht_us = r_ms * 1e3 / kern_steps
+
+    # end to end through the public API with host buffers
+    Xpin = torch.from_numpy(Xh.view(np.int16)).view(torch.bfloat16).pin_memory()
+    Ypin = torch.empty((M, N), dtype=torch.float32).pin_memory()
+    Xe = torch.empty_like(X)
+    e2e_steps = min(args.steps, 2000)
+    with torch.cuda.stream(stream):
+        for i in range(max(3, min(args.warmup, 50))):
+            Xe.copy_(Xpin, non_blocking=True)
+            step(i)
+            Ypin.copy_(Y, non_blocking=True)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(e2e_steps):
+            Xe.copy_(Xpin, non_blocking=True)
+            c1, c2 = codes[i % ROTATE]
+            e8.e8_gemm(cb, Xe, c1, c2, N, K, bpw, rs, s, mode=mode, Y=Y, workspace=wsb,
+                       stream=stream)
+            Ypin.copy_(Y, non_blocking=True)
+        b.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = _max_over_ranks(a.elapsed_time(b), ws, dev)
+    e2e_val = flop_step * e2e_steps * ws / (e2e_ms / 1e3) / 1e12
+
+    rows_out = {}
+    if rank == 0 and not args.quick:
+        rows_out = _other_rows(e8, synth, cb, Wd, W, codes, X, N, K, bpw, rs, s, dev, stream, args,
+                               peaks)
+    if rank == 0:
+        launches = 2 * args.steps
+        traffic = _traffic_from_profile()
+        out = {
+            "metric": METRIC,
+            "value": round(value, 3),
+            "unit": "TFLOP/s",
+            "n_gpus": ws,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": step_us / 1e3,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic",
+            "config": {
+                "workload": "%s: W %dx%d N(0,%.2f^2) seed %d, %d bpw, X %dx%d bf16 N(0,1) seed %d"
+                            % (WORKLOAD, N, K, lay.std, lay.w_seed, bpw, M, K,
+                               synth.workloads()[WORKLOAD].x_seed),
+                "M": M, "N": N, "K": K, "bpw": bpw, "gemm_mode": "act_rht (fused, TMEM operand)",
+                "l2": "inputs larger than L2: %d rotating code sets, %.0f MB" %
+                      (ROTATE, ROTATE * code_bytes / 1e6),
+                "launch": "CUDA graphs of %d steps" % GRAPH_STEPS,
+                "parallelism": "independent layer per GPU" if ws > 1 else "single GPU",
+            },
+            "decoded_weights_per_s": N * K * args.steps * ws / sec,
+            "roofline": {
+                "bound": "hbm",
+                "kernel": "k_act_gemm (fused decode + tcgen05 GEMM)",
+                "achieved": round(achieved, 1),
+                "peak": peaks["hbm_gbs"],
+                "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": traffic,
+                "algorithmic_bytes": alg_bytes,
+                "kernel_us": round(k_us, 3),
+                "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs)",
+                "step_frac": round(alg_bytes / (step_us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
+                "act_rht_us": round(rht_us, 3),
+            },
+            "e2e": {"value": round(e2e_val, 3), "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 4,
+                    "steps": e2e_steps, "path": "pinned host X -> e8_gemm -> pinned host Y"},
+            "gpu_launches": launches,
+            "clocks": clocks,
+            "rows": rows_out,
+        }
+        if not args.no_cpu:
+            out["cpu_baseline"] = _cpu_baseline(M)
+        sampler.stop()
+        print(json.dumps(out), flush=True)
+    cb.free()
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def _traffic_from_profile():
+    """DRAM bytes per launch of k_act_gemm from the committed ncu summary, or None
+    when the kernel source changed since the counters were taken."""
+    import hashlib
+    prof = os.path.join(ROOT, "profiles", "k_act_gemm_llama4096_m16.md")
+    src = os.path.join(ROOT, "decode_gemm_e8_b200", "csrc", "e8_gemm_act.cu")
+    if not os.path.exists(prof):
+        return None
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    text = open(prof).read()
+    import re
+    m_h = re.search(r"source sha256\[:16\]: ([0-9a-f]{16})", text)
+    m_t = re.search(r"dram bytes per launch: ([0-9]+)", text)
+    if not m_h or not m_t or m_h.group(1) != h:
+        return None
+    return int(m_t.group(1))
+
+
+def _other_rows(e8, synth, cb, Wd, W, codes, X, N, K, bpw, rs, s, dev, stream, args, peaks):
+    """Encode, decode-to-bf16 and the 1- and 4-token GEMM on the same layer."""
+    import torch
+    rows = {}
+    reps = 4
+    # encode: rotate over copies of W so the 64 MB matrix is read from HBM
+    Ws = [Wd] + [Wd.clone() for _ in range(reps - 1)]
+    wsb = torch.empty(e8.e8_workspace_bytes(e8.E8_OP_ENCODE, 0, N, K, bpw), dtype=torch.uint8,
+                      device=dev)
+    i1 = torch.empty((N, K // 8), dtype=torch.uint16, device=dev)
+    i2 = torch.empty((N, K // 8), dtype=torch.uint16, device=dev)
+    n_enc = 8
+
+    def enc(i):
+        e8.e8_encode(cb, Ws[i % reps], bpw, rs, s, idx1=i1, idx2=i2, workspace=wsb, stream=stream)
+
+    ms = _time_graphs(enc, n_enc, 2, stream)
+    t = ms / 1e3 / n_enc
+    byt = N * K * (4 + bpw / 8)
+    rows["encode"] = {"weights_per_s": N * K / t, "ms": t * 1e3, "GB_s": byt / t / 1e9,
+                      "hbm_frac": round(byt / t / 1e9 / peaks["hbm_gbs"], 4),
+                      "bytes_per_weight": 4 + bpw / 8}
+    out = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+
+    def dec(i):
+        c1, c2 = codes[i % len(codes)]
+        e8.e8_decode_to_bf16(cb, c1, c2, N, K, bpw, rs, s, out=out, stream=stream)
+
+    ms = _time_graphs(dec, 200, 10, stream)
+    t = ms / 1e3 / 200
+    byt = N * K * (2 + bpw / 8)
+    rows["decode_to_bf16"] = {"weights_per_s": N * K / t, "us": t * 1e6, "GB_s": byt / t / 1e9,
+                              "hbm_frac": round(byt / t / 1e9 / peaks["hbm_gbs"], 4),
+                              "bytes_per_weight": 2 + bpw / 8}
+    for Mx in (1, 4):
+        Xm = X[:Mx].contiguous()
+        Ym = torch.empty((Mx, N), dtype=torch.float32, device=dev)
+        mode = e8.e8_gemm_auto_mode(Mx, N, K, bpw)
+        wsm = torch.empty(max(16, e8.e8_workspace_bytes(mode, Mx, N, K, bpw)), dtype=torch.uint8,
+                          device=dev)
+
+        def g(i, Xm=Xm, Ym=Ym, wsm=wsm, mode=mode):
+            c1, c2 = codes[i % len(codes)]
+            e8.e8_gemm(cb, Xm, c1, c2, N, K, bpw, rs, s, mode=mode, Y=Ym, workspace=wsm,
+                       stream=stream)
+
+        ms = _time_graphs(g, 2000, 100, stream)
+        t = ms / 1e3 / 2000
+        byt = N * K * bpw // 8 + Mx * K * 2 + Mx * N * 4
+        rows["gemm_m%d" % Mx] = {"TFLOP_s": 2.0 * Mx * N * K / t / 1e12, "us": t * 1e6,
+                                 "hbm_frac": round(byt / t / 1e9 / peaks["hbm_gbs"], 4)}
+    return rows
+
+
+def _cpu_baseline(M):
+    """The CPU oracle (decode + binary64 GEMM) on the same workload, this host's cores."""
+    from decode_gemm_e8_b200 import synth
+    from oracle import oracle as orc
+    lay = synth.workloads()[WORKLOAD].layers[0]
+    N, K, bpw = lay.N, lay.K, lay.bpw
+    rng = np.random.default_rng(0)
+    i1 = rng.integers(0, 65536, (N, K // 8)).astype(np.uint16)
+    i2 = rng.integers(0, 65536, (N, K // 8)).astype(np.uint16)
+    X = synth.activations_bf16(M, K, synth.workloads()[WORKLOAD].x_seed)
+    threads = orc.threads()
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        wd = orc.decode(i1, i2, N, K, bpw, lay.rht_seed, 0.02)
+        orc.gemm(X, wd)
+        n += 1
+        if time.perf_counter() - t0 > 10.0:
+            break
+    dt = (time.perf_counter() - t0) / n
+    return {"value": 2.0 * M * N * K / dt / 1e12, "unit": "TFLOP/s", "cores": threads,
+            "kind": "oracle",
+            "sample": "whole step of the workload (decode 4096x4096 at 4 bpw + binary64 GEMM with "
+                      "%d rows), repeated %d times over %.1f s; codes random" % (M, n, dt * n)}
+
+
+# -------------------------------------------------------- reference arm ----
+def run_reference(args):
+    ws, rank, _ = _dist()
+    if rank != 0:
+        return
+    from decode_gemm_e8_b200 import synth
+    from oracle import oracle as orc
+    lay = synth.workloads()[WORKLOAD].layers[0]
+    N, K, bpw, M = lay.N, lay.K, lay.bpw, args.M
+    rng = np.random.default_rng(0)
+    i1 = rng.integers(0, 65536, (N, K // 8)).astype(np.uint16)
+    i2 = rng.integers(0, 65536, (N, K // 8)).astype(np.uint16)
+    X = synth.activations_bf16(M, K, synth.workloads()[WORKLOAD].x_seed)
+    # bounded sample: each step decodes and multiplies a slice of the rows
+    rows = max(64, min(N, 4096))
+    steps, warm = min(args.steps, 20), min(args.warmup, 3)
+
+    def one():
+        wd = orc.decode(i1[:rows], i2[:rows], rows, K, bpw, lay.rht_seed, 0.02)
+        orc.gemm(X, wd)
+
+    for _ in range(warm):
+        one()
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        one()
+    dt = (time.perf_counter() - t0) / steps
+    v = 2.0 * M * rows * K / dt / 1e12
+    out = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": ws,
+           "steps": steps, "warmup": warm, "ms_per_step": dt * 1e3, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": "%s: decode %dx%d at %d bpw + GEMM with %d tokens" %
+                                  (WORKLOAD, rows, K, bpw, M), "M": M, "N": rows, "K": K},
+           "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": orc.threads(),
+                            "kind": "oracle", "sample": "%d weight rows per step" % rows},
+           "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200000)
+    ap.add_argument("--warmup", type=int, default=2000)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--M", type=int, default=M_HEAD)
+    ap.add_argument("--quick", action="store_true", help="skip the extra rows")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--no-load", action="store_true",
+                    help="skip the load phase that precedes the timed region (clock record)")
+    ap.add_argument("--profile", action="store_true",
+                    help="run 8 eager steps of the headline call and exit (ncu captures)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -26,7 +26,8 @@ E8_OP_ENCODE = 100
 
 # every symbol include/e8.h declares
 EXPORTED = ("e8_codebook_build", "e8_codebook_free", "e8_codebook_export", "e8_rht_forward",
-            "e8_encode", "e8_decode_to_bf16", "e8_act_rht", "e8_gemm", "e8_gemm_auto_mode",
+            "e8_encode", "e8_decode_to_bf16", "e8_act_rht", "e8_gemm", "e8_gemm_xt",
+            "e8_gemm_xt_rows", "e8_gemm_auto_mode",
             "e8_workspace_bytes", "e8_sync_status", "e8_debug_wait_timeout", "e8_status_str",
             "e8_version")
 
@@ -59,6 +60,9 @@ def load_library(path: str = LIB_PATH):
         "e8_act_rht": ([P, I64, I64, U64, P, I64, P], c.c_int),
         "e8_gemm": ([P, P, I64, P, P, I64, I64, c.c_int, U64, c.c_float, P, c.c_int, P,
                      c.c_size_t, P], c.c_int),
+        "e8_gemm_xt": ([P, P, I64, I64, P, P, I64, I64, c.c_int, c.c_float, P, c.c_int, P],
+                       c.c_int),
+        "e8_gemm_xt_rows": ([I64], c.c_int),
         "e8_gemm_auto_mode": ([I64, I64, I64, c.c_int], c.c_int),
         "e8_workspace_bytes": ([c.c_int, I64, I64, I64, c.c_int], c.c_size_t),
         "e8_sync_status": ([P, P], c.c_int),
@@ -219,6 +223,22 @@ def e8_gemm(cb: Codebook, X, idx1, idx2, N: int, K: int, bpw: int, rht_seed: int
     _check(load_library().e8_gemm(cb.handle, _ptr(X), M, _ptr(idx1), _ptr(idx2), N, K, int(bpw),
                                   int(rht_seed) & (2**64 - 1), float(scale), _ptr(Y), int(mode),
                                   _ptr(ws), ws.numel(), _stream(stream)), "e8_gemm")
+    return Y
+
+
+def e8_gemm_xt_rows(M: int) -> int:
+    return int(load_library().e8_gemm_xt_rows(int(M)))
+
+
+def e8_gemm_xt(cb: Codebook, Xt, M: int, idx1, idx2, N: int, K: int, bpw: int, scale: float,
+               mode: int = E8_GEMM_ACT_RHT, Y=None, stream=None):
+    """Fused decode-GEMM on activations already transformed by e8_act_rht."""
+    import torch
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float32, device=Xt.device)
+    _check(load_library().e8_gemm_xt(cb.handle, _ptr(Xt), Xt.shape[0], int(M), _ptr(idx1),
+                                     _ptr(idx2), int(N), int(K), int(bpw), float(scale), _ptr(Y),
+                                     int(mode), _stream(stream)), "e8_gemm_xt")
     return Y
 
 

@@ -14,8 +14,19 @@ namespace e8 {
 
 __global__ void __launch_bounds__(256) k_act_rht(const uint16_t* __restrict__ X, int64_t M,
                                                  int64_t K, int nh, int elems_per_cta,
-                                                 uint64_t seed, uint16_t* __restrict__ Xt) {
+                                                 uint64_t seed, uint16_t* __restrict__ Xt,
+                                                 int64_t data_ctas, int64_t pad_elems) {
   extern __shared__ __align__(16) float s_x[];
+  if ((int64_t)blockIdx.x >= data_ctas) {
+    // trailing CTAs zero the padding rows 2M..rows-1 (16-byte stores)
+    uint4* pad = reinterpret_cast<uint4*>(Xt + 2 * M * K);
+    const int64_t n16 = pad_elems / 8;
+    const int64_t nct = (int64_t)gridDim.x - data_ctas;
+    for (int64_t i = ((int64_t)blockIdx.x - data_ctas) * blockDim.x + threadIdx.x; i < n16;
+         i += nct * blockDim.x)
+      pad[i] = make_uint4(0u, 0u, 0u, 0u);
+    return;
+  }
   const int64_t total = M * K;
   const int64_t base = (int64_t)blockIdx.x * elems_per_cta;
   const int E = (int)(int64_t)min((long long)elems_per_cta, (long long)(total - base));
@@ -88,14 +99,12 @@ cudaError_t launch_act_rht(const uint16_t* X, int64_t M, int64_t K, uint64_t see
   const int64_t total = M * K;
   const int64_t ctas = (total + epc - 1) / epc;
   const size_t smem = (size_t)epc * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(k_act_rht, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  cudaError_t e = ensure_smem_limit(k_act_rht, kMaxDynSmem);
   if (e != cudaSuccess) return e;
-  if (rows > 2 * M) {
-    e = cudaMemsetAsync(Xt + 2 * M * K, 0, (size_t)(rows - 2 * M) * K * sizeof(uint16_t), st);
-    if (e != cudaSuccess) return e;
-  }
-  k_act_rht<<<(unsigned)ctas, 256, smem, st>>>(X, M, K, nh, epc, seed, Xt);
+  const int64_t pad_elems = (rows - 2 * M) * K;  // multiple of 8 since K is
+  const int64_t pad_ctas = pad_elems > 0 ? (pad_elems / 8 + 2047) / 2048 : 0;
+  k_act_rht<<<(unsigned)(ctas + pad_ctas), 256, smem, st>>>(X, M, K, nh, epc, seed, Xt, ctas,
+                                                            pad_elems);
   return cudaGetLastError();
 }
 

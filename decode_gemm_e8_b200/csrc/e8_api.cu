@@ -4,6 +4,8 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <utility>
+#include <vector>
 
 #include "e8.h"
 #include "e8_common.cuh"
@@ -20,6 +22,24 @@ struct e8_codebook {
   uint32_t* status;
   int max_probe;
 };
+
+namespace e8 {
+
+cudaError_t ensure_smem_limit_ptr(const void* kernel, int bytes) {
+  static std::mutex mu;
+  static std::vector<std::pair<const void*, int>> done;  // (kernel, device)
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const auto& d : done)
+    if (d.first == kernel && d.second == dev) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.emplace_back(kernel, dev);
+  return e;
+}
+
+}  // namespace e8
 
 namespace {
 
@@ -166,6 +186,7 @@ int e8_codebook_export(const e8_codebook* cb, int8_t* host_vecs) {
 
 int e8_rht_forward(const e8_codebook* cb, const float* W, int64_t N, int64_t K,
                    uint64_t rht_seed, float scale, float* U, void* stream) {
+  (void)cudaGetLastError();  // a failed earlier launch must not be reported here
   int rc = check_device(cb);
   if (rc != E8_OK) return rc;
   if (N < 0 || !valid_k(K) || !(scale > 0.0f) || !std::isfinite(scale)) return E8_EINVAL;
@@ -207,6 +228,7 @@ int e8_gemm_auto_mode(int64_t M, int64_t N, int64_t K, int bpw) {
 int e8_encode(const e8_codebook* cb, const float* W, int64_t N, int64_t K, int bpw,
               uint64_t rht_seed, float scale, uint16_t* idx1, void* idx2, void* workspace,
               size_t ws_bytes, void* stream) {
+  (void)cudaGetLastError();  // a failed earlier launch must not be reported here
   int rc = check_device(cb);
   if (rc != E8_OK) return rc;
   if (N < 0 || !valid_k(K) || !valid_bpw(bpw) || !(scale > 0.0f) || !std::isfinite(scale))
@@ -231,6 +253,7 @@ int e8_encode(const e8_codebook* cb, const float* W, int64_t N, int64_t K, int b
 int e8_decode_to_bf16(const e8_codebook* cb, const uint16_t* idx1, const void* idx2, int64_t N,
                       int64_t K, int bpw, uint64_t rht_seed, float scale, uint16_t* W_dec,
                       void* stream) {
+  (void)cudaGetLastError();  // a failed earlier launch must not be reported here
   int rc = check_device(cb);
   if (rc != E8_OK) return rc;
   if (N < 0 || !valid_k(K) || !valid_bpw(bpw) || !(scale > 0.0f) || !std::isfinite(scale))
@@ -247,6 +270,7 @@ int e8_decode_to_bf16(const e8_codebook* cb, const uint16_t* idx1, const void* i
 
 int e8_act_rht(const uint16_t* X, int64_t M, int64_t K, uint64_t rht_seed, uint16_t* Xt,
                int64_t rows, void* stream) {
+  (void)cudaGetLastError();  // a failed earlier launch must not be reported here
   if (M < 0 || !valid_k(K) || rows < 2 * M) return E8_EINVAL;
   if (M == 0) return E8_OK;
   if (!X || !Xt || !aligned16(X) || !aligned16(Xt)) return E8_EINVAL;
@@ -256,6 +280,7 @@ int e8_act_rht(const uint16_t* X, int64_t M, int64_t K, uint64_t rht_seed, uint1
 int e8_gemm(const e8_codebook* cb, const uint16_t* X, int64_t M, const uint16_t* idx1,
             const void* idx2, int64_t N, int64_t K, int bpw, uint64_t rht_seed, float scale,
             float* Y, int mode, void* workspace, size_t ws_bytes, void* stream) {
+  (void)cudaGetLastError();  // a failed earlier launch must not be reported here
   int rc = check_device(cb);
   if (rc != E8_OK) return rc;
   if (M < 0 || N < 0 || !valid_k(K) || !valid_bpw(bpw) || !(scale > 0.0f) ||
@@ -308,6 +333,41 @@ int e8_gemm(const e8_codebook* cb, const uint16_t* X, int64_t M, const uint16_t*
   return cuda_status(e);
 }
 
+int e8_gemm_xt(const e8_codebook* cb, const uint16_t* Xt, int64_t rows, int64_t M,
+               const uint16_t* idx1, const void* idx2, int64_t N, int64_t K, int bpw,
+               float scale, float* Y, int mode, void* stream) {
+  (void)cudaGetLastError();  // a failed earlier launch must not be reported here
+  int rc = check_device(cb);
+  if (rc != E8_OK) return rc;
+  if (M < 0 || N < 0 || !valid_k(K) || !valid_bpw(bpw) || !(scale > 0.0f) ||
+      !std::isfinite(scale))
+    return E8_EINVAL;
+  if ((bpw == 2) != (idx2 == nullptr)) return E8_EINVAL;
+  if (mode == E8_GEMM_AUTO) mode = E8_GEMM_ACT_RHT;
+  if (mode != E8_GEMM_ACT_RHT && mode != E8_GEMM_ACT_RHT_SMEM) return E8_EINVAL;
+  if (M > 64 || (K % 128) != 0 || N > INT32_MAX || K > INT32_MAX) return E8_EINVAL;
+  if (M == 0 || N == 0) return E8_OK;
+  if (rows != rows_b_for(M)) return E8_EINVAL;
+  if (!Xt || !idx1 || !Y || !aligned16(Xt) || !aligned16(idx1) || !aligned16(Y) ||
+      (idx2 && !aligned16(idx2)))
+    return E8_EINVAL;
+  e8::ActGemmArgs a;
+  a.Xt = Xt;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.rows_b = (int)rows;
+  a.idx1 = idx1;
+  a.idx2 = idx2;
+  a.bpw = bpw;
+  a.alpha = alpha_of(scale, e8::hadamard_block(K), bpw);
+  a.Y = Y;
+  a.variant = mode == E8_GEMM_ACT_RHT ? 1 : 0;
+  return cuda_status(e8::launch_act_gemm(dev_view(cb), a, cb->sm_count, (cudaStream_t)stream));
+}
+
+int e8_gemm_xt_rows(int64_t M) { return M < 0 ? 0 : rows_b_for(M); }
+
 int e8_sync_status(const e8_codebook* cb, void* stream) {
   int rc = check_device(cb);
   if (rc != E8_OK) return rc;
@@ -323,6 +383,7 @@ int e8_sync_status(const e8_codebook* cb, void* stream) {
 }
 
 int e8_debug_wait_timeout(const e8_codebook* cb, int wait_ms, void* stream) {
+  (void)cudaGetLastError();  // a failed earlier launch must not be reported here
   int rc = check_device(cb);
   if (rc != E8_OK) return rc;
   if (wait_ms < 1 || wait_ms > 5000) return E8_EINVAL;

@@ -272,6 +272,16 @@ __device__ __forceinline__ float bf16_hi_to_f32(uint32_t v) {
   return __uint_as_float(v & 0xFFFF0000u);
 }
 
+// Raises a kernel's dynamic shared-memory limit once per (kernel, device) on
+// the host.  Done on first use rather than per launch so that launches can be
+// captured into CUDA graphs without any non-stream API call in between.
+cudaError_t ensure_smem_limit_ptr(const void* kernel, int bytes);
+template <class Kernel>
+inline cudaError_t ensure_smem_limit(Kernel* k, int bytes) {
+  return ensure_smem_limit_ptr(reinterpret_cast<const void*>(k), bytes);
+}
+constexpr int kMaxDynSmem = 232448;   // 227 KB per block on sm_100
+
 // Hadamard block of a row of length K: largest power of two dividing K.
 __host__ __device__ __forceinline__ int64_t hadamard_block(int64_t K) {
   return K & (-K);

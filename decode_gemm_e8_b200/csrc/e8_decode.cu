@@ -131,8 +131,7 @@ cudaError_t launch_decode(const DeviceCodebook& cb, const uint16_t* idx1, const 
   const int64_t total = N * K;
   const int64_t ctas = (total + p.elems_per_cta - 1) / p.elems_per_cta;
   const size_t smem = (size_t)p.elems_per_cta * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(k_decode, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  cudaError_t e = ensure_smem_limit(k_decode, kMaxDynSmem);
   if (e != cudaSuccess) return e;
   k_decode<<<(unsigned)ctas, 256, smem, st>>>(p, cb);
   return cudaGetLastError();

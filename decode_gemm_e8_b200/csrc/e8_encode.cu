@@ -415,8 +415,7 @@ cudaError_t launch_encode(const DeviceCodebook& cb, const float* W, int64_t N, i
   const int64_t total = N * K;
   const int64_t ctas = (total + p.elems_per_cta - 1) / p.elems_per_cta;
   const size_t smem = (size_t)p.elems_per_cta * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(k_encode, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  cudaError_t e = ensure_smem_limit(k_encode, kMaxDynSmem);
   if (e != cudaSuccess) return e;
   if (do_quantise) {
     e = cudaMemsetAsync(work_count, 0, sizeof(uint32_t), st);

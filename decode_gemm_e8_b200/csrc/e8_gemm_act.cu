@@ -361,14 +361,12 @@ cudaError_t launch_act_gemm(const DeviceCodebook& cb, const ActGemmArgs& a, int 
   cfg.numAttrs = 1;
   cudaError_t e;
   if (tm) {
-    e = cudaFuncSetAttribute(k_act_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             plan.total);
+    e = ensure_smem_limit(k_act_gemm<true>, kMaxDynSmem);
     if (e != cudaSuccess) return e;
     e = cudaLaunchKernelEx(&cfg, k_act_gemm<true>, tb, ti1, ti2, cb, (int)a.M, (int)a.N, (int)a.K,
                            a.rows_b, a.bpw, a.alpha, a.Y);
   } else {
-    e = cudaFuncSetAttribute(k_act_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             plan.total);
+    e = ensure_smem_limit(k_act_gemm<false>, kMaxDynSmem);
     if (e != cudaSuccess) return e;
     e = cudaLaunchKernelEx(&cfg, k_act_gemm<false>, tb, ti1, ti2, cb, (int)a.M, (int)a.N,
                            (int)a.K, a.rows_b, a.bpw, a.alpha, a.Y);

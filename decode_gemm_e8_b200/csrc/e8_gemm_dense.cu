@@ -201,8 +201,7 @@ cudaError_t launch_dense_gemm(const uint16_t* X, int64_t M, const uint16_t* W, i
   if (!make_tmap_2d(&tb, W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)N, (uint64_t)K, BN, BK,
                     CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(k_dense_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)SMEM_BYTES);
+  cudaError_t e = ensure_smem_limit(k_dense_gemm, kMaxDynSmem);
   if (e != cudaSuccess) return e;
   const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   const int grid = (int)(tiles < sm_count ? tiles : sm_count);

@@ -135,6 +135,20 @@ int e8_gemm(const e8_codebook* cb, const uint16_t* X, int64_t M, const uint16_t*
             const void* idx2, int64_t N, int64_t K, int bpw, uint64_t rht_seed, float scale,
             float* Y, int mode, void* workspace, size_t ws_bytes, void* stream);
 
+/* Second half of E8_GEMM_ACT_RHT on activations already transformed by
+ * e8_act_rht: Y fp32 [M][N] = alpha * (Xt[0:M] + Xt[M:2M]) * Z^T, with Z the
+ * integer codebook vectors decoded on chip and alpha from `scale`.  Xt is bf16
+ * [rows][K] with rows == e8_gemm_xt_rows(M) (2M rounded up to a multiple of
+ * 16; padding rows must be zero, as e8_act_rht leaves them).  One transform can
+ * serve every weight matrix that shares K and rht_seed.  mode: E8_GEMM_ACT_RHT
+ * (or AUTO) or E8_GEMM_ACT_RHT_SMEM; M <= 64, K % 128 == 0.  No workspace. */
+int e8_gemm_xt(const e8_codebook* cb, const uint16_t* Xt, int64_t rows, int64_t M,
+               const uint16_t* idx1, const void* idx2, int64_t N, int64_t K, int bpw,
+               float scale, float* Y, int mode, void* stream);
+
+/* Row count of the transformed-activation buffer for M tokens (see e8_gemm_xt). */
+int e8_gemm_xt_rows(int64_t M);
+
 /* Mode that E8_GEMM_AUTO selects for these sizes. */
 int e8_gemm_auto_mode(int64_t M, int64_t N, int64_t K, int bpw);
 

@@ -149,3 +149,37 @@ def test_act_gemm_is_deterministic(gcb):
                             mode=e8.E8_GEMM_ACT_RHT))
     assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
     assert e8.e8_sync_status(gcb) == e8.E8_OK
+
+
+def test_gemm_xt_matches_gemm_and_graph_capture(gcb):
+    import torch
+    wl = synth.workloads()["llama_4096_b4"]
+    lay = wl.layers[0]
+    W = lay.weights()
+    s = synth.suggest_scale(W, lay.bpw)
+    X = gu.bf16_dev(synth.activations_bf16(16, lay.K, wl.x_seed))
+    i1, i2 = _layer_codes(gcb, W, lay.bpw, lay.rht_seed, s)
+    a = e8.e8_gemm(gcb, X, i1, i2, lay.N, lay.K, lay.bpw, lay.rht_seed, s,
+                   mode=e8.E8_GEMM_ACT_RHT)
+    rows = e8.e8_gemm_xt_rows(16)
+    assert rows == 32
+    Xt = e8.e8_act_rht(X, lay.rht_seed, rows=rows)
+    b = e8.e8_gemm_xt(gcb, Xt, 16, i1, i2, lay.N, lay.K, lay.bpw, s)
+    assert np.array_equal(gu.to_np(a).view(np.uint32), gu.to_np(b).view(np.uint32))
+    # the same call captured in a CUDA graph and replayed
+    Y = torch.empty_like(a)
+    ws = torch.empty(e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT, 16, lay.N, lay.K, lay.bpw),
+                     dtype=torch.uint8, device=X.device)
+    st = torch.cuda.Stream()
+    e8.e8_gemm(gcb, X, i1, i2, lay.N, lay.K, lay.bpw, lay.rht_seed, s, mode=e8.E8_GEMM_ACT_RHT,
+               Y=Y, workspace=ws, stream=st)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=st):
+        e8.e8_gemm(gcb, X, i1, i2, lay.N, lay.K, lay.bpw, lay.rht_seed, s,
+                   mode=e8.E8_GEMM_ACT_RHT, Y=Y, workspace=ws, stream=st)
+    Y.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert np.array_equal(gu.to_np(Y).view(np.uint32), gu.to_np(a).view(np.uint32))
+    assert e8.e8_sync_status(gcb) == e8.E8_OK
