@@ -4,8 +4,6 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
-#include <utility>
-#include <vector>
 
 #include "e8.h"
 #include "e8_common.cuh"
@@ -26,16 +24,24 @@ struct e8_codebook {
 namespace e8 {
 
 cudaError_t ensure_smem_limit_ptr(const void* kernel, int bytes) {
+  // fixed table, no heap use on any launch path
+  constexpr int kSlots = 256;
   static std::mutex mu;
-  static std::vector<std::pair<const void*, int>> done;  // (kernel, device)
+  static const void* kern[kSlots];
+  static int devs[kSlots];
+  static int used = 0;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> lock(mu);
-  for (const auto& d : done)
-    if (d.first == kernel && d.second == dev) return cudaSuccess;
+  for (int i = 0; i < used; ++i)
+    if (kern[i] == kernel && devs[i] == dev) return cudaSuccess;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess) done.emplace_back(kernel, dev);
+  if (e == cudaSuccess && used < kSlots) {
+    kern[used] = kernel;
+    devs[used] = dev;
+    ++used;
+  }
   return e;
 }
 
