@@ -27,7 +27,7 @@ E8_OP_ENCODE = 100
 # every symbol include/e8.h declares
 EXPORTED = ("e8_codebook_build", "e8_codebook_free", "e8_codebook_export", "e8_rht_forward",
             "e8_encode", "e8_decode_to_bf16", "e8_act_rht", "e8_gemm", "e8_gemm_xt",
-            "e8_gemm_xt_rows", "e8_gemm_auto_mode",
+            "e8_gemm_xt_rows", "e8_gemm_act_noalloc", "e8_gemm_auto_mode",
             "e8_workspace_bytes", "e8_sync_status", "e8_debug_wait_timeout", "e8_status_str",
             "e8_version")
 
@@ -63,6 +63,8 @@ def load_library(path: str = LIB_PATH):
         "e8_gemm_xt": ([P, P, I64, I64, P, P, I64, I64, c.c_int, c.c_float, P, c.c_int, P],
                        c.c_int),
         "e8_gemm_xt_rows": ([I64], c.c_int),
+        "e8_gemm_act_noalloc": ([P, P, I64, P, P, I64, I64, c.c_int, U64, c.c_float, P, P],
+                                c.c_int),
         "e8_gemm_auto_mode": ([I64, I64, I64, c.c_int], c.c_int),
         "e8_workspace_bytes": ([c.c_int, I64, I64, I64, c.c_int], c.c_size_t),
         "e8_sync_status": ([P, P], c.c_int),
@@ -239,6 +241,20 @@ def e8_gemm_xt(cb: Codebook, Xt, M: int, idx1, idx2, N: int, K: int, bpw: int, s
     _check(load_library().e8_gemm_xt(cb.handle, _ptr(Xt), Xt.shape[0], int(M), _ptr(idx1),
                                      _ptr(idx2), int(N), int(K), int(bpw), float(scale), _ptr(Y),
                                      int(mode), _stream(stream)), "e8_gemm_xt")
+    return Y
+
+
+def e8_gemm_act_noalloc(cb: Codebook, X, idx1, idx2, N: int, K: int, bpw: int, rht_seed: int,
+                        scale: float, Y, stream=None):
+    """E8_GEMM_ACT_RHT with the library's fixed scratch array instead of a workspace.
+
+    For callers that may not allocate device memory when they run the layer (CUDA
+    graph capture, framework-owned memory, latency-critical loops).  Y must be
+    given: this call allocates nothing."""
+    _check(load_library().e8_gemm_act_noalloc(cb.handle, _ptr(X), X.shape[0], _ptr(idx1),
+                                              _ptr(idx2), int(N), int(K), int(bpw),
+                                              int(rht_seed) & (2**64 - 1), float(scale), _ptr(Y),
+                                              _stream(stream)), "e8_gemm_act_noalloc")
     return Y
 
 

@@ -10,16 +10,6 @@
 #include "e8_codebook.cuh"
 #include "e8_internal.h"
 
-struct e8_codebook {
-  int device;
-  int sm_count;
-  int8_t* vecs;
-  uint32_t* table;
-  uint32_t* hkeys;
-  uint32_t* hvals;
-  uint32_t* status;
-  int max_probe;
-};
 
 namespace e8 {
 

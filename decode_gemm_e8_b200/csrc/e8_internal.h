@@ -6,6 +6,18 @@
 
 #include "e8_codebook.cuh"
 
+// The opaque handle of include/e8.h: device tables of one codebook.
+struct e8_codebook {
+  int device;
+  int sm_count;
+  int8_t* vecs;
+  uint32_t* table;
+  uint32_t* hkeys;
+  uint32_t* hvals;
+  uint32_t* status;
+  int max_probe;
+};
+
 namespace e8 {
 
 // One group that the encoder's fast path could not decide exactly.

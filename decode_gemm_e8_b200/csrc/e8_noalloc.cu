@@ -1,0 +1,109 @@
+// e8_gemm_act_noalloc: the small-batch fused GEMM (E8_GEMM_ACT_RHT) for callers
+// that cannot hand the library a workspace.
+//
+// Some callers are not allowed to allocate device memory at the point where
+// they run the layer: code being captured into a CUDA graph (cudaMalloc is not a
+// capturable call), plugins whose host framework owns every byte of device
+// memory and gives them none at enqueue time, and latency-critical loops where
+// an allocation could synchronise the device.  This entry point keeps its only
+// scratch buffer -- the transformed activations, hi and lo rows -- in a
+// fixed-size array that lives in the library's own device image, so it needs
+// neither a workspace argument nor any allocation.
+//
+// Limits and rules (also stated in include/e8.h):
+//   - the scratch holds kNoallocXtElems bf16 values (2 MiB): rows * K must not
+//     exceed it, where rows = e8_gemm_xt_rows(M); larger requests return
+//     E8_EWORKSPACE without launching anything;
+//   - every GPU that loads the library keeps this 2 MiB until the process exits;
+//   - all calls share the one array and it keeps the last call's contents; the
+//     padding rows that must be zero are cleared by every call, but two calls
+//     whose kernels overlap on the GPU (different streams without ordering)
+//     race on the array and give wrong results;
+//   - the first call on each device looks up the array's device address there
+//     (cudaGetSymbolAddress, with that device current); make that first call
+//     before any stream capture begins.
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "e8.h"
+#include "e8_common.cuh"
+#include "e8_codebook.cuh"
+#include "e8_internal.h"
+
+namespace {
+
+constexpr int64_t kNoallocXtElems = 1 << 20;   // 1 Mi bf16 = 2 MiB
+constexpr int kMaxDevices = 64;
+
+// Device-resident scratch: transformed activations of the last call.
+static __device__ __align__(256) uint16_t g_noalloc_xt[kNoallocXtElems];
+
+std::mutex g_mu;
+void* g_xt_addr[kMaxDevices];   // device address of g_noalloc_xt, per device
+
+// Device address of the scratch array on the current device (looked up once).
+int scratch_address(int dev, uint16_t** out) {
+  if (dev < 0 || dev >= kMaxDevices) return E8_EDEVICE;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_xt_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_xt) != cudaSuccess || !p) return E8_ECUDA;
+    g_xt_addr[dev] = p;
+  }
+  *out = static_cast<uint16_t*>(g_xt_addr[dev]);
+  return E8_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+extern "C" int e8_gemm_act_noalloc(const e8_codebook* cb, const uint16_t* X, int64_t M,
+                                   const uint16_t* idx1, const void* idx2, int64_t N, int64_t K,
+                                   int bpw, uint64_t rht_seed, float scale, float* Y,
+                                   void* stream) {
+  if (!cb) return E8_EINVAL;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return E8_ECUDA;
+  if (dev != cb->device) return E8_EDEVICE;
+  (void)cudaGetLastError();  // an earlier failed launch must not be reported here
+  if (M < 0 || N < 0 || K < 8 || (K % 8) != 0 || bpw < 2 || bpw > 4 || !(scale > 0.0f) ||
+      !std::isfinite(scale))
+    return E8_EINVAL;
+  const int64_t nh = e8::hadamard_block(K);
+  if (nh > 32768) return E8_EINVAL;
+  if ((bpw == 2) != (idx2 == nullptr)) return E8_EINVAL;
+  if (M > 64 || (K % 128) != 0 || N > INT32_MAX || K > INT32_MAX) return E8_EINVAL;
+  if (M == 0 || N == 0) return E8_OK;
+  const int64_t rows = (2 * M + 15) / 16 * 16;
+  if (rows * K > kNoallocXtElems) return E8_EWORKSPACE;
+  if (!X || !idx1 || !Y || !aligned16(X) || !aligned16(idx1) || !aligned16(Y) ||
+      (idx2 && !aligned16(idx2)))
+    return E8_EINVAL;
+  uint16_t* xt = nullptr;
+  int rc = scratch_address(dev, &xt);
+  if (rc != E8_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (e8::launch_act_rht(X, M, K, rht_seed, xt, rows, st) != cudaSuccess) return E8_ECUDA;
+  e8::DeviceCodebook d;
+  d.vecs = cb->vecs;
+  d.table = cb->table;
+  d.hkeys = cb->hkeys;
+  d.hvals = cb->hvals;
+  d.status = cb->status;
+  e8::ActGemmArgs a;
+  a.Xt = xt;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.rows_b = (int)rows;
+  a.idx1 = idx1;
+  a.idx2 = idx2;
+  a.bpw = bpw;
+  const int m = bpw == 2 ? 2 : (bpw == 3 ? 4 : 8);
+  a.alpha = (float)((double)scale / ((double)m * std::sqrt((double)nh)));
+  a.Y = Y;
+  a.variant = 1;
+  return e8::launch_act_gemm(d, a, cb->sm_count, st) == cudaSuccess ? E8_OK : E8_ECUDA;
+}

@@ -149,6 +149,24 @@ int e8_gemm_xt(const e8_codebook* cb, const uint16_t* Xt, int64_t rows, int64_t 
 /* Row count of the transformed-activation buffer for M tokens (see e8_gemm_xt). */
 int e8_gemm_xt_rows(int64_t M);
 
+/* E8_GEMM_ACT_RHT without a workspace, for callers that may not allocate device
+ * memory where they run the layer: code being captured into a CUDA graph,
+ * plugins whose host framework owns all device memory, latency-critical loops
+ * that cannot risk an allocation synchronising the device.  The paper has no
+ * counterpart; this is a deployment convenience of this library.
+ * Same arguments and result as e8_gemm with mode E8_GEMM_ACT_RHT, minus the
+ * workspace.  The transformed activations go to a fixed 2 MiB array compiled
+ * into the library (every GPU that loads the library holds it until the process
+ * exits): requests with e8_gemm_xt_rows(M) * K > 1048576 return E8_EWORKSPACE
+ * and launch nothing.  Nothing is allocated.  All calls share that array and it
+ * keeps the last call's contents (each call clears what must start at zero);
+ * calls whose kernels overlap on the GPU race on it, so order them on one
+ * stream.  The first call on a device looks up the array's address on that
+ * device; make it before any stream capture begins. */
+int e8_gemm_act_noalloc(const e8_codebook* cb, const uint16_t* X, int64_t M,
+                        const uint16_t* idx1, const void* idx2, int64_t N, int64_t K, int bpw,
+                        uint64_t rht_seed, float scale, float* Y, void* stream);
+
 /* Mode that E8_GEMM_AUTO selects for these sizes. */
 int e8_gemm_auto_mode(int64_t M, int64_t N, int64_t K, int bpw);
 
