@@ -5,8 +5,10 @@
 //     y[m][n] = sum_k x_mk w_nk = alpha * sum_k (H D x_m)_k z_nk,
 // so the GEMM can run on the integer codebook vectors z (exact in bf16) once
 // the activations are transformed.  The transformed row xt = FWHT(D x) is
-// split into two bf16 parts, hi = bf16(xt) and lo = bf16(xt - hi), so that the
-// bf16 tensor-core product keeps about 16 significant bits of xt.
+// split into two bf16 parts, hi = bf16(xt) and lo = bf16(xt - hi), stored as
+// rows 2m and 2m + 1, so that the bf16 tensor-core product keeps about 16
+// significant bits of xt and the two parts of a token sit in adjacent
+// accumulator columns.
 #include "e8_common.cuh"
 #include "e8_internal.h"
 
@@ -87,13 +89,148 @@ __global__ void __launch_bounds__(256) k_act_rht(const uint16_t* __restrict__ X,
       float r1 = y[2 * i + 1] - bf16_hi_to_f32(hw[i]);
       lw[i] = pack_bf16x2(r0, r1);
     }
-    *reinterpret_cast<uint4*>(Xt + m * K + k0) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-    *reinterpret_cast<uint4*>(Xt + (M + m) * K + k0) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    *reinterpret_cast<uint4*>(Xt + (2 * m) * K + k0) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    *reinterpret_cast<uint4*>(Xt + (2 * m + 1) * K + k0) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+  }
+}
+
+// Fast path for Hadamard blocks of 256..4096 (others use k_act_rht): one CTA of nh/8 threads per
+// (row, block).  Stages h = 1, 2, 4 inside a thread's group of 8, stages
+// 8..128 by warp shuffles, stages 256..nh/2 after one transpose through shared
+// memory, where 256 threads hold nh/256 elements 256 apart.  Launched with
+// programmatic serialization: it waits for the previous kernel before reading
+// X (and before overwriting Xt, which that kernel may still read), then lets
+// the GEMM that follows start its prologue.
+__global__ void __launch_bounds__(512) k_act_rht_fast(const uint16_t* __restrict__ X, int64_t M,
+                                                      int64_t K, int nh, uint64_t seed,
+                                                      uint16_t* __restrict__ Xt,
+                                                      int64_t data_ctas, int64_t pad_elems) {
+  __shared__ __align__(16) float s_x[4096];
+  grid_dep_wait();
+  grid_dep_launch();
+  if ((int64_t)blockIdx.x >= data_ctas) {
+    uint4* pad = reinterpret_cast<uint4*>(Xt + 2 * M * K);
+    const int64_t n16 = pad_elems / 8;
+    const int64_t nct = (int64_t)gridDim.x - data_ctas;
+    for (int64_t i = ((int64_t)blockIdx.x - data_ctas) * blockDim.x + threadIdx.x; i < n16;
+         i += nct * blockDim.x)
+      pad[i] = make_uint4(0u, 0u, 0u, 0u);
+    return;
+  }
+  const int t = threadIdx.x, lane = t & 31;
+  const int64_t base = (int64_t)blockIdx.x * nh;   // first element of this block
+  const int64_t m = base / K, kb = base % K;
+  // blocks of 512..1024 run 256 threads for the second phase; only nh/8 of
+  // them (whole warps) own a group in the first phase
+  const bool owner = t < (nh >> 3);
+  const int64_t e0 = base + 8 * t;
+  const int64_t k0 = kb + 8 * t;
+  uint4 raw = owner ? __ldg(reinterpret_cast<const uint4*>(X + e0)) : make_uint4(0u, 0u, 0u, 0u);
+  const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
+  float y[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    y[2 * i] = bf16_lo_to_f32(rw[i]);
+    y[2 * i + 1] = bf16_hi_to_f32(rw[i]);
+  }
+  const uint64_t word = splitmix64_output(seed, (uint64_t)(k0 >> 6));
+  const uint32_t bits = (uint32_t)(word >> (k0 & 63));
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    y[i] = __uint_as_float(__float_as_uint(y[i]) ^ (((bits >> i) & 1u) << 31));
+#pragma unroll
+  for (int h = 1; h < 8; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if ((i & h) == 0) {
+        float a = y[i], c = y[i + h];
+        y[i] = a + c;
+        y[i + h] = a - c;
+      }
+    }
+  }
+#pragma unroll
+  for (int h = 8; h < 256; h <<= 1) {
+    const int lm = h >> 3;
+    const bool upper = (lane & lm) != 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float o = __shfl_xor_sync(0xffffffffu, y[i], lm);
+      y[i] = upper ? o - y[i] : y[i] + o;
+    }
+  }
+  if (nh <= 256) {
+    uint32_t hw[4], lw[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      hw[i] = pack_bf16x2(y[2 * i], y[2 * i + 1]);
+      lw[i] = pack_bf16x2(y[2 * i] - bf16_lo_to_f32(hw[i]), y[2 * i + 1] - bf16_hi_to_f32(hw[i]));
+    }
+    *reinterpret_cast<uint4*>(Xt + (2 * m) * K + k0) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    *reinterpret_cast<uint4*>(Xt + (2 * m + 1) * K + k0) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    return;
+  }
+  if (owner) {
+    float4* dst = reinterpret_cast<float4*>(s_x + 8 * t);
+    dst[0] = make_float4(y[0], y[1], y[2], y[3]);
+    dst[1] = make_float4(y[4], y[5], y[6], y[7]);
+  }
+  __syncthreads();
+  if (t >= 256) return;
+  const int per = nh >> 8;   // elements per thread, 256 apart
+  float z[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j)
+    if (j < per) z[j] = s_x[t + 256 * j];
+#pragma unroll
+  for (int h = 1; h < 16; h <<= 1) {
+    if (h >= per) break;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      if (j < per && (j & h) == 0) {
+        float a = z[j], c = z[j + h];
+        z[j] = a + c;
+        z[j + h] = a - c;
+      }
+    }
+  }
+  uint16_t* hi_row = Xt + (2 * m) * K + kb;
+  uint16_t* lo_row = Xt + (2 * m + 1) * K + kb;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    if (j < per) {
+      const uint32_t hb = f32_to_bf16_rne(z[j]);
+      const float rest = z[j] - __uint_as_float(hb << 16);
+      hi_row[t + 256 * j] = (uint16_t)hb;
+      lo_row[t + 256 * j] = (uint16_t)f32_to_bf16_rne(rest);
+    }
   }
 }
 
 cudaError_t launch_act_rht(const uint16_t* X, int64_t M, int64_t K, uint64_t seed, uint16_t* Xt,
-                           int64_t rows, cudaStream_t st) {
+                           int64_t rows, cudaStream_t st, int pdl) {
+  {
+    const int nh = (int)hadamard_block(K);
+    if (nh >= 256 && nh <= 4096) {
+      const int64_t data = M * K / nh;
+      const int64_t pad_elems = (rows - 2 * M) * K;
+      const int64_t pad_ctas = pad_elems > 0 ? (pad_elems / 8 + 4095) / 4096 : 0;
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((unsigned)(data + pad_ctas));
+      cfg.blockDim = dim3((unsigned)(nh <= 256 ? 32 : (nh / 8 < 256 ? 256 : nh / 8)));
+      cfg.dynamicSmemBytes = 0;
+      cfg.stream = st;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      cudaError_t e = cudaLaunchKernelEx(&cfg, k_act_rht_fast, X, M, K, nh, seed, Xt, data,
+                                         pad_elems);
+      if (e != cudaSuccess) return e;
+      return cudaGetLastError();
+    }
+  }
   const int nh = (int)hadamard_block(K);
   const int epc = nh < 2048 ? 2048 : nh;
   const int64_t total = M * K;

@@ -302,7 +302,7 @@ int e8_gemm(const e8_codebook* cb, const uint16_t* X, int64_t M, const uint16_t*
   if (act) {
     const int rows_b = rows_b_for(M);
     uint16_t* Xt = static_cast<uint16_t*>(workspace);
-    e = e8::launch_act_rht(X, M, K, rht_seed, Xt, rows_b, st);
+    e = e8::launch_act_rht(X, M, K, rht_seed, Xt, rows_b, st, 1);
     if (e != cudaSuccess) return E8_ECUDA;
     e8::ActGemmArgs a;
     a.Xt = Xt;
@@ -316,6 +316,8 @@ int e8_gemm(const e8_codebook* cb, const uint16_t* X, int64_t M, const uint16_t*
     a.alpha = alpha;
     a.Y = Y;
     a.variant = mode == E8_GEMM_ACT_RHT ? 1 : 0;
+    a.pdl = 1;          // overlaps the prologue with the transform just launched
+    a.early_codes = 1;  // that transform writes only Xt
     e = e8::launch_act_gemm(d, a, cb->sm_count, st);
     return cuda_status(e);
   }
@@ -359,6 +361,8 @@ int e8_gemm_xt(const e8_codebook* cb, const uint16_t* Xt, int64_t rows, int64_t 
   a.alpha = alpha_of(scale, e8::hadamard_block(K), bpw);
   a.Y = Y;
   a.variant = mode == E8_GEMM_ACT_RHT ? 1 : 0;
+  a.pdl = 1;          // only the library's table is read before the previous kernel ends
+  a.early_codes = 0;  // the previous kernel is the caller's and may write the codes
   return cuda_status(e8::launch_act_gemm(dev_view(cb), a, cb->sm_count, (cudaStream_t)stream));
 }
 

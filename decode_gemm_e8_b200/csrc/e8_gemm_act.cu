@@ -4,9 +4,9 @@
 //
 // z_n = m (c1 + beta c2) is the integer codebook vector of each group of row
 // n ("glq 0.1.1", "How it works", item 1); |z| <= 30 is exact in bf16.  The
-// transformed activations arrive as bf16 hi/lo row pairs (Xt, built by
-// k_act_rht), so one MMA with N = 2M columns computes both parts at once and
-// the epilogue adds them.
+// transformed activations arrive as bf16 hi/lo row pairs (Xt rows 2m and
+// 2m + 1, built by k_act_rht), so one MMA with N = 2M columns computes both
+// parts at once and the epilogue adds adjacent columns.
 //
 // One CTA owns 128 weight rows and a contiguous range of K; the CTAs of a
 // thread-block cluster split K and reduce their partial tiles through
@@ -303,8 +303,8 @@ __global__ void __launch_bounds__(ag::THREADS, 1)
       float acc = 0.0f;
       for (uint32_t src = 0; src < ncl; ++src) {
         const uint32_t base = mapa_shared(part_addr, src);
-        const uint32_t off = (uint32_t)(((r0 + row) * ld + m) * 4);
-        const uint32_t off2 = (uint32_t)(((r0 + row) * ld + M + m) * 4);
+        const uint32_t off = (uint32_t)(((r0 + row) * ld + 2 * m) * 4);
+        const uint32_t off2 = off + 4u;
         acc += ld_shared_cluster_f32(base + off) + ld_shared_cluster_f32(base + off2);
       }
       if (n < N) Y[(size_t)m * N + n] = alpha * acc;
@@ -319,8 +319,8 @@ __global__ void __launch_bounds__(ag::THREADS, 1)
   }
 }
 
-cudaError_t launch_act_gemm(const DeviceCodebook& cb, const ActGemmArgs& a, int sm_count,
-                            cudaStream_t st) {
+static cudaError_t launch_act_gemm_generic(const DeviceCodebook& cb, const ActGemmArgs& a,
+                                           int sm_count, cudaStream_t st) {
   using namespace ag;
   const bool tm = a.variant == 1;
   CUtensorMap tb, ti1, ti2;
@@ -373,6 +373,441 @@ cudaError_t launch_act_gemm(const DeviceCodebook& cb, const ActGemmArgs& a, int 
   }
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+// ===========================================================================
+// Tensor-memory variant for up to 32 tokens (rows_b <= 64), the small-batch
+// hot path.  Differences from k_act_gemm<true> above:
+//   - K steps of 256 (32 groups); index tiles 64 B per row loaded with a
+//     64-byte TMA swizzle so that 32 threads reading 16 B each from 32
+//     consecutive rows hit 32 distinct banks;
+//   - 16 decode warps (four per tensor-memory lane quarter, 8 groups each);
+//   - the group decode works on packed bytes: the nibble-packed table entries
+//     are widened to biased bytes, stage 1 and stage 2 are combined with one
+//     add per 4 coordinates, byte pairs become bf16 pairs with one byte
+//     permute (0x43XX = 128 + XX) and one packed bf16 FMA that removes the
+//     bias and applies the sign;
+//   - the codebook table is read with explicit shared-memory loads;
+//   - programmatic dependent launch: the table copy, the tensor-memory
+//     allocation and (when the previous kernel is this library's activation
+//     transform) the first index tiles are issued before waiting for the
+//     previous kernel; only the transformed activations wait.
+// ===========================================================================
+namespace agt {
+constexpr int ROWS = 128;
+constexpr int KSTEP = 256;
+constexpr int GROUPS = KSTEP / 8;
+constexpr int DEC_WARPS = 16;
+constexpr int THREADS = 64 + DEC_WARPS * 32;
+constexpr int I1_BYTES = ROWS * GROUPS * 2;
+constexpr int TABLE_BYTES = 131088;
+constexpr int STAGE0 = 132096;        // table, rounded up to 1 KB
+constexpr uint32_t D_COLS = 64;       // accumulator columns (rows_b <= 64)
+constexpr uint32_t A_COLS = KSTEP / 2;
+constexpr int BAR_LIMIT = kMaxDynSmem - 1024 - 256;  // alignment slack, barriers
+}  // namespace agt
+
+struct TmPlan {
+  int stages, b_bytes, i2_bytes, stage_bytes, bar_off, total;
+};
+
+__host__ __device__ inline TmPlan tm_plan(int rows_b, int bpw) {
+  using namespace agt;
+  TmPlan p;
+  p.b_bytes = rows_b * KSTEP * 2;
+  p.i2_bytes = bpw == 2 ? 0 : (bpw == 3 ? ROWS * GROUPS : ROWS * GROUPS * 2);
+  p.stage_bytes = (p.b_bytes + I1_BYTES + p.i2_bytes + 1023) & ~1023;
+  p.stages = (BAR_LIMIT - STAGE0) / p.stage_bytes;
+  if (p.stages > 3) p.stages = 3;
+  int end = STAGE0 + p.stages * p.stage_bytes;
+  // the receive area of the reduction (128 rows x 8 float4 at most) reuses the stage area
+  const int part = STAGE0 + ROWS * 32 * 4;
+  if (part > end) end = part;
+  p.bar_off = end;
+  p.total = 1024 + p.bar_off + 256;
+  return p;
+}
+
+// Offset of group-part `part` (8 groups) of row r in a 64-byte-swizzled index tile.
+__device__ __forceinline__ uint32_t sw64_off(int r, int part) {
+  return (uint32_t)(r * 64 + ((part ^ ((r >> 1) & 3)) << 4));
+}
+
+// Packed decode of one group: codebook entries ea (stage 1) and eb (stage 2,
+// unused for 2 bpw), signs taken from the index parities.  Writes the 8 bf16
+// values of z = m (c1 + beta c2) as four bf16x2 words.
+template <int BPW>
+__device__ __forceinline__ void decode_group(uint32_t i1, uint32_t i2, uint32_t ea, uint32_t eb,
+                                             uint32_t* out) {
+  // neg1: index even (index 0 is the zero vector, whose sign does not matter)
+  const uint32_t neg1 = (~i1) & 1u;
+  const uint32_t mulc = 0x3F803F80u + neg1 * 0x80008000u;  // (+1, +1) or (-1, -1)
+  uint32_t wlo, whi, addc;
+  if (BPW == 2) {
+    wlo = ea & 0x0F0F0F0Fu;                  // v + 8, coordinates 0..3
+    whi = (ea >> 4) & 0x0F0F0F0Fu;           // coordinates 4..7
+    addc = 0xC308C308u - neg1 * 0x80008000u; // -(128 + 8) or +(128 + 8)
+  } else {
+    const uint32_t s = (i1 ^ i2) & 1u;       // stage signs differ
+    const uint32_t m = s * 0x1F1F1F1Fu;      // 31 - b = b ^ 31 for bytes b < 32
+    const uint32_t nk = s * 0xF0F0F0F1u;     // - 0x0F0F0F0F when signs differ
+    const uint32_t lo2 = (eb & 0x0F0F0F0Fu) ^ m;
+    const uint32_t hi2 = ((eb >> 4) & 0x0F0F0F0Fu) ^ m;
+    if (BPW == 4) {
+      // bytes 4 (v1 + 8) + (s ? 16 - (v2 + 8) : v2 + 8) = 4 v1 +- v2 + 40
+      wlo = ((ea << 2) & 0x3C3C3C3Cu) + lo2 + nk;
+      whi = ((ea >> 2) & 0x3C3C3C3Cu) + hi2 + nk;
+      addc = 0xC328C328u - neg1 * 0x80008000u;  // -(128 + 40) or +(128 + 40)
+    } else {
+      // bytes 2 (v1 + 8) + ... = 2 v1 +- v2 + 24
+      wlo = ((ea << 1) & 0x1E1E1E1Eu) + lo2 + nk;
+      whi = ((ea >> 3) & 0x1E1E1E1Eu) + hi2 + nk;
+      addc = 0xC318C318u - neg1 * 0x80008000u;  // -(128 + 24) or +(128 + 24)
+    }
+  }
+  // byte pair -> bf16 pair 0x43XX = 128 + XX (XX < 128), then x * (+-1) + (-+bias)
+  const uint32_t p0 = __byte_perm(wlo, 0x43434343u, 0x5140);
+  const uint32_t p1 = __byte_perm(wlo, 0x43434343u, 0x5342);
+  const uint32_t p2 = __byte_perm(whi, 0x43434343u, 0x5140);
+  const uint32_t p3 = __byte_perm(whi, 0x43434343u, 0x5342);
+  uint32_t r0, r1, r2, r3;
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r0) : "r"(p0), "r"(mulc), "r"(addc));
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r1) : "r"(p1), "r"(mulc), "r"(addc));
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r2) : "r"(p2), "r"(mulc), "r"(addc));
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r3) : "r"(p3), "r"(mulc), "r"(addc));
+  out[0] = r0;
+  out[1] = r1;
+  out[2] = r2;
+  out[3] = r3;
+}
+
+// Byte offset, inside the pair table, of the entry of codebook index i.
+__device__ __forceinline__ uint32_t table_off(uint32_t i) { return ((i + 1u) >> 1) << 2; }
+
+template <int BPW>
+__global__ void __launch_bounds__(agt::THREADS, 1)
+    k_act_gemm_tm(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmI1,
+                  const __grid_constant__ CUtensorMap tmI2, DeviceCodebook cb, int M, int N, int K,
+                  int rows_b, float alpha, float* __restrict__ Y, int early_codes) {
+  using namespace agt;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const TmPlan plan = tm_plan(rows_b, BPW);
+  const int S = plan.stages;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + plan.bar_off);
+  uint64_t* full_code = bars;       // [3]
+  uint64_t* full_b = bars + 3;      // [3]
+  uint64_t* full_a = bars + 6;      // [3]
+  uint64_t* empty = bars + 9;       // [3]
+  uint64_t* acc_full = bars + 12;
+  uint64_t* table_full = bars + 13;
+  uint64_t* drain = bars + 14;
+  uint64_t* red_full = bars + 15;   // partial tiles pushed by the cluster peers
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+  const uint32_t table_s = smem_u32(smem);
+  uint8_t* stage0 = smem + STAGE0;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t crank = cluster_ctarank();
+  uint32_t ncl;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(ncl));
+  const int n0 = (int)(blockIdx.x / ncl) * ROWS;
+  const int ksteps = K / KSTEP;
+  const int ks_begin = (int)((int64_t)crank * ksteps / ncl);
+  const int nks = (int)((int64_t)(crank + 1) * ksteps / ncl) - ks_begin;
+  const uint32_t code_tx = (uint32_t)(I1_BYTES + plan.i2_bytes);
+  const int chunks = (M + 3) >> 2;          // float4 chunks of a partial row
+  const int R = ROWS / (int)ncl;            // rows of the tile this CTA reduces
+  uint32_t* status = cb.status;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full_code[s], 1);
+      mbar_init(&full_b[s], 1);
+      mbar_init(&full_a[s], DEC_WARPS);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(table_full, 1);
+    mbar_init(drain, 1);
+    mbar_init(red_full, 1);
+    fence_mbar_init();
+    // bytes this CTA receives from its ncl - 1 peers: R rows x chunks float4
+    mbar_arrive_expect_tx(red_full, (uint32_t)((ncl - 1) * R * chunks * 16));
+    *abort_flag = 0u;
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmB);
+      tma_prefetch_desc(&tmI1);
+      if (BPW > 2) tma_prefetch_desc(&tmI2);
+      mbar_arrive_expect_tx(table_full, TABLE_BYTES);
+      bulk_load(smem, cb.table, TABLE_BYTES, table_full);
+      const int pre = early_codes ? (nks < S ? nks : S) : 0;
+      for (int i = 0; i < pre; ++i) {
+        uint8_t* si1 = stage0 + i * plan.stage_bytes + plan.b_bytes;
+        const int g0 = (ks_begin + i) * GROUPS;
+        mbar_arrive_expect_tx(&full_code[i], code_tx);
+        tma_load_2d(si1, &tmI1, &full_code[i], g0, n0);
+        if (BPW > 2) tma_load_2d(si1 + I1_BYTES, &tmI2, &full_code[i], g0, n0);
+      }
+      grid_dep_wait();
+      uint32_t issued = 0;
+      for (int i = 0; i < nks; ++i) {
+        const int s = i % S;
+        const uint32_t round = (uint32_t)(i / S);
+        if (round > 0 &&
+            !mbar_wait_bounded(&empty[s], (round - 1u) & 1u, abort_flag, status, kDevTimeoutEmpty))
+          break;
+        uint8_t* sb = stage0 + s * plan.stage_bytes;
+        uint8_t* si1 = sb + plan.b_bytes;
+        const int k0 = (ks_begin + i) * KSTEP;
+        if (i >= pre) {
+          mbar_arrive_expect_tx(&full_code[s], code_tx);
+          tma_load_2d(si1, &tmI1, &full_code[s], k0 / 8, n0);
+          if (BPW > 2) tma_load_2d(si1 + I1_BYTES, &tmI2, &full_code[s], k0 / 8, n0);
+        }
+        mbar_arrive_expect_tx(&full_b[s], (uint32_t)plan.b_bytes);
+#pragma unroll
+        for (int bx = 0; bx < KSTEP / 64; ++bx)
+          tma_load_2d(sb + bx * rows_b * 128, &tmB, &full_b[s], k0 + 64 * bx, 0);
+        ++issued;
+      }
+      if (*abort_flag) {
+        uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(table_full, 0))
+          if (global_timer_ns() - t0 > 100000000ull) break;
+        for (uint32_t j = 0; j < (uint32_t)S && j < issued; ++j) {
+          const uint32_t idx = issued - 1 - j;
+          t0 = global_timer_ns();
+          while (!(mbar_try_wait(&full_b[idx % S], (idx / S) & 1u) &&
+                   mbar_try_wait(&full_code[idx % S], (idx / S) & 1u)))
+            if (global_timer_ns() - t0 > 100000000ull) break;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(ROWS, (uint32_t)rows_b);
+      // descriptor of the first 16-column slice of stage 0's B tile; slice j of
+      // stage s adds s * stage_bytes + (j >> 2) * rows_b * 128 + (j & 3) * 32 bytes
+      const uint64_t bd0 = smem_desc(smem_u32(stage0), 16, 1024, 2);
+      const uint32_t box16 = (uint32_t)(rows_b * 128) >> 4;
+      const uint32_t stage16 = (uint32_t)plan.stage_bytes >> 4;
+      bool ok = true;
+      for (int i = 0; i < nks && ok; ++i) {
+        const int s = i % S;
+        const uint32_t ph = (uint32_t)(i / S) & 1u;
+        if (!mbar_wait_bounded(&full_a[s], ph, abort_flag, status, kDevTimeoutFull) ||
+            !mbar_wait_bounded(&full_b[s], ph, abort_flag, status, kDevTimeoutFull)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t bds = bd0 + (uint64_t)((uint32_t)s * stage16);
+        const uint32_t a0 = tmem_base + D_COLS + (uint32_t)s * A_COLS;
+#pragma unroll
+        for (int j = 0; j < KSTEP / 16; ++j) {
+          const uint64_t bd = bds + (uint64_t)((uint32_t)(j >> 2) * box16 + (uint32_t)(j & 3) * 2u);
+          mma_ts(tmem_base, a0 + (uint32_t)(j * 8), bd, idesc, (i > 0 || j > 0) ? 1u : 0u);
+        }
+        mma_commit(&empty[s]);
+      }
+      if (ok) mma_commit(acc_full);
+      mma_commit(drain);
+      uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(drain, 0))
+        if (global_timer_ns() - t0 > 200000000ull) break;
+    }
+  } else {
+    // ------------------------------------------------------------ decoders
+    const int q = warp & 3;
+    const int part = (warp - 2) >> 2;
+    const int r = q * 32 + lane;
+    const uint32_t lane_bits = (uint32_t)(q * 32) << 16;
+    bool ok = mbar_wait_sleep(table_full, 0, abort_flag, status, kDevTimeoutFull);
+    for (int i = 0; i < nks && ok; ++i) {
+      const int s = i % S;
+      const uint32_t ph = (uint32_t)(i / S) & 1u;
+      if (!mbar_wait_sleep(&full_code[s], ph, abort_flag, status, kDevTimeoutFull)) break;
+      tc_fence_after();
+      const uint32_t si1 = smem_u32(stage0 + s * plan.stage_bytes + plan.b_bytes);
+      const uint4 c1 = lds128(si1 + sw64_off(r, part));
+      const uint32_t w1[4] = {c1.x, c1.y, c1.z, c1.w};
+      uint32_t w2[4] = {0u, 0u, 0u, 0u};
+      if (BPW == 4) {
+        const uint4 c2 = lds128(si1 + I1_BYTES + sw64_off(r, part));
+        w2[0] = c2.x; w2[1] = c2.y; w2[2] = c2.z; w2[3] = c2.w;
+      } else if (BPW == 3) {
+        // 32 one-byte indices per row, 32-byte swizzle: chunk (part >> 1), half (part & 1)
+        const uint32_t off = (uint32_t)(r * 32 + ((((part >> 1) ^ ((r >> 2) & 1))) << 4) +
+                                        (part & 1) * 8);
+        const uint2 c2 = lds64(si1 + I1_BYTES + off);
+        w2[0] = __byte_perm(c2.x, 0u, 0x4140);
+        w2[1] = __byte_perm(c2.x, 0u, 0x4342);
+        w2[2] = __byte_perm(c2.y, 0u, 0x4140);
+        w2[3] = __byte_perm(c2.y, 0u, 0x4342);
+      }
+      uint32_t v[32];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t a = (w1[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
+        const uint32_t bb = (w2[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
+        const uint32_t ea = lds32(table_s + table_off(a));
+        const uint32_t eb = BPW > 2 ? lds32(table_s + table_off(bb)) : 0u;
+        decode_group<BPW>(a, bb, ea, eb, v + 4 * j);
+      }
+      tmem_st32(tmem_base + lane_bits + D_COLS + (uint32_t)s * A_COLS + (uint32_t)(part * 32), v);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&full_a[s]);
+    }
+  }
+
+  // ------------------------------------------------------------ epilogue ---
+  // Warps 2-5 hold row r of the 128 x rows_b accumulator (TMEM lane r); the
+  // token sums y[m] = D[r][2m] + D[r][2m + 1] (hi + lo) stay in registers.
+  float y[32];
+  const bool epi = warp >= 2 && warp < 6;
+  const int er = (warp & 3) * 32 + lane;
+  if (epi) {
+    const bool have = nks > 0 && mbar_wait_sleep(acc_full, 0, abort_flag, status, kDevTimeoutMma);
+    tc_fence_after();
+    uint32_t dv[D_COLS];
+#pragma unroll
+    for (int c = 0; c < (int)D_COLS; c += 16)
+      if (c < rows_b)
+        tmem_ld16(tmem_base + (uint32_t)c + ((uint32_t)((warp & 3) * 32) << 16),
+                  *reinterpret_cast<uint32_t(*)[16]>(dv + c));
+    tmem_ld_wait();
+#pragma unroll
+    for (int m = 0; m < 32; ++m)
+      y[m] = (have && m < M) ? __uint_as_float(dv[2 * m]) + __uint_as_float(dv[2 * m + 1]) : 0.0f;
+  }
+  // Every CTA of the cluster has finished with its stage area once all its
+  // threads arrive here; after the wait the peers may write into it.
+  tc_fence_before();
+  __syncthreads();
+  cluster_arrive();
+  cluster_wait();
+  // Reduce-scatter: row r goes to the CTA owning rows [owner*R, owner*R + R),
+  // slot [source rank][row - owner*R] of its receive area (the stage area).
+  float4* recv = reinterpret_cast<float4*>(stage0);
+  if (epi) {
+    const int owner = er / R;
+    const int slot = ((int)crank * R + (er - owner * R)) * chunks;
+    if (owner == (int)crank) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        if (c < chunks) recv[slot + c] = make_float4(y[4 * c], y[4 * c + 1], y[4 * c + 2], y[4 * c + 3]);
+    } else {
+      const uint32_t raddr = mapa_shared(smem_u32(recv + slot), (uint32_t)owner);
+      const uint32_t rbar = mapa_shared(smem_u32(red_full), (uint32_t)owner);
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        if (c < chunks)
+          st_async_v4(raddr + 16u * c, rbar,
+                      make_float4(y[4 * c], y[4 * c + 1], y[4 * c + 2], y[4 * c + 3]));
+    }
+  }
+  __syncthreads();   // local rows written
+  {
+    const bool got = mbar_wait_sleep(red_full, 0, abort_flag, status, kDevTimeoutCluster);
+    const int r0 = (int)crank * R;
+    for (int e = threadIdx.x; e < R * chunks; e += blockDim.x) {
+      const int row = e % R, c = e / R;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int src = 0; src < (int)ncl; ++src) {
+        const float4 v4 = recv[(src * R + row) * chunks + c];
+        acc.x += v4.x; acc.y += v4.y; acc.z += v4.z; acc.w += v4.w;
+      }
+      const int n = n0 + r0 + row;
+      if (got && n < N) {
+        const float o[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+          if (4 * c + t < M) Y[(size_t)(4 * c + t) * N + n] = alpha * o[t];
+      }
+    }
+  }
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+template <int BPW>
+static cudaError_t launch_tm(const DeviceCodebook& cb, const ActGemmArgs& a, int sm_count,
+                             cudaStream_t st) {
+  using namespace agt;
+  CUtensorMap tb, ti1, ti2;
+  if (!make_tmap_2d(&tb, a.Xt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.rows_b,
+                    (uint64_t)a.K, (uint32_t)a.rows_b, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&ti1, a.idx1, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)a.N,
+                    (uint64_t)(a.K / 8), ROWS, GROUPS, CU_TENSOR_MAP_SWIZZLE_64B))
+    return cudaErrorInvalidValue;
+  if (BPW == 4) {
+    if (!make_tmap_2d(&ti2, a.idx2, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)a.N,
+                      (uint64_t)(a.K / 8), ROWS, GROUPS, CU_TENSOR_MAP_SWIZZLE_64B))
+      return cudaErrorInvalidValue;
+  } else if (BPW == 3) {
+    if (!make_tmap_2d(&ti2, a.idx2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.N,
+                      (uint64_t)(a.K / 8), ROWS, GROUPS, CU_TENSOR_MAP_SWIZZLE_32B))
+      return cudaErrorInvalidValue;
+  } else {
+    ti2 = ti1;
+  }
+  const TmPlan plan = tm_plan(a.rows_b, BPW);
+  if (plan.stages < 2 || plan.total > kMaxDynSmem) return cudaErrorInvalidValue;
+  const int tiles = (int)((a.N + ROWS - 1) / ROWS);
+  const int ksteps = (int)(a.K / KSTEP);
+  int csize = 1;
+  while (csize < 8 && tiles * csize * 2 <= sm_count && csize * 2 <= ksteps) csize *= 2;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(tiles * csize));
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = (size_t)plan.total;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)csize;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = a.pdl ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  cudaError_t e = ensure_smem_limit(k_act_gemm_tm<BPW>, kMaxDynSmem);
+  if (e != cudaSuccess) return e;
+  e = cudaLaunchKernelEx(&cfg, k_act_gemm_tm<BPW>, tb, ti1, ti2, cb, (int)a.M, (int)a.N,
+                         (int)a.K, a.rows_b, a.alpha, a.Y, a.early_codes);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+// Tensor-memory variant: the 256-wide kernel above when the shape allows it
+// (up to 32 tokens, K a multiple of 256), else the generic kernel.
+cudaError_t launch_act_gemm(const DeviceCodebook& cb, const ActGemmArgs& a, int sm_count,
+                            cudaStream_t st) {
+  const bool tm = a.variant == 1 && a.rows_b <= (int)agt::D_COLS && (a.K % agt::KSTEP) == 0;
+  if (!tm) return launch_act_gemm_generic(cb, a, sm_count, st);
+  if (a.bpw == 2) return launch_tm<2>(cb, a, sm_count, st);
+  if (a.bpw == 3) return launch_tm<3>(cb, a, sm_count, st);
+  return launch_tm<4>(cb, a, sm_count, st);
 }
 
 }  // namespace e8

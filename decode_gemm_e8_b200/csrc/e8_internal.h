@@ -45,7 +45,7 @@ cudaError_t launch_decode(const DeviceCodebook& cb, const uint16_t* idx1, const 
 // X [M][K] bf16 -> Xt [rows][K] bf16: rows [0, M) hi parts, [M, 2M) lo parts of
 // FWHT(D x), rows [2M, rows) zero.
 cudaError_t launch_act_rht(const uint16_t* X, int64_t M, int64_t K, uint64_t seed, uint16_t* Xt,
-                           int64_t rows, cudaStream_t st);
+                           int64_t rows, cudaStream_t st, int pdl = 0);
 
 // Fused decode + GEMM with the transform moved onto the activations:
 // Y[m][n] = alpha * sum_k Xt[m][k] Z[n][k] (hi + lo rows), Z decoded on chip.
@@ -59,6 +59,8 @@ struct ActGemmArgs {
   float alpha;
   float* Y;             // [M][N] fp32
   int variant;          // 0: decoded operand in shared memory, 1: in tensor memory
+  int pdl;              // 1: launch with programmatic stream serialization
+  int early_codes;      // 1: codes may be fetched before the predecessor kernel ends
 };
 cudaError_t launch_act_gemm(const DeviceCodebook& cb, const ActGemmArgs& a, int sm_count,
                             cudaStream_t st);

@@ -85,7 +85,7 @@ extern "C" int e8_gemm_act_noalloc(const e8_codebook* cb, const uint16_t* X, int
   int rc = scratch_address(dev, &xt);
   if (rc != E8_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (e8::launch_act_rht(X, M, K, rht_seed, xt, rows, st) != cudaSuccess) return E8_ECUDA;
+  if (e8::launch_act_rht(X, M, K, rht_seed, xt, rows, st, 1) != cudaSuccess) return E8_ECUDA;
   e8::DeviceCodebook d;
   d.vecs = cb->vecs;
   d.table = cb->table;
@@ -105,5 +105,7 @@ extern "C" int e8_gemm_act_noalloc(const e8_codebook* cb, const uint16_t* X, int
   a.alpha = (float)((double)scale / ((double)m * std::sqrt((double)nh)));
   a.Y = Y;
   a.variant = 1;
+  a.pdl = 1;
+  a.early_codes = 1;
   return e8::launch_act_gemm(d, a, cb->sm_count, st) == cudaSuccess ? E8_OK : E8_ECUDA;
 }

@@ -119,8 +119,8 @@ int e8_decode_to_bf16(const e8_codebook* cb, const uint16_t* idx1, const void* i
                       void* stream);
 
 /* Activation-side transform used by E8_GEMM_ACT_RHT: X bf16 [M][K] ->
- * Xt bf16 [rows][K] with rows >= 2M; row m holds hi = bf16(FWHT(D x_m)) and
- * row M + m holds lo = bf16(FWHT(D x_m) - hi); rows 2M..rows-1 are zeroed.
+ * Xt bf16 [rows][K] with rows >= 2M; row 2m holds hi = bf16(FWHT(D x_m)) and
+ * row 2m + 1 holds lo = bf16(FWHT(D x_m) - hi); rows 2M..rows-1 are zeroed.
  * No normalisation is applied (the GEMM multiplies by alpha). */
 int e8_act_rht(const uint16_t* X, int64_t M, int64_t K, uint64_t rht_seed, uint16_t* Xt,
                int64_t rows, void* stream);
@@ -136,7 +136,7 @@ int e8_gemm(const e8_codebook* cb, const uint16_t* X, int64_t M, const uint16_t*
             float* Y, int mode, void* workspace, size_t ws_bytes, void* stream);
 
 /* Second half of E8_GEMM_ACT_RHT on activations already transformed by
- * e8_act_rht: Y fp32 [M][N] = alpha * (Xt[0:M] + Xt[M:2M]) * Z^T, with Z the
+ * e8_act_rht: Y fp32 [M][N] = alpha * (Xt[2m] + Xt[2m+1]) * Z^T, with Z the
  * integer codebook vectors decoded on chip and alpha from `scale`.  Xt is bf16
  * [rows][K] with rows == e8_gemm_xt_rows(M) (2M rounded up to a multiple of
  * 16; padding rows must be zero, as e8_act_rht leaves them).  One transform can
