@@ -253,20 +253,19 @@ def run_ours(args):
     alg_bytes = code_bytes + M * K * 2 + M * N * 4
 
     # dominant kernel alone: fused decode-GEMM on pre-transformed activations
-    rows = e8.e8_gemm_xt_rows(M)
-    Xt = e8.e8_act_rht(X, rs, rows=rows)
+    xq = e8.e8_act_rht_q8(X, rs)
 
-    def gemm_only(i, M=M, Xt=Xt, Y=Y):
+    def gemm_only(i, M=M, xq=xq, Y=Y):
         c1, c2 = codes[i % ROTATE]
-        e8.e8_gemm_xt(cb, Xt, M, c1, c2, N, K, bpw, s, Y=Y, stream=stream)
+        e8.e8_gemm_xt(cb, xq, M, c1, c2, N, K, bpw, s, Y=Y, stream=stream)
 
     kern_steps = min(args.steps, 20 * GRAPH_STEPS)
     k_ms = _time_graphs(gemm_only, kern_steps, args.warmup, stream)
     k_us = k_ms * 1e3 / kern_steps
     achieved = alg_bytes / (k_us * 1e-6) / 1e9
 
-    def rht_only(i, X=X, Xt=Xt):
-        e8.e8_act_rht(X, rs, rows=rows, out=Xt, stream=stream)
+    def rht_only(i, X=X, xq=xq):
+        e8.e8_act_rht_q8(X, rs, out=xq, stream=stream)
 
     r_ms = _time_graphs(rht_only, kern_steps, args.warmup, stream)
     rht_us = r_ms * 1e3 / kern_steps
@@ -319,7 +318,9 @@ def run_ours(args):
                 "workload": "%s: W %dx%d N(0,%.2f^2) seed %d, %d bpw, X %dx%d bf16 N(0,1) seed %d"
                             % (WORKLOAD, N, K, lay.std, lay.w_seed, bpw, M, K,
                                synth.workloads()[WORKLOAD].x_seed),
-                "M": M, "N": N, "K": K, "bpw": bpw, "gemm_mode": "act_rht (fused, TMEM operand)",
+                "M": M, "N": N, "K": K, "bpw": bpw,
+                "gemm_mode": "act_rht: int8 activation pieces, codes decoded into tensor memory, "
+                             "tcgen05 kind::i8",
                 "l2": "inputs larger than L2: %d rotating code sets, %.0f MB" %
                       (ROTATE, ROTATE * code_bytes / 1e6),
                 "launch": "CUDA graphs of %d steps" % GRAPH_STEPS,
@@ -328,7 +329,7 @@ def run_ours(args):
             "decoded_weights_per_s": N * K * args.steps * ws / sec,
             "roofline": {
                 "bound": "hbm",
-                "kernel": "k_act_gemm (fused decode + tcgen05 GEMM)",
+                "kernel": "k_act_gemm_q8 (fused decode + tcgen05 GEMM)",
                 "achieved": round(achieved, 1),
                 "peak": peaks["hbm_gbs"],
                 "unit": "GB/s",
@@ -361,7 +362,7 @@ def _traffic_from_profile():
     """DRAM bytes per launch of k_act_gemm from the committed ncu summary, or None
     when the kernel source changed since the counters were taken."""
     import hashlib
-    prof = os.path.join(ROOT, "profiles", "k_act_gemm_llama4096_m16.md")
+    prof = os.path.join(ROOT, "profiles", "k_act_gemm_q8_llama4096_m16.md")
     src = os.path.join(ROOT, "decode_gemm_e8_b200", "csrc", "e8_gemm_act.cu")
     if not os.path.exists(prof):
         return None

@@ -26,7 +26,8 @@ E8_OP_ENCODE = 100
 
 # every symbol include/e8.h declares
 EXPORTED = ("e8_codebook_build", "e8_codebook_free", "e8_codebook_export", "e8_rht_forward",
-            "e8_encode", "e8_decode_to_bf16", "e8_act_rht", "e8_gemm", "e8_gemm_xt",
+            "e8_encode", "e8_decode_to_bf16", "e8_act_rht", "e8_act_rht_q8", "e8_act_q8_bytes",
+            "e8_gemm", "e8_gemm_xt",
             "e8_gemm_xt_rows", "e8_gemm_act_noalloc", "e8_gemm_auto_mode",
             "e8_workspace_bytes", "e8_sync_status", "e8_debug_wait_timeout", "e8_status_str",
             "e8_version")
@@ -60,8 +61,9 @@ def load_library(path: str = LIB_PATH):
         "e8_act_rht": ([P, I64, I64, U64, P, I64, P], c.c_int),
         "e8_gemm": ([P, P, I64, P, P, I64, I64, c.c_int, U64, c.c_float, P, c.c_int, P,
                      c.c_size_t, P], c.c_int),
-        "e8_gemm_xt": ([P, P, I64, I64, P, P, I64, I64, c.c_int, c.c_float, P, c.c_int, P],
-                       c.c_int),
+        "e8_act_rht_q8": ([P, I64, I64, U64, P, P], c.c_int),
+        "e8_act_q8_bytes": ([I64, I64], c.c_size_t),
+        "e8_gemm_xt": ([P, P, I64, P, P, I64, I64, c.c_int, c.c_float, P, P], c.c_int),
         "e8_gemm_xt_rows": ([I64], c.c_int),
         "e8_gemm_act_noalloc": ([P, P, I64, P, P, I64, I64, c.c_int, U64, c.c_float, P, P],
                                 c.c_int),
@@ -232,15 +234,30 @@ def e8_gemm_xt_rows(M: int) -> int:
     return int(load_library().e8_gemm_xt_rows(int(M)))
 
 
-def e8_gemm_xt(cb: Codebook, Xt, M: int, idx1, idx2, N: int, K: int, bpw: int, scale: float,
-               mode: int = E8_GEMM_ACT_RHT, Y=None, stream=None):
-    """Fused decode-GEMM on activations already transformed by e8_act_rht."""
+def e8_act_q8_bytes(M: int, K: int) -> int:
+    return int(load_library().e8_act_q8_bytes(int(M), int(K)))
+
+
+def e8_act_rht_q8(X, rht_seed: int, out=None, stream=None):
+    """X bf16 [M, K] -> the int8 activation buffer (uint8 tensor) of e8_gemm_xt."""
+    import torch
+    M, K = X.shape
+    if out is None:
+        out = torch.empty(max(16, e8_act_q8_bytes(M, K)), dtype=torch.uint8, device=X.device)
+    _check(load_library().e8_act_rht_q8(_ptr(X), M, K, int(rht_seed) & (2**64 - 1), _ptr(out),
+                                        _stream(stream)), "e8_act_rht_q8")
+    return out
+
+
+def e8_gemm_xt(cb: Codebook, xq, M: int, idx1, idx2, N: int, K: int, bpw: int, scale: float,
+               Y=None, stream=None):
+    """Fused decode + int8 GEMM on a buffer from e8_act_rht_q8."""
     import torch
     if Y is None:
-        Y = torch.empty((M, N), dtype=torch.float32, device=Xt.device)
-    _check(load_library().e8_gemm_xt(cb.handle, _ptr(Xt), Xt.shape[0], int(M), _ptr(idx1),
-                                     _ptr(idx2), int(N), int(K), int(bpw), float(scale), _ptr(Y),
-                                     int(mode), _stream(stream)), "e8_gemm_xt")
+        Y = torch.empty((M, N), dtype=torch.float32, device=xq.device)
+    _check(load_library().e8_gemm_xt(cb.handle, _ptr(xq), int(M), _ptr(idx1), _ptr(idx2), int(N),
+                                     int(K), int(bpw), float(scale), _ptr(Y), _stream(stream)),
+           "e8_gemm_xt")
     return Y
 
 

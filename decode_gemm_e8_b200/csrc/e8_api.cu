@@ -26,6 +26,14 @@ cudaError_t ensure_smem_limit_ptr(const void* kernel, int bytes) {
   std::lock_guard<std::mutex> lock(mu);
   for (int i = 0; i < used; ++i)
     if (kern[i] == kernel && devs[i] == dev) return cudaSuccess;
+  // the limit may not exceed the opt-in maximum minus the kernel's static shared memory
+  int optin = 0;
+  cudaFuncAttributes fa;
+  if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) == cudaSuccess &&
+      cudaFuncGetAttributes(&fa, kernel) == cudaSuccess) {
+    const int cap = optin - (int)fa.sharedSizeBytes;
+    if (bytes > cap) bytes = cap;
+  }
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e == cudaSuccess && used < kSlots) {
     kern[used] = kernel;
@@ -33,6 +41,67 @@ cudaError_t ensure_smem_limit_ptr(const void* kernel, int bytes) {
     ++used;
   }
   return e;
+}
+
+size_t act_scratch_bytes(int64_t M, int64_t K, int smem_variant) {
+  const int64_t rows = (2 * M + 15) / 16 * 16;
+  if (!smem_variant && q8_eligible(M, K)) return q8_layout(M, K, rows).total;
+  return (((size_t)rows * (size_t)K * 2) + 255) & ~size_t(255);
+}
+
+cudaError_t run_act_gemm(const e8_codebook* cb, const uint16_t* X, int64_t M,
+                         const uint16_t* idx1, const void* idx2, int64_t N, int64_t K, int bpw,
+                         uint64_t seed, float alpha, float* Y, int smem_variant, void* scratch,
+                         cudaStream_t st) {
+  DeviceCodebook d;
+  d.vecs = cb->vecs;
+  d.table = cb->table;
+  d.hkeys = cb->hkeys;
+  d.hvals = cb->hvals;
+  d.status = cb->status;
+  const int rows = (int)((2 * M + 15) / 16 * 16);
+  if (!smem_variant && q8_eligible(M, K)) {
+    const Q8Layout l = q8_layout(M, K, rows);
+    uint8_t* buf = static_cast<uint8_t*>(scratch);
+    ActQ8Args a;
+    a.Xq = reinterpret_cast<int8_t*>(buf);
+    a.scales = reinterpret_cast<float*>(buf + l.scales_off);
+    a.colsum = reinterpret_cast<int32_t*>(buf + l.colsum_off);
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.rows_b = rows;
+    a.idx1 = idx1;
+    a.idx2 = idx2;
+    a.bpw = bpw;
+    a.alpha = alpha;
+    a.Y = Y;
+    a.pdl = 1;          // the fused kernel's prologue overlaps the transform
+    a.early_codes = 1;  // which writes only the activation buffer
+    cudaError_t e = launch_act_q8(X, M, K, seed, reinterpret_cast<int8_t*>(buf),
+                                  reinterpret_cast<float*>(buf + l.scales_off),
+                                  reinterpret_cast<int32_t*>(buf + l.colsum_off), rows, st, 1);
+    if (e != cudaSuccess) return e;
+    return launch_act_gemm_q8(d, a, cb->sm_count, st);
+  }
+  uint16_t* Xt = static_cast<uint16_t*>(scratch);
+  cudaError_t e = launch_act_rht(X, M, K, seed, Xt, rows, st, 0);
+  if (e != cudaSuccess) return e;
+  ActGemmArgs a;
+  a.Xt = Xt;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.rows_b = rows;
+  a.idx1 = idx1;
+  a.idx2 = idx2;
+  a.bpw = bpw;
+  a.alpha = alpha;
+  a.Y = Y;
+  a.variant = smem_variant ? 0 : 1;
+  a.pdl = 0;
+  a.early_codes = 0;
+  return launch_act_gemm(d, a, cb->sm_count, st);
 }
 
 }  // namespace e8
@@ -109,6 +178,7 @@ const char* e8_status_str(int s) {
 }
 
 int e8_codebook_build(e8_codebook** out, int device) {
+  (void)cudaGetLastError();  // a failed earlier launch must not be reported here
   if (!out) return E8_EINVAL;
   *out = nullptr;
   int ndev = 0;
@@ -204,8 +274,9 @@ size_t e8_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int bpw) {
     case E8_GEMM_AUTO:
       return e8_workspace_bytes(e8_gemm_auto_mode(M, N, K, bpw), M, N, K, bpw);
     case E8_GEMM_ACT_RHT:
+      return e8::act_scratch_bytes(M, K, 0);
     case E8_GEMM_ACT_RHT_SMEM:
-      return round256((size_t)rows_b_for(M) * (size_t)K * 2);
+      return e8::act_scratch_bytes(M, K, 1);
     case E8_GEMM_DECODED_W:
     case E8_GEMM_SIMT:
       return round256((size_t)N * (size_t)K * 2);
@@ -300,25 +371,8 @@ int e8_gemm(const e8_codebook* cb, const uint16_t* X, int64_t M, const uint16_t*
   const e8::DeviceCodebook d = dev_view(cb);
   cudaError_t e;
   if (act) {
-    const int rows_b = rows_b_for(M);
-    uint16_t* Xt = static_cast<uint16_t*>(workspace);
-    e = e8::launch_act_rht(X, M, K, rht_seed, Xt, rows_b, st, 1);
-    if (e != cudaSuccess) return E8_ECUDA;
-    e8::ActGemmArgs a;
-    a.Xt = Xt;
-    a.M = M;
-    a.N = N;
-    a.K = K;
-    a.rows_b = rows_b;
-    a.idx1 = idx1;
-    a.idx2 = idx2;
-    a.bpw = bpw;
-    a.alpha = alpha;
-    a.Y = Y;
-    a.variant = mode == E8_GEMM_ACT_RHT ? 1 : 0;
-    a.pdl = 1;          // overlaps the prologue with the transform just launched
-    a.early_codes = 1;  // that transform writes only Xt
-    e = e8::launch_act_gemm(d, a, cb->sm_count, st);
+    e = e8::run_act_gemm(cb, X, M, idx1, idx2, N, K, bpw, rht_seed, alpha, Y,
+                         mode == E8_GEMM_ACT_RHT_SMEM ? 1 : 0, workspace, st);
     return cuda_status(e);
   }
   uint16_t* Wd = static_cast<uint16_t*>(workspace);
@@ -331,9 +385,30 @@ int e8_gemm(const e8_codebook* cb, const uint16_t* X, int64_t M, const uint16_t*
   return cuda_status(e);
 }
 
-int e8_gemm_xt(const e8_codebook* cb, const uint16_t* Xt, int64_t rows, int64_t M,
-               const uint16_t* idx1, const void* idx2, int64_t N, int64_t K, int bpw,
-               float scale, float* Y, int mode, void* stream) {
+int e8_act_rht_q8(const uint16_t* X, int64_t M, int64_t K, uint64_t rht_seed, void* buf,
+                  void* stream) {
+  (void)cudaGetLastError();  // a failed earlier launch must not be reported here
+  if (M < 0 || !valid_k(K)) return E8_EINVAL;
+  if (M == 0) return E8_OK;
+  if (!e8::q8_eligible(M, K)) return E8_EINVAL;
+  if (!X || !buf || !aligned16(X) || !aligned16(buf)) return E8_EINVAL;
+  const int64_t rows = rows_b_for(M);
+  const e8::Q8Layout l = e8::q8_layout(M, K, rows);
+  uint8_t* b = static_cast<uint8_t*>(buf);
+  return cuda_status(e8::launch_act_q8(X, M, K, rht_seed, reinterpret_cast<int8_t*>(b),
+                                       reinterpret_cast<float*>(b + l.scales_off),
+                                       reinterpret_cast<int32_t*>(b + l.colsum_off), rows,
+                                       (cudaStream_t)stream, 0));
+}
+
+size_t e8_act_q8_bytes(int64_t M, int64_t K) {
+  if (M < 1 || !valid_k(K) || !e8::q8_eligible(M, K)) return 0;
+  return e8::q8_layout(M, K, rows_b_for(M)).total;
+}
+
+int e8_gemm_xt(const e8_codebook* cb, const void* xq, int64_t M, const uint16_t* idx1,
+               const void* idx2, int64_t N, int64_t K, int bpw, float scale, float* Y,
+               void* stream) {
   (void)cudaGetLastError();  // a failed earlier launch must not be reported here
   int rc = check_device(cb);
   if (rc != E8_OK) return rc;
@@ -341,16 +416,19 @@ int e8_gemm_xt(const e8_codebook* cb, const uint16_t* Xt, int64_t rows, int64_t 
       !std::isfinite(scale))
     return E8_EINVAL;
   if ((bpw == 2) != (idx2 == nullptr)) return E8_EINVAL;
-  if (mode == E8_GEMM_AUTO) mode = E8_GEMM_ACT_RHT;
-  if (mode != E8_GEMM_ACT_RHT && mode != E8_GEMM_ACT_RHT_SMEM) return E8_EINVAL;
-  if (M > 64 || (K % 128) != 0 || N > INT32_MAX || K > INT32_MAX) return E8_EINVAL;
+  if (N > INT32_MAX) return E8_EINVAL;
   if (M == 0 || N == 0) return E8_OK;
-  if (rows != rows_b_for(M)) return E8_EINVAL;
-  if (!Xt || !idx1 || !Y || !aligned16(Xt) || !aligned16(idx1) || !aligned16(Y) ||
+  if (!e8::q8_eligible(M, K)) return E8_EINVAL;
+  if (!xq || !idx1 || !Y || !aligned16(xq) || !aligned16(idx1) || !aligned16(Y) ||
       (idx2 && !aligned16(idx2)))
     return E8_EINVAL;
-  e8::ActGemmArgs a;
-  a.Xt = Xt;
+  const int64_t rows = rows_b_for(M);
+  const e8::Q8Layout l = e8::q8_layout(M, K, rows);
+  const uint8_t* b = static_cast<const uint8_t*>(xq);
+  e8::ActQ8Args a;
+  a.Xq = reinterpret_cast<const int8_t*>(b);
+  a.scales = reinterpret_cast<const float*>(b + l.scales_off);
+  a.colsum = reinterpret_cast<const int32_t*>(b + l.colsum_off);
   a.M = M;
   a.N = N;
   a.K = K;
@@ -360,10 +438,9 @@ int e8_gemm_xt(const e8_codebook* cb, const uint16_t* Xt, int64_t rows, int64_t 
   a.bpw = bpw;
   a.alpha = alpha_of(scale, e8::hadamard_block(K), bpw);
   a.Y = Y;
-  a.variant = mode == E8_GEMM_ACT_RHT ? 1 : 0;
   a.pdl = 1;          // only the library's table is read before the previous kernel ends
   a.early_codes = 0;  // the previous kernel is the caller's and may write the codes
-  return cuda_status(e8::launch_act_gemm(dev_view(cb), a, cb->sm_count, (cudaStream_t)stream));
+  return cuda_status(e8::launch_act_gemm_q8(dev_view(cb), a, cb->sm_count, (cudaStream_t)stream));
 }
 
 int e8_gemm_xt_rows(int64_t M) { return M < 0 ? 0 : rows_b_for(M); }

@@ -376,24 +376,24 @@ static cudaError_t launch_act_gemm_generic(const DeviceCodebook& cb, const ActGe
 }
 
 // ===========================================================================
-// Tensor-memory variant for up to 32 tokens (rows_b <= 64), the small-batch
-// hot path.  Differences from k_act_gemm<true> above:
-//   - K steps of 256 (32 groups); index tiles 64 B per row loaded with a
-//     64-byte TMA swizzle so that 32 threads reading 16 B each from 32
-//     consecutive rows hit 32 distinct banks;
-//   - 16 decode warps (four per tensor-memory lane quarter, 8 groups each);
-//   - the group decode works on packed bytes: the nibble-packed table entries
-//     are widened to biased bytes, stage 1 and stage 2 are combined with one
-//     add per 4 coordinates, byte pairs become bf16 pairs with one byte
-//     permute (0x43XX = 128 + XX) and one packed bf16 FMA that removes the
-//     bias and applies the sign;
-//   - the codebook table is read with explicit shared-memory loads;
-//   - programmatic dependent launch: the table copy, the tensor-memory
-//     allocation and (when the previous kernel is this library's activation
-//     transform) the first index tiles are issued before waiting for the
-//     previous kernel; only the transformed activations wait.
+// int8 tensor-core variant for up to 32 tokens: the small-batch hot path.
+//
+// The transformed activations arrive as two int8 pieces per token (rows 2m
+// and 2m + 1 of Xq, see k_act_q8) with a per-token step s_m, so that
+//   xt_m = s_m (q0_m + q1_m / 128)   (error below s_m / 256).
+// The weight operand is z + 128 as unsigned bytes (|z| <= 30), decoded on chip
+// straight into tensor memory; tcgen05.mma kind::i8 (K = 32 per instruction)
+// accumulates exactly in int32, and the epilogue removes the bias with the
+// per-row column sums of Xq:
+//   y[m][n] = alpha s_m ((D[n][2m] - 128 cs[2m]) + (D[n][2m+1] - 128 cs[2m+1]) / 128).
+// Structure: warp 0 TMA producer (index tiles with a 64-byte swizzle, Xq tiles
+// with a 128-byte swizzle), warp 1 tensor-memory allocation + one MMA issuer,
+// 16 decode warps (four per tensor-memory lane quarter, 8 groups each per K
+// step of 256), programmatic dependent launch (table copy and index tiles
+// before waiting for the transform), split-K over a cluster with the partial
+// tiles pushed to their owner CTA by st.async.
 // ===========================================================================
-namespace agt {
+namespace agq {
 constexpr int ROWS = 128;
 constexpr int KSTEP = 256;
 constexpr int GROUPS = KSTEP / 8;
@@ -402,28 +402,31 @@ constexpr int THREADS = 64 + DEC_WARPS * 32;
 constexpr int I1_BYTES = ROWS * GROUPS * 2;
 constexpr int TABLE_BYTES = 131088;
 constexpr int STAGE0 = 132096;        // table, rounded up to 1 KB
-constexpr uint32_t D_COLS = 64;       // accumulator columns (rows_b <= 64)
-constexpr uint32_t A_COLS = KSTEP / 2;
-constexpr int BAR_LIMIT = kMaxDynSmem - 1024 - 256;  // alignment slack, barriers
-}  // namespace agt
+constexpr uint32_t D_COLS = 64;       // int32 accumulator columns (rows_b <= 64)
+constexpr uint32_t A_COLS = KSTEP / 4;  // 4 int8 per tensor-memory column
+constexpr uint32_t TMEM_COLS = 256;
+constexpr int BAR_LIMIT = kMaxDynSmem - 1024 - 256;
+constexpr int RECV_BYTES = ROWS * 8 * 16;
+}  // namespace agq
 
-struct TmPlan {
-  int stages, b_bytes, i2_bytes, stage_bytes, bar_off, total;
+struct Q8Plan {
+  int stages, b_bytes, i2_bytes, stage_bytes, recv_off, aux_off, bar_off, total;
 };
 
-__host__ __device__ inline TmPlan tm_plan(int rows_b, int bpw) {
-  using namespace agt;
-  TmPlan p;
-  p.b_bytes = rows_b * KSTEP * 2;
+__host__ __device__ inline Q8Plan q8_plan(int rows_b, int bpw) {
+  using namespace agq;
+  Q8Plan p;
+  p.b_bytes = rows_b * KSTEP;
   p.i2_bytes = bpw == 2 ? 0 : (bpw == 3 ? ROWS * GROUPS : ROWS * GROUPS * 2);
   p.stage_bytes = (p.b_bytes + I1_BYTES + p.i2_bytes + 1023) & ~1023;
-  p.stages = (BAR_LIMIT - STAGE0) / p.stage_bytes;
+  // after the stages: the reduction's receive area (128 rows x 8 float4) and the
+  // per-token steps and row sums (32 + 64 words), so peers can push partial
+  // tiles while this CTA is still in its main loop
+  p.stages = (BAR_LIMIT - STAGE0 - RECV_BYTES - 512) / p.stage_bytes;
   if (p.stages > 3) p.stages = 3;
-  int end = STAGE0 + p.stages * p.stage_bytes;
-  // the receive area of the reduction (128 rows x 8 float4 at most) reuses the stage area
-  const int part = STAGE0 + ROWS * 32 * 4;
-  if (part > end) end = part;
-  p.bar_off = end;
+  p.recv_off = STAGE0 + p.stages * p.stage_bytes;
+  p.aux_off = p.recv_off + RECV_BYTES;
+  p.bar_off = p.aux_off + 512;
   p.total = 1024 + p.bar_off + 256;
   return p;
 }
@@ -433,67 +436,83 @@ __device__ __forceinline__ uint32_t sw64_off(int r, int part) {
   return (uint32_t)(r * 64 + ((part ^ ((r >> 1) & 3)) << 4));
 }
 
-// Packed decode of one group: codebook entries ea (stage 1) and eb (stage 2,
-// unused for 2 bpw), signs taken from the index parities.  Writes the 8 bf16
-// values of z = m (c1 + beta c2) as four bf16x2 words.
-template <int BPW>
-__device__ __forceinline__ void decode_group(uint32_t i1, uint32_t i2, uint32_t ea, uint32_t eb,
-                                             uint32_t* out) {
-  // neg1: index even (index 0 is the zero vector, whose sign does not matter)
-  const uint32_t neg1 = (~i1) & 1u;
-  const uint32_t mulc = 0x3F803F80u + neg1 * 0x80008000u;  // (+1, +1) or (-1, -1)
-  uint32_t wlo, whi, addc;
-  if (BPW == 2) {
-    wlo = ea & 0x0F0F0F0Fu;                  // v + 8, coordinates 0..3
-    whi = (ea >> 4) & 0x0F0F0F0Fu;           // coordinates 4..7
-    addc = 0xC308C308u - neg1 * 0x80008000u; // -(128 + 8) or +(128 + 8)
-  } else {
-    const uint32_t s = (i1 ^ i2) & 1u;       // stage signs differ
-    const uint32_t m = s * 0x1F1F1F1Fu;      // 31 - b = b ^ 31 for bytes b < 32
-    const uint32_t nk = s * 0xF0F0F0F1u;     // - 0x0F0F0F0F when signs differ
-    const uint32_t lo2 = (eb & 0x0F0F0F0Fu) ^ m;
-    const uint32_t hi2 = ((eb >> 4) & 0x0F0F0F0Fu) ^ m;
-    if (BPW == 4) {
-      // bytes 4 (v1 + 8) + (s ? 16 - (v2 + 8) : v2 + 8) = 4 v1 +- v2 + 40
-      wlo = ((ea << 2) & 0x3C3C3C3Cu) + lo2 + nk;
-      whi = ((ea >> 2) & 0x3C3C3C3Cu) + hi2 + nk;
-      addc = 0xC328C328u - neg1 * 0x80008000u;  // -(128 + 40) or +(128 + 40)
-    } else {
-      // bytes 2 (v1 + 8) + ... = 2 v1 +- v2 + 24
-      wlo = ((ea << 1) & 0x1E1E1E1Eu) + lo2 + nk;
-      whi = ((ea >> 3) & 0x1E1E1E1Eu) + hi2 + nk;
-      addc = 0xC318C318u - neg1 * 0x80008000u;  // -(128 + 24) or +(128 + 24)
-    }
-  }
-  // byte pair -> bf16 pair 0x43XX = 128 + XX (XX < 128), then x * (+-1) + (-+bias)
-  const uint32_t p0 = __byte_perm(wlo, 0x43434343u, 0x5140);
-  const uint32_t p1 = __byte_perm(wlo, 0x43434343u, 0x5342);
-  const uint32_t p2 = __byte_perm(whi, 0x43434343u, 0x5140);
-  const uint32_t p3 = __byte_perm(whi, 0x43434343u, 0x5342);
-  uint32_t r0, r1, r2, r3;
-  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r0) : "r"(p0), "r"(mulc), "r"(addc));
-  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r1) : "r"(p1), "r"(mulc), "r"(addc));
-  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r2) : "r"(p2), "r"(mulc), "r"(addc));
-  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r3) : "r"(p3), "r"(mulc), "r"(addc));
-  out[0] = r0;
-  out[1] = r1;
-  out[2] = r2;
-  out[3] = r3;
-}
-
 // Byte offset, inside the pair table, of the entry of codebook index i.
 __device__ __forceinline__ uint32_t table_off(uint32_t i) { return ((i + 1u) >> 1) << 2; }
 
+// Packed decode of one group into 8 unsigned bytes z + 128 (two words, the
+// coordinates 0..3 and 4..7).  ea / eb: pair-table entries of the stage-1 and
+// stage-2 indices (8 nibbles v + 8); the sign of a stage is set when its index
+// is even (index 0 is the zero vector, whose sign does not matter).  With
+// B = v + 8 in [2, 14], the negated value's biased byte is B ^ 31 = 23 - v,
+// so one XOR per word applies a stage's sign and a per-group constant fixes
+// the bias:  byte = mul (B1 or B1 ^ 31) + (B2 or B2 ^ 31) + c(s1, s2) = z + 128.
 template <int BPW>
-__global__ void __launch_bounds__(agt::THREADS, 1)
-    k_act_gemm_tm(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmI1,
+__device__ __forceinline__ void decode_group_q8(uint32_t i1, uint32_t i2, uint32_t ea, uint32_t eb,
+                                                uint32_t& lo, uint32_t& hi) {
+  const uint32_t s1 = (~i1) & 1u;
+  const uint32_t m1 = s1 * 0x1F1F1F1Fu;
+  const uint32_t lo1 = (ea & 0x0F0F0F0Fu) ^ m1;
+  const uint32_t hi1 = ((ea >> 4) & 0x0F0F0F0Fu) ^ m1;
+  if (BPW == 2) {
+    // v + 128: B + 120, or (23 - v) + 105 = -v + 128
+    const uint32_t c = 0x78787878u - s1 * 0x0F0F0F0Fu;
+    lo = lo1 + c;
+    hi = hi1 + c;
+  } else {
+    const uint32_t s2 = (~i2) & 1u;
+    const uint32_t m2 = s2 * 0x1F1F1F1Fu;
+    const uint32_t lo2 = (eb & 0x0F0F0F0Fu) ^ m2;
+    const uint32_t hi2 = ((eb >> 4) & 0x0F0F0F0Fu) ^ m2;
+    if (BPW == 4) {
+      // 4 (+-v1) + (+-v2) + 128
+      const uint32_t c = 0x58585858u - s1 * 0x3C3C3C3Cu - s2 * 0x0F0F0F0Fu;
+      lo = lo1 * 4u + lo2 + c;
+      hi = hi1 * 4u + hi2 + c;
+    } else {
+      // 2 (+-v1) + (+-v2) + 128
+      const uint32_t c = 0x68686868u - s1 * 0x1E1E1E1Eu - s2 * 0x0F0F0F0Fu;
+      lo = lo1 * 2u + lo2 + c;
+      hi = hi1 * 2u + hi2 + c;
+    }
+  }
+}
+
+__device__ __forceinline__ void mma_ts_i8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// kind::i8 instruction descriptor: A unsigned 8-bit, B signed 8-bit, D int32, K-major.
+__host__ __device__ constexpr uint32_t idesc_u8s8_s32(uint32_t M, uint32_t N) {
+  return (2u << 4) | (0u << 7) | (1u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+
+// 32 lanes x 32 bit, 16 consecutive columns per thread.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15])
+      : "memory");
+}
+
+template <int BPW>
+__global__ void __launch_bounds__(agq::THREADS, 1)
+    k_act_gemm_q8(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmI1,
                   const __grid_constant__ CUtensorMap tmI2, DeviceCodebook cb, int M, int N, int K,
-                  int rows_b, float alpha, float* __restrict__ Y, int early_codes) {
-  using namespace agt;
+                  int rows_b, float alpha, const float* __restrict__ tok_scale,
+                  const int32_t* __restrict__ colsum, float* __restrict__ Y, int early_codes) {
+  using namespace agq;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  const TmPlan plan = tm_plan(rows_b, BPW);
+  const Q8Plan plan = q8_plan(rows_b, BPW);
   const int S = plan.stages;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + plan.bar_off);
   uint64_t* full_code = bars;       // [3]
@@ -534,18 +553,20 @@ __global__ void __launch_bounds__(agt::THREADS, 1)
     mbar_init(drain, 1);
     mbar_init(red_full, 1);
     fence_mbar_init();
-    // bytes this CTA receives from its ncl - 1 peers: R rows x chunks float4
     mbar_arrive_expect_tx(red_full, (uint32_t)((ncl - 1) * R * chunks * 16));
     *abort_flag = 0u;
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 512);
+    tmem_alloc(tmem_slot, TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // publishes the initialised receive barrier to the cluster; the matching
+  // wait comes right before the first push into a peer
+  cluster_arrive();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -579,9 +600,8 @@ __global__ void __launch_bounds__(agt::THREADS, 1)
           if (BPW > 2) tma_load_2d(si1 + I1_BYTES, &tmI2, &full_code[s], k0 / 8, n0);
         }
         mbar_arrive_expect_tx(&full_b[s], (uint32_t)plan.b_bytes);
-#pragma unroll
-        for (int bx = 0; bx < KSTEP / 64; ++bx)
-          tma_load_2d(sb + bx * rows_b * 128, &tmB, &full_b[s], k0 + 64 * bx, 0);
+        tma_load_2d(sb, &tmB, &full_b[s], k0, 0);
+        tma_load_2d(sb + rows_b * 128, &tmB, &full_b[s], k0 + 128, 0);
         ++issued;
       }
       if (*abort_flag) {
@@ -599,9 +619,8 @@ __global__ void __launch_bounds__(agt::THREADS, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(ROWS, (uint32_t)rows_b);
-      // descriptor of the first 16-column slice of stage 0's B tile; slice j of
-      // stage s adds s * stage_bytes + (j >> 2) * rows_b * 128 + (j & 3) * 32 bytes
+      const uint32_t idesc = idesc_u8s8_s32(ROWS, (uint32_t)rows_b);
+      // slice j (32 int8 of K) of stage s: box (j >> 2) of 128 bytes of K, + (j & 3) * 32 bytes
       const uint64_t bd0 = smem_desc(smem_u32(stage0), 16, 1024, 2);
       const uint32_t box16 = (uint32_t)(rows_b * 128) >> 4;
       const uint32_t stage16 = (uint32_t)plan.stage_bytes >> 4;
@@ -618,9 +637,9 @@ __global__ void __launch_bounds__(agt::THREADS, 1)
         const uint64_t bds = bd0 + (uint64_t)((uint32_t)s * stage16);
         const uint32_t a0 = tmem_base + D_COLS + (uint32_t)s * A_COLS;
 #pragma unroll
-        for (int j = 0; j < KSTEP / 16; ++j) {
+        for (int j = 0; j < KSTEP / 32; ++j) {
           const uint64_t bd = bds + (uint64_t)((uint32_t)(j >> 2) * box16 + (uint32_t)(j & 3) * 2u);
-          mma_ts(tmem_base, a0 + (uint32_t)(j * 8), bd, idesc, (i > 0 || j > 0) ? 1u : 0u);
+          mma_ts_i8(tmem_base, a0 + (uint32_t)(j * 8), bd, idesc, (i > 0 || j > 0) ? 1u : 0u);
         }
         mma_commit(&empty[s]);
       }
@@ -659,16 +678,16 @@ __global__ void __launch_bounds__(agt::THREADS, 1)
         w2[2] = __byte_perm(c2.y, 0u, 0x4140);
         w2[3] = __byte_perm(c2.y, 0u, 0x4342);
       }
-      uint32_t v[32];
+      uint32_t v[16];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const uint32_t a = (w1[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
         const uint32_t bb = (w2[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
         const uint32_t ea = lds32(table_s + table_off(a));
         const uint32_t eb = BPW > 2 ? lds32(table_s + table_off(bb)) : 0u;
-        decode_group<BPW>(a, bb, ea, eb, v + 4 * j);
+        decode_group_q8<BPW>(a, bb, ea, eb, v[2 * j], v[2 * j + 1]);
       }
-      tmem_st32(tmem_base + lane_bits + D_COLS + (uint32_t)s * A_COLS + (uint32_t)(part * 32), v);
+      tmem_st16(tmem_base + lane_bits + D_COLS + (uint32_t)s * A_COLS + (uint32_t)(part * 16), v);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -677,12 +696,22 @@ __global__ void __launch_bounds__(agt::THREADS, 1)
   }
 
   // ------------------------------------------------------------ epilogue ---
-  // Warps 2-5 hold row r of the 128 x rows_b accumulator (TMEM lane r); the
-  // token sums y[m] = D[r][2m] + D[r][2m + 1] (hi + lo) stay in registers.
+  // Warps 2-5 hold row r of the int32 accumulator (TMEM lane r).  They first
+  // stage the per-token steps and row sums (written by the transform kernel)
+  // in shared memory, then wait for the accumulator.
+  float* s_sc = reinterpret_cast<float*>(smem + plan.aux_off);      // [32]
+  int32_t* s_cs = reinterpret_cast<int32_t*>(smem + plan.aux_off + 128);  // [64]
+  float4* recv = reinterpret_cast<float4*>(smem + plan.recv_off);
   float y[32];
   const bool epi = warp >= 2 && warp < 6;
   const int er = (warp & 3) * 32 + lane;
   if (epi) {
+    if (warp == 2) {
+      s_sc[lane] = lane < M ? __ldg(tok_scale + lane) : 0.0f;
+      s_cs[lane] = lane < rows_b ? __ldg(colsum + lane) : 0;
+      s_cs[32 + lane] = 32 + lane < rows_b ? __ldg(colsum + 32 + lane) : 0;
+    }
+    asm volatile("bar.sync 1, 128;" ::: "memory");
     const bool have = nks > 0 && mbar_wait_sleep(acc_full, 0, abort_flag, status, kDevTimeoutMma);
     tc_fence_after();
     uint32_t dv[D_COLS];
@@ -692,19 +721,23 @@ __global__ void __launch_bounds__(agt::THREADS, 1)
         tmem_ld16(tmem_base + (uint32_t)c + ((uint32_t)((warp & 3) * 32) << 16),
                   *reinterpret_cast<uint32_t(*)[16]>(dv + c));
     tmem_ld_wait();
+    // the +128 bias of the weight bytes contributes 128 * (row sum of Xq) over the
+    // whole K; the cluster's partial tiles are summed, so rank 0 alone removes it
+    const int corr = crank == 0 ? 128 : 0;
 #pragma unroll
-    for (int m = 0; m < 32; ++m)
-      y[m] = (have && m < M) ? __uint_as_float(dv[2 * m]) + __uint_as_float(dv[2 * m + 1]) : 0.0f;
+    for (int m = 0; m < 32; ++m) {
+      if (have && m < M) {
+        const int d0 = (int)dv[2 * m] - corr * s_cs[2 * m];
+        const int d1 = (int)dv[2 * m + 1] - corr * s_cs[2 * m + 1];
+        y[m] = s_sc[m] * ((float)d0 + (float)d1 * (1.0f / 128.0f));
+      } else {
+        y[m] = 0.0f;
+      }
+    }
   }
-  // Every CTA of the cluster has finished with its stage area once all its
-  // threads arrive here; after the wait the peers may write into it.
-  tc_fence_before();
-  __syncthreads();
-  cluster_arrive();
-  cluster_wait();
   // Reduce-scatter: row r goes to the CTA owning rows [owner*R, owner*R + R),
-  // slot [source rank][row - owner*R] of its receive area (the stage area).
-  float4* recv = reinterpret_cast<float4*>(stage0);
+  // slot [source rank][row - owner*R] of its receive area.
+  cluster_wait();
   if (epi) {
     const int owner = er / R;
     const int slot = ((int)crank * R + (er - owner * R)) * chunks;
@@ -722,12 +755,13 @@ __global__ void __launch_bounds__(agt::THREADS, 1)
                       make_float4(y[4 * c], y[4 * c + 1], y[4 * c + 2], y[4 * c + 3]));
     }
   }
-  __syncthreads();   // local rows written
+  tc_fence_before();
+  __syncthreads();   // local rows written, every tensor-memory read done
   {
-    const bool got = mbar_wait_sleep(red_full, 0, abort_flag, status, kDevTimeoutCluster);
     const int r0 = (int)crank * R;
-    for (int e = threadIdx.x; e < R * chunks; e += blockDim.x) {
-      const int row = e % R, c = e / R;
+    if (threadIdx.x < R * chunks) {
+      const bool got = mbar_wait_sleep(red_full, 0, abort_flag, status, kDevTimeoutCluster);
+      const int row = threadIdx.x % R, c = threadIdx.x / R;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
       for (int src = 0; src < (int)ncl; ++src) {
         const float4 v4 = recv[(src * R + row) * chunks + c];
@@ -745,17 +779,17 @@ __global__ void __launch_bounds__(agt::THREADS, 1)
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, 512);
+    tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 
 template <int BPW>
-static cudaError_t launch_tm(const DeviceCodebook& cb, const ActGemmArgs& a, int sm_count,
+static cudaError_t launch_q8(const DeviceCodebook& cb, const ActQ8Args& a, int sm_count,
                              cudaStream_t st) {
-  using namespace agt;
+  using namespace agq;
   CUtensorMap tb, ti1, ti2;
-  if (!make_tmap_2d(&tb, a.Xt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.rows_b,
-                    (uint64_t)a.K, (uint32_t)a.rows_b, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+  if (!make_tmap_2d(&tb, a.Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.rows_b,
+                    (uint64_t)a.K, (uint32_t)a.rows_b, 128, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   if (!make_tmap_2d(&ti1, a.idx1, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)a.N,
                     (uint64_t)(a.K / 8), ROWS, GROUPS, CU_TENSOR_MAP_SWIZZLE_64B))
@@ -771,7 +805,7 @@ static cudaError_t launch_tm(const DeviceCodebook& cb, const ActGemmArgs& a, int
   } else {
     ti2 = ti1;
   }
-  const TmPlan plan = tm_plan(a.rows_b, BPW);
+  const Q8Plan plan = q8_plan(a.rows_b, BPW);
   if (plan.stages < 2 || plan.total > kMaxDynSmem) return cudaErrorInvalidValue;
   const int tiles = (int)((a.N + ROWS - 1) / ROWS);
   const int ksteps = (int)(a.K / KSTEP);
@@ -791,23 +825,24 @@ static cudaError_t launch_tm(const DeviceCodebook& cb, const ActGemmArgs& a, int
   attr[1].val.programmaticStreamSerializationAllowed = a.pdl ? 1 : 0;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  cudaError_t e = ensure_smem_limit(k_act_gemm_tm<BPW>, kMaxDynSmem);
+  cudaError_t e = ensure_smem_limit(k_act_gemm_q8<BPW>, kMaxDynSmem);
   if (e != cudaSuccess) return e;
-  e = cudaLaunchKernelEx(&cfg, k_act_gemm_tm<BPW>, tb, ti1, ti2, cb, (int)a.M, (int)a.N,
-                         (int)a.K, a.rows_b, a.alpha, a.Y, a.early_codes);
+  e = cudaLaunchKernelEx(&cfg, k_act_gemm_q8<BPW>, tb, ti1, ti2, cb, (int)a.M, (int)a.N,
+                         (int)a.K, a.rows_b, a.alpha, a.scales, a.colsum, a.Y, a.early_codes);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
-// Tensor-memory variant: the 256-wide kernel above when the shape allows it
-// (up to 32 tokens, K a multiple of 256), else the generic kernel.
+cudaError_t launch_act_gemm_q8(const DeviceCodebook& cb, const ActQ8Args& a, int sm_count,
+                               cudaStream_t st) {
+  if (a.bpw == 2) return launch_q8<2>(cb, a, sm_count, st);
+  if (a.bpw == 3) return launch_q8<3>(cb, a, sm_count, st);
+  return launch_q8<4>(cb, a, sm_count, st);
+}
+
 cudaError_t launch_act_gemm(const DeviceCodebook& cb, const ActGemmArgs& a, int sm_count,
                             cudaStream_t st) {
-  const bool tm = a.variant == 1 && a.rows_b <= (int)agt::D_COLS && (a.K % agt::KSTEP) == 0;
-  if (!tm) return launch_act_gemm_generic(cb, a, sm_count, st);
-  if (a.bpw == 2) return launch_tm<2>(cb, a, sm_count, st);
-  if (a.bpw == 3) return launch_tm<3>(cb, a, sm_count, st);
-  return launch_tm<4>(cb, a, sm_count, st);
+  return launch_act_gemm_generic(cb, a, sm_count, st);
 }
 
 }  // namespace e8

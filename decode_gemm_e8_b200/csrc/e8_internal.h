@@ -65,6 +65,57 @@ struct ActGemmArgs {
 cudaError_t launch_act_gemm(const DeviceCodebook& cb, const ActGemmArgs& a, int sm_count,
                             cudaStream_t st);
 
+// int8 path for up to 32 tokens: Xq int8 [rows_b][K] (token m: rows 2m, 2m + 1),
+// per-token steps and per-row column sums from launch_act_q8.
+struct ActQ8Args {
+  const int8_t* Xq;
+  const float* scales;   // [M]
+  const int32_t* colsum; // [rows_b]
+  int64_t M, N, K;
+  int rows_b;
+  const uint16_t* idx1;
+  const void* idx2;
+  int bpw;
+  float alpha;
+  float* Y;
+  int pdl;
+  int early_codes;
+};
+cudaError_t launch_act_gemm_q8(const DeviceCodebook& cb, const ActQ8Args& a, int sm_count,
+                               cudaStream_t st);
+cudaError_t launch_act_q8(const uint16_t* X, int64_t M, int64_t K, uint64_t seed, int8_t* Xq,
+                          float* scales, int32_t* colsum, int64_t rows, cudaStream_t st,
+                          int pdl);
+
+// Layout of the int8 activation buffer: Xq [rows][K] int8, then the per-token
+// steps (fp32 [M]) and the per-row column sums (int32 [rows]), each part
+// starting on a 256-byte boundary.
+struct Q8Layout {
+  size_t scales_off, colsum_off, total;
+};
+inline Q8Layout q8_layout(int64_t M, int64_t K, int64_t rows) {
+  auto r256 = [](size_t x) { return (x + 255) & ~size_t(255); };
+  Q8Layout l;
+  l.scales_off = r256((size_t)rows * (size_t)K);
+  l.colsum_off = l.scales_off + r256((size_t)M * 4);
+  l.total = l.colsum_off + r256((size_t)rows * 4);
+  return l;
+}
+// Shapes served by the int8 path: up to 32 tokens, K a multiple of 256 whose
+// Hadamard block lies in 256..4096, K <= 32768.
+inline bool q8_eligible(int64_t M, int64_t K) {
+  const int64_t nh = K & (-K);
+  return M >= 1 && M <= 32 && (K % 256) == 0 && nh >= 256 && nh <= 4096 && K <= 32768;
+}
+
+// Activation-side GEMM (E8_GEMM_ACT_RHT / _SMEM) on caller-provided scratch of
+// act_scratch_bytes() bytes: the transform and the fused kernel.
+size_t act_scratch_bytes(int64_t M, int64_t K, int smem_variant);
+cudaError_t run_act_gemm(const e8_codebook* cb, const uint16_t* X, int64_t M,
+                         const uint16_t* idx1, const void* idx2, int64_t N, int64_t K, int bpw,
+                         uint64_t seed, float alpha, float* Y, int smem_variant, void* scratch,
+                         cudaStream_t st);
+
 // Dense Y[M][N] fp32 = X[M][K] bf16 * W[N][K]^T bf16 on tcgen05.
 cudaError_t launch_dense_gemm(const uint16_t* X, int64_t M, const uint16_t* W, int64_t N,
                               int64_t K, float* Y, uint32_t* status, int sm_count,

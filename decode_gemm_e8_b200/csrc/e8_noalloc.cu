@@ -11,9 +11,9 @@
 // neither a workspace argument nor any allocation.
 //
 // Limits and rules (also stated in include/e8.h):
-//   - the scratch holds kNoallocXtElems bf16 values (2 MiB): rows * K must not
-//     exceed it, where rows = e8_gemm_xt_rows(M); larger requests return
-//     E8_EWORKSPACE without launching anything;
+//   - the scratch is 2 MiB: requests whose activation buffer (the workspace
+//     e8_gemm would need for E8_GEMM_ACT_RHT) is larger return E8_EWORKSPACE
+//     without launching anything;
 //   - every GPU that loads the library keeps this 2 MiB until the process exits;
 //   - all calls share the one array and it keeps the last call's contents; the
 //     padding rows that must be zero are cleared by every call, but two calls
@@ -34,6 +34,7 @@
 namespace {
 
 constexpr int64_t kNoallocXtElems = 1 << 20;   // 1 Mi bf16 = 2 MiB
+constexpr int64_t kNoallocBytes = kNoallocXtElems * 2;
 constexpr int kMaxDevices = 64;
 
 // Device-resident scratch: transformed activations of the last call.
@@ -76,36 +77,17 @@ extern "C" int e8_gemm_act_noalloc(const e8_codebook* cb, const uint16_t* X, int
   if ((bpw == 2) != (idx2 == nullptr)) return E8_EINVAL;
   if (M > 64 || (K % 128) != 0 || N > INT32_MAX || K > INT32_MAX) return E8_EINVAL;
   if (M == 0 || N == 0) return E8_OK;
-  const int64_t rows = (2 * M + 15) / 16 * 16;
-  if (rows * K > kNoallocXtElems) return E8_EWORKSPACE;
+  const size_t need = e8::act_scratch_bytes(M, K, 0);
+  if (need > (size_t)kNoallocBytes) return E8_EWORKSPACE;
   if (!X || !idx1 || !Y || !aligned16(X) || !aligned16(idx1) || !aligned16(Y) ||
       (idx2 && !aligned16(idx2)))
     return E8_EINVAL;
   uint16_t* xt = nullptr;
   int rc = scratch_address(dev, &xt);
   if (rc != E8_OK) return rc;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (e8::launch_act_rht(X, M, K, rht_seed, xt, rows, st, 1) != cudaSuccess) return E8_ECUDA;
-  e8::DeviceCodebook d;
-  d.vecs = cb->vecs;
-  d.table = cb->table;
-  d.hkeys = cb->hkeys;
-  d.hvals = cb->hvals;
-  d.status = cb->status;
-  e8::ActGemmArgs a;
-  a.Xt = xt;
-  a.M = M;
-  a.N = N;
-  a.K = K;
-  a.rows_b = (int)rows;
-  a.idx1 = idx1;
-  a.idx2 = idx2;
-  a.bpw = bpw;
   const int m = bpw == 2 ? 2 : (bpw == 3 ? 4 : 8);
-  a.alpha = (float)((double)scale / ((double)m * std::sqrt((double)nh)));
-  a.Y = Y;
-  a.variant = 1;
-  a.pdl = 1;
-  a.early_codes = 1;
-  return e8::launch_act_gemm(d, a, cb->sm_count, st) == cudaSuccess ? E8_OK : E8_ECUDA;
+  const float alpha = (float)((double)scale / ((double)m * std::sqrt((double)nh)));
+  const cudaError_t e = e8::run_act_gemm(cb, X, M, idx1, idx2, N, K, bpw, rht_seed, alpha, Y, 0,
+                                         xt, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? E8_OK : E8_ECUDA;
 }

@@ -72,7 +72,8 @@ extern "C" {
 /* GEMM modes (e8_gemm `mode`, and `op` of e8_workspace_bytes). */
 #define E8_GEMM_AUTO 0          /* ACT_RHT for M <= 64 and K % 128 == 0, else DECODED_W */
 #define E8_GEMM_ACT_RHT 1       /* transform on the activations, codes decoded on chip into
-                                   tensor memory, fused tcgen05 GEMM (M <= 64, K % 128 == 0) */
+                                   tensor memory, fused tcgen05 GEMM (M <= 64, K % 128 == 0);
+                                   int8 MMA for the shapes of e8_act_rht_q8, bf16 otherwise */
 #define E8_GEMM_DECODED_W 2     /* decode to a bf16 workspace, then a dense tcgen05 GEMM */
 #define E8_GEMM_ACT_RHT_SMEM 3  /* as ACT_RHT, decoded operand staged in shared memory */
 #define E8_GEMM_SIMT 4          /* decode to bf16, CUDA-core fp32 GEMM (diagnostic) */
@@ -135,18 +136,34 @@ int e8_gemm(const e8_codebook* cb, const uint16_t* X, int64_t M, const uint16_t*
             const void* idx2, int64_t N, int64_t K, int bpw, uint64_t rht_seed, float scale,
             float* Y, int mode, void* workspace, size_t ws_bytes, void* stream);
 
-/* Second half of E8_GEMM_ACT_RHT on activations already transformed by
- * e8_act_rht: Y fp32 [M][N] = alpha * (Xt[2m] + Xt[2m+1]) * Z^T, with Z the
- * integer codebook vectors decoded on chip and alpha from `scale`.  Xt is bf16
- * [rows][K] with rows == e8_gemm_xt_rows(M) (2M rounded up to a multiple of
- * 16; padding rows must be zero, as e8_act_rht leaves them).  One transform can
- * serve every weight matrix that shares K and rht_seed.  mode: E8_GEMM_ACT_RHT
- * (or AUTO) or E8_GEMM_ACT_RHT_SMEM; M <= 64, K % 128 == 0.  No workspace. */
-int e8_gemm_xt(const e8_codebook* cb, const uint16_t* Xt, int64_t rows, int64_t M,
-               const uint16_t* idx1, const void* idx2, int64_t N, int64_t K, int bpw,
-               float scale, float* Y, int mode, void* stream);
+/* int8 activation transform, first half of E8_GEMM_ACT_RHT for up to 32
+ * tokens: X bf16 [M][K] -> one buffer of e8_act_q8_bytes(M, K) bytes holding
+ *   Xq int8 [rows][K], rows = e8_gemm_xt_rows(M): row 2m = q0 and row 2m + 1 =
+ *     q1 of token m, where xt = FWHT(D x_m) per Hadamard block,
+ *     s_m = max|xt| / 127, q0 = rint(xt / s_m), q1 = rint((xt - q0 s_m) 128 / s_m),
+ *     so xt = s_m (q0 + q1 / 128) within s_m / 256; padding rows are zero;
+ *   then s_m (fp32 [M]) and the row sums of Xq (int32 [rows]), each part
+ *     starting on a 256-byte boundary after the previous one.
+ * Shapes: 1 <= M <= 32, K a multiple of 256 whose Hadamard block is 256..4096,
+ * K <= 32768 (else E8_EINVAL). */
+int e8_act_rht_q8(const uint16_t* X, int64_t M, int64_t K, uint64_t rht_seed, void* buf,
+                  void* stream);
 
-/* Row count of the transformed-activation buffer for M tokens (see e8_gemm_xt). */
+/* Size in bytes of the e8_act_rht_q8 buffer (0 if the shape is not served). */
+size_t e8_act_q8_bytes(int64_t M, int64_t K);
+
+/* Second half of E8_GEMM_ACT_RHT: the fused decode + int8 tensor-core GEMM on
+ * a buffer written by e8_act_rht_q8 for the same M, K and rht_seed:
+ * Y fp32 [M][N] = alpha * s_m * ((q0 + q1 / 128) . z) over each weight row, z
+ * the integer codebook vectors decoded on chip.  One transform can serve every
+ * weight matrix that shares K and rht_seed (for instance q, k and v).  Same
+ * shape limits as e8_act_rht_q8.  No workspace. */
+int e8_gemm_xt(const e8_codebook* cb, const void* xq, int64_t M, const uint16_t* idx1,
+               const void* idx2, int64_t N, int64_t K, int bpw, float scale, float* Y,
+               void* stream);
+
+/* Row count of the transformed-activation buffers for M tokens: 2M rounded up to
+ * a multiple of 16. */
 int e8_gemm_xt_rows(int64_t M);
 
 /* E8_GEMM_ACT_RHT without a workspace, for callers that may not allocate device
@@ -157,8 +174,8 @@ int e8_gemm_xt_rows(int64_t M);
  * Same arguments and result as e8_gemm with mode E8_GEMM_ACT_RHT, minus the
  * workspace.  The transformed activations go to a fixed 2 MiB array compiled
  * into the library (every GPU that loads the library holds it until the process
- * exits): requests with e8_gemm_xt_rows(M) * K > 1048576 return E8_EWORKSPACE
- * and launch nothing.  Nothing is allocated.  All calls share that array and it
+ * exits): requests for which e8_workspace_bytes(E8_GEMM_ACT_RHT, ...) exceeds
+ * 2 MiB return E8_EWORKSPACE and launch nothing.  Nothing is allocated.  All calls share that array and it
  * keeps the last call's contents (each call clears what must start at zero);
  * calls whose kernels overlap on the GPU race on it, so order them on one
  * stream.  The first call on a device looks up the array's address on that

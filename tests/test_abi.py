@@ -46,10 +46,14 @@ def test_workspace_sizes(lib):
     N, K = 4096, 4096
     assert e8.e8_workspace_bytes(e8.E8_OP_ENCODE, 0, N, K, 4) == 256 + 48 * N * K // 8
     assert e8.e8_workspace_bytes(e8.E8_GEMM_DECODED_W, 4096, N, K, 3) == N * K * 2
-    # hi and lo rows for 16 tokens: 32 rows of K bf16
-    assert e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT, 16, N, K, 4) == 32 * K * 2
-    assert e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT, 1, N, K, 4) == 16 * K * 2
-    assert e8.e8_workspace_bytes(e8.E8_GEMM_AUTO, 16, N, K, 4) == 32 * K * 2
+    # int8 pieces for 16 tokens: 32 rows of K bytes, 16 steps, 32 row sums
+    assert e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT, 16, N, K, 4) == 32 * K + 256 + 256
+    assert e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT, 1, N, K, 4) == 16 * K + 256 + 256
+    assert e8.e8_workspace_bytes(e8.E8_GEMM_AUTO, 16, N, K, 4) == 32 * K + 256 + 256
+    assert e8.e8_act_q8_bytes(16, K) == 32 * K + 512
+    # bf16 hi and lo rows where the int8 path does not apply (more than 32 tokens)
+    assert e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT, 40, N, K, 4) == 80 * K * 2
+    assert e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT_SMEM, 16, N, K, 4) == 32 * K * 2
     assert e8.e8_workspace_bytes(e8.E8_GEMM_AUTO, 4096, N, K, 4) == N * K * 2
     # invalid arguments give 0
     assert e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT, 16, N, 100, 4) == 0

@@ -161,10 +161,9 @@ def test_gemm_xt_matches_gemm_and_graph_capture(gcb):
     i1, i2 = _layer_codes(gcb, W, lay.bpw, lay.rht_seed, s)
     a = e8.e8_gemm(gcb, X, i1, i2, lay.N, lay.K, lay.bpw, lay.rht_seed, s,
                    mode=e8.E8_GEMM_ACT_RHT)
-    rows = e8.e8_gemm_xt_rows(16)
-    assert rows == 32
-    Xt = e8.e8_act_rht(X, lay.rht_seed, rows=rows)
-    b = e8.e8_gemm_xt(gcb, Xt, 16, i1, i2, lay.N, lay.K, lay.bpw, s)
+    assert e8.e8_gemm_xt_rows(16) == 32
+    xq = e8.e8_act_rht_q8(X, lay.rht_seed)
+    b = e8.e8_gemm_xt(gcb, xq, 16, i1, i2, lay.N, lay.K, lay.bpw, s)
     assert np.array_equal(gu.to_np(a).view(np.uint32), gu.to_np(b).view(np.uint32))
     # the same call captured in a CUDA graph and replayed
     Y = torch.empty_like(a)
@@ -183,3 +182,30 @@ def test_gemm_xt_matches_gemm_and_graph_capture(gcb):
     torch.cuda.synchronize()
     assert np.array_equal(gu.to_np(Y).view(np.uint32), gu.to_np(a).view(np.uint32))
     assert e8.e8_sync_status(gcb) == e8.E8_OK
+
+
+@pytest.mark.parametrize("M,K", [(16, 4096), (3, 3072), (32, 256), (1, 12288)])
+def test_act_rht_q8_pieces(gcb, M, K):
+    # xt = s_m (q0 + q1 / 128) within s_m / 256, s_m = max|xt| / 127, column sums
+    X = synth.activations_bf16(M, K, 40 + M)
+    buf = gu.to_np(e8.e8_act_rht_q8(gu.bf16_dev(X), 17))
+    rows = e8.e8_gemm_xt_rows(M)
+    assert len(buf) >= e8.e8_act_q8_bytes(M, K)
+    xq = buf[:rows * K].view(np.int8).reshape(rows, K).astype(np.int64)
+    off_s = (rows * K + 255) // 256 * 256
+    off_c = off_s + (M * 4 + 255) // 256 * 256
+    sc = buf[off_s:off_s + 4 * M].view(np.float32).astype(np.float64)
+    cs = buf[off_c:off_c + 4 * rows].view(np.int32)
+    x = synth.bf16_bits_to_f32(X).astype(np.float64)
+    d = orc.signs(17, K).astype(np.float64)
+    from tests import indep
+    nh = orc.hadamard_block(K)
+    H = indep.sylvester(nh).astype(np.float64)
+    ref = np.concatenate([(x * d[None, :])[:, b:b + nh] @ H for b in range(0, K, nh)], axis=1)
+    amax = np.abs(ref).max(1)
+    assert np.allclose(sc, amax / 127, rtol=1e-5)
+    rec = sc[:, None] * (xq[0:2 * M:2] + xq[1:2 * M:2] / 128.0)
+    assert np.all(np.abs(rec - ref) <= sc[:, None] / 256 * 1.01 + 1e-6)
+    assert np.all(np.abs(xq[1:2 * M:2]) <= 64)
+    assert np.array_equal(cs, xq.sum(1))
+    assert not xq[2 * M:].any()
