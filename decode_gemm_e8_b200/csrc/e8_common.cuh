@@ -87,7 +87,19 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
   return ok != 0;
 }
 
-// Same contract as mbar_wait_bounded, sleeping between polls.
+__device__ __forceinline__ uint32_t ld_shared_volatile(const volatile uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.volatile.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32((const void*)p)));
+  return v;
+}
+__device__ __forceinline__ void st_shared_volatile(volatile uint32_t* p, uint32_t v) {
+  asm volatile("st.volatile.shared.u32 [%0], %1;" ::"r"(smem_u32((const void*)p)), "r"(v)
+               : "memory");
+}
+
+// Same contract as mbar_wait_bounded, sleeping in the hardware between polls
+// (the thread wakes when the phase completes); the abort flag lives in shared
+// memory and is read with an explicit shared load.
 __device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity,
                                                 volatile uint32_t* abort_flag, uint32_t* status,
                                                 uint32_t code) {
@@ -95,9 +107,9 @@ __device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity,
   const uint64_t t0 = global_timer_ns();
   for (;;) {
     if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
-    if (*abort_flag) return false;
+    if (ld_shared_volatile(abort_flag)) return false;
     if (global_timer_ns() - t0 > kWaitLimitNs) {
-      *abort_flag = 1u;
+      st_shared_volatile(abort_flag, 1u);
       if (status) atomicOr(status, code);
       return false;
     }

@@ -589,7 +589,7 @@ __global__ void __launch_bounds__(agq::THREADS, 1)
         const int s = i % S;
         const uint32_t round = (uint32_t)(i / S);
         if (round > 0 &&
-            !mbar_wait_bounded(&empty[s], (round - 1u) & 1u, abort_flag, status, kDevTimeoutEmpty))
+            !mbar_wait_sleep(&empty[s], (round - 1u) & 1u, abort_flag, status, kDevTimeoutEmpty))
           break;
         uint8_t* sb = stage0 + s * plan.stage_bytes;
         uint8_t* si1 = sb + plan.b_bytes;
@@ -604,7 +604,7 @@ __global__ void __launch_bounds__(agq::THREADS, 1)
         tma_load_2d(sb + rows_b * 128, &tmB, &full_b[s], k0 + 128, 0);
         ++issued;
       }
-      if (*abort_flag) {
+      if (ld_shared_volatile(abort_flag)) {
         uint64_t t0 = global_timer_ns();
         while (!mbar_try_wait(table_full, 0))
           if (global_timer_ns() - t0 > 100000000ull) break;
@@ -628,8 +628,8 @@ __global__ void __launch_bounds__(agq::THREADS, 1)
       for (int i = 0; i < nks && ok; ++i) {
         const int s = i % S;
         const uint32_t ph = (uint32_t)(i / S) & 1u;
-        if (!mbar_wait_bounded(&full_a[s], ph, abort_flag, status, kDevTimeoutFull) ||
-            !mbar_wait_bounded(&full_b[s], ph, abort_flag, status, kDevTimeoutFull)) {
+        if (!mbar_wait_sleep(&full_a[s], ph, abort_flag, status, kDevTimeoutFull) ||
+            !mbar_wait_sleep(&full_b[s], ph, abort_flag, status, kDevTimeoutFull)) {
           ok = false;
           break;
         }
