@@ -56,6 +56,7 @@ cudaError_t run_act_gemm(const e8_codebook* cb, const uint16_t* X, int64_t M,
   DeviceCodebook d;
   d.vecs = cb->vecs;
   d.table = cb->table;
+  d.h8table = cb->h8table;
   d.hkeys = cb->hkeys;
   d.hvals = cb->hvals;
   d.status = cb->status;
@@ -142,6 +143,7 @@ e8::DeviceCodebook dev_view(const e8_codebook* cb) {
   e8::DeviceCodebook d;
   d.vecs = cb->vecs;
   d.table = cb->table;
+  d.h8table = cb->h8table;
   d.hkeys = cb->hkeys;
   d.hvals = cb->hvals;
   d.status = cb->status;
@@ -196,6 +198,7 @@ int e8_codebook_build(e8_codebook** out, int device) {
   auto fail = [&](int code) {
     cudaFree(cb->vecs);
     cudaFree(cb->table);
+    cudaFree(cb->h8table);
     cudaFree(cb->hkeys);
     cudaFree(cb->hvals);
     cudaFree(cb->status);
@@ -205,6 +208,7 @@ int e8_codebook_build(e8_codebook** out, int device) {
   };
   if (cudaMalloc(&cb->vecs, (size_t)e8::kCbSize * 8) != cudaSuccess) return fail(E8_ENOMEM);
   if (cudaMalloc(&cb->table, kTableAlloc) != cudaSuccess) return fail(E8_ENOMEM);
+  if (cudaMalloc(&cb->h8table, kTableAlloc) != cudaSuccess) return fail(E8_ENOMEM);
   if (cudaMalloc(&cb->hkeys, e8::kHashSlots * sizeof(uint32_t)) != cudaSuccess)
     return fail(E8_ENOMEM);
   if (cudaMalloc(&cb->hvals, e8::kHashSlots * sizeof(uint32_t)) != cudaSuccess)
@@ -214,8 +218,9 @@ int e8_codebook_build(e8_codebook** out, int device) {
   if (cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking) != cudaSuccess) return fail(E8_ECUDA);
   cudaMemsetAsync(cb->status, 0, 16, st);
   cudaMemsetAsync(cb->table, 0, kTableAlloc, st);
-  int reps = e8::build_codebook_tables(cb->vecs, cb->table, cb->hkeys, cb->hvals, &cb->max_probe,
-                                       st);
+  cudaMemsetAsync(cb->h8table, 0, kTableAlloc, st);
+  int reps = e8::build_codebook_tables(cb->vecs, cb->table, cb->h8table, cb->hkeys, cb->hvals,
+                                       &cb->max_probe, st);
   cudaStreamDestroy(st);
   // the E8 shells of squared norm 2..12 hold 117360 vectors, half of them
   // positive representatives
@@ -233,6 +238,7 @@ void e8_codebook_free(e8_codebook* cb) {
   cudaSetDevice(cb->device);
   cudaFree(cb->vecs);
   cudaFree(cb->table);
+  cudaFree(cb->h8table);
   cudaFree(cb->hkeys);
   cudaFree(cb->hvals);
   cudaFree(cb->status);
@@ -331,7 +337,8 @@ int e8_decode_to_bf16(const e8_codebook* cb, const uint16_t* idx1, const void* i
     return E8_EINVAL;
   const int64_t nh = e8::hadamard_block(K);
   cudaError_t e = e8::launch_decode(dev_view(cb), idx1, idx2, N, K, bpw, rht_seed,
-                                    alpha_of(scale, nh, bpw), W_dec, (cudaStream_t)stream);
+                                    alpha_of(scale, nh, bpw), W_dec, cb->sm_count,
+                                    (cudaStream_t)stream);
   return cuda_status(e);
 }
 
@@ -376,7 +383,7 @@ int e8_gemm(const e8_codebook* cb, const uint16_t* X, int64_t M, const uint16_t*
     return cuda_status(e);
   }
   uint16_t* Wd = static_cast<uint16_t*>(workspace);
-  e = e8::launch_decode(d, idx1, idx2, N, K, bpw, rht_seed, alpha, Wd, st);
+  e = e8::launch_decode(d, idx1, idx2, N, K, bpw, rht_seed, alpha, Wd, cb->sm_count, st);
   if (e != cudaSuccess) return E8_ECUDA;
   if (mode == E8_GEMM_SIMT)
     e = e8::launch_simt_gemm(X, M, Wd, N, K, Y, st);

@@ -141,16 +141,45 @@ __global__ void k_cb_hash(const uint32_t* table, uint32_t* hkeys, uint32_t* hval
   }
 }
 
-// Builds vecs, table and the hash on the current device (synchronous).
+// Transformed pair table: slot q holds H8 v / 4 (v the slot's vector, H8 the
+// natural-order 8-point Walsh-Hadamard matrix).  A slot whose transform is not
+// a multiple of 4 in [-16, 16] is counted in *bad (none is expected).
+__global__ void k_cb_h8(const uint32_t* table, uint32_t* h8, int* bad) {
+  int q = blockIdx.x * blockDim.x + threadIdx.x;
+  if (q >= kPairSlots) return;
+  const uint32_t e = table[q];
+  int v[8];
+  for (int j = 0; j < 4; ++j) {
+    v[j] = (int)((e >> (8 * j)) & 0xFu) - 8;
+    v[j + 4] = (int)((e >> (8 * j + 4)) & 0xFu) - 8;
+  }
+  for (int h = 1; h < 8; h <<= 1)
+    for (int i = 0; i < 8; ++i)
+      if ((i & h) == 0) {
+        const int a = v[i], b = v[i + h];
+        v[i] = a + b;
+        v[i + h] = a - b;
+      }
+  bool ok = true;
+  for (int j = 0; j < 8; ++j) {
+    ok = ok && (v[j] % 4 == 0) && v[j] >= -16 && v[j] <= 16;
+    v[j] /= 4;
+  }
+  if (!ok) atomicAdd(bad, 1);
+  h8[q] = pack_vec(v);
+}
+
+// Builds vecs, table, the transformed table and the hash on the current
+// device (synchronous).
 // Returns the number of positive representatives found over all shells
 // (58680 for the E8 shells of norm 2..12), or -1 on a CUDA error.
-int build_codebook_tables(int8_t* d_vecs, uint32_t* d_table, uint32_t* d_hkeys,
-                          uint32_t* d_hvals, int* h_max_probe, cudaStream_t st) {
+int build_codebook_tables(int8_t* d_vecs, uint32_t* d_table, uint32_t* d_h8table,
+                          uint32_t* d_hkeys, uint32_t* d_hvals, int* h_max_probe, cudaStream_t st) {
   int *d_counts = nullptr, *d_offsets = nullptr, *d_scalars = nullptr;
   if (cudaMalloc(&d_counts, kCells * sizeof(int)) != cudaSuccess) return -1;
   if (cudaMalloc(&d_offsets, kCells * sizeof(int)) != cudaSuccess) return -1;
-  if (cudaMalloc(&d_scalars, 2 * sizeof(int)) != cudaSuccess) return -1;
-  cudaMemsetAsync(d_scalars, 0, 2 * sizeof(int), st);
+  if (cudaMalloc(&d_scalars, 3 * sizeof(int)) != cudaSuccess) return -1;
+  cudaMemsetAsync(d_scalars, 0, 3 * sizeof(int), st);
   cudaMemsetAsync(d_hkeys, 0, kHashSlots * sizeof(uint32_t), st);
   cudaMemsetAsync(d_hvals, 0, kHashSlots * sizeof(uint32_t), st);
   const int tpb = 128, nb = (kCells + tpb - 1) / tpb;
@@ -159,13 +188,15 @@ int build_codebook_tables(int8_t* d_vecs, uint32_t* d_table, uint32_t* d_hkeys,
   k_cb_emit<<<nb, tpb, 0, st>>>(d_offsets, d_vecs, d_table);
   k_cb_hash<<<(kNumPosReps + 255) / 256, 256, 0, st>>>(d_table, d_hkeys, d_hvals,
                                                        d_scalars + 1);
-  int h[2] = {0, 0};
+  k_cb_h8<<<(kPairSlots + 255) / 256, 256, 0, st>>>(d_table, d_h8table, d_scalars + 2);
+  int h[3] = {0, 0, 0};
   cudaMemcpyAsync(h, d_scalars, sizeof(h), cudaMemcpyDeviceToHost, st);
   cudaError_t e = cudaStreamSynchronize(st);
   cudaFree(d_counts);
   cudaFree(d_offsets);
   cudaFree(d_scalars);
   if (e != cudaSuccess || cudaGetLastError() != cudaSuccess) return -1;
+  if (h[2] != 0) return -1;
   if (h_max_probe) *h_max_probe = h[1];
   return h[0];
 }

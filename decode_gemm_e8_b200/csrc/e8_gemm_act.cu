@@ -439,44 +439,6 @@ __device__ __forceinline__ uint32_t sw64_off(int r, int part) {
 // Byte offset, inside the pair table, of the entry of codebook index i.
 __device__ __forceinline__ uint32_t table_off(uint32_t i) { return ((i + 1u) >> 1) << 2; }
 
-// Packed decode of one group into 8 unsigned bytes z + 128 (two words, the
-// coordinates 0..3 and 4..7).  ea / eb: pair-table entries of the stage-1 and
-// stage-2 indices (8 nibbles v + 8); the sign of a stage is set when its index
-// is even (index 0 is the zero vector, whose sign does not matter).  With
-// B = v + 8 in [2, 14], the negated value's biased byte is B ^ 31 = 23 - v,
-// so one XOR per word applies a stage's sign and a per-group constant fixes
-// the bias:  byte = mul (B1 or B1 ^ 31) + (B2 or B2 ^ 31) + c(s1, s2) = z + 128.
-template <int BPW>
-__device__ __forceinline__ void decode_group_q8(uint32_t i1, uint32_t i2, uint32_t ea, uint32_t eb,
-                                                uint32_t& lo, uint32_t& hi) {
-  const uint32_t s1 = (~i1) & 1u;
-  const uint32_t m1 = s1 * 0x1F1F1F1Fu;
-  const uint32_t lo1 = (ea & 0x0F0F0F0Fu) ^ m1;
-  const uint32_t hi1 = ((ea >> 4) & 0x0F0F0F0Fu) ^ m1;
-  if (BPW == 2) {
-    // v + 128: B + 120, or (23 - v) + 105 = -v + 128
-    const uint32_t c = 0x78787878u - s1 * 0x0F0F0F0Fu;
-    lo = lo1 + c;
-    hi = hi1 + c;
-  } else {
-    const uint32_t s2 = (~i2) & 1u;
-    const uint32_t m2 = s2 * 0x1F1F1F1Fu;
-    const uint32_t lo2 = (eb & 0x0F0F0F0Fu) ^ m2;
-    const uint32_t hi2 = ((eb >> 4) & 0x0F0F0F0Fu) ^ m2;
-    if (BPW == 4) {
-      // 4 (+-v1) + (+-v2) + 128
-      const uint32_t c = 0x58585858u - s1 * 0x3C3C3C3Cu - s2 * 0x0F0F0F0Fu;
-      lo = lo1 * 4u + lo2 + c;
-      hi = hi1 * 4u + hi2 + c;
-    } else {
-      // 2 (+-v1) + (+-v2) + 128
-      const uint32_t c = 0x68686868u - s1 * 0x1E1E1E1Eu - s2 * 0x0F0F0F0Fu;
-      lo = lo1 * 2u + lo2 + c;
-      hi = hi1 * 2u + hi2 + c;
-    }
-  }
-}
-
 __device__ __forceinline__ void mma_ts_i8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                           uint32_t idesc, uint32_t accumulate) {
   asm volatile(

@@ -12,6 +12,7 @@ struct e8_codebook {
   int sm_count;
   int8_t* vecs;
   uint32_t* table;
+  uint32_t* h8table;
   uint32_t* hkeys;
   uint32_t* hvals;
   uint32_t* status;
@@ -29,8 +30,8 @@ struct WorkItem {
 };
 static_assert(sizeof(WorkItem) == 48, "WorkItem layout");
 
-int build_codebook_tables(int8_t* d_vecs, uint32_t* d_table, uint32_t* d_hkeys, uint32_t* d_hvals,
-                          int* h_max_probe, cudaStream_t st);
+int build_codebook_tables(int8_t* d_vecs, uint32_t* d_table, uint32_t* d_h8table,
+                          uint32_t* d_hkeys, uint32_t* d_hvals, int* h_max_probe, cudaStream_t st);
 
 int encode_elems_per_cta(int nh);
 cudaError_t launch_encode(const DeviceCodebook& cb, const float* W, int64_t N, int64_t K, int bpw,
@@ -40,7 +41,7 @@ cudaError_t launch_encode(const DeviceCodebook& cb, const float* W, int64_t N, i
 
 cudaError_t launch_decode(const DeviceCodebook& cb, const uint16_t* idx1, const void* idx2,
                           int64_t N, int64_t K, int bpw, uint64_t seed, float alpha,
-                          uint16_t* Wdec, cudaStream_t st);
+                          uint16_t* Wdec, int sm_count, cudaStream_t st);
 
 // X [M][K] bf16 -> Xt [rows][K] bf16: rows [0, M) hi parts, [M, 2M) lo parts of
 // FWHT(D x), rows [2M, rows) zero.

@@ -163,7 +163,8 @@ def _random_codes(N, K, bpw, seed):
 
 
 @pytest.mark.parametrize("bpw,N,K", [(2, 256, 256), (3, 33, 3072), (4, 17, 4096), (4, 5, 14336),
-                                     (3, 9, 12288), (2, 3, 32768), (4, 130, 264), (2, 1, 8)])
+                                     (3, 9, 12288), (2, 3, 32768), (4, 130, 264), (2, 1, 8),
+                                     (2, 2, 28672), (4, 7, 4224), (3, 5, 1280), (4, 1, 128)])
 def test_decode_bit_exact(gcb, bpw, N, K):
     i1, i2 = _random_codes(N, K, bpw, N + K + bpw)
     s = 0.0173
