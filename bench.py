@@ -376,6 +376,93 @@ def _traffic_from_profile():
     return int(m_t.group(1))
 
 
+def _random_codes(torch, dev, N, K, bpw, gen):
+    """Uniform random indices of the given rate (decode cost does not depend on
+    which entries are chosen beyond shared-memory bank spread)."""
+    c1 = torch.randint(0, 65536, (N, K // 8), dtype=torch.int32, device=dev,
+                       generator=gen).to(torch.uint16)
+    c2 = None
+    if bpw == 4:
+        c2 = torch.randint(0, 65536, (N, K // 8), dtype=torch.int32, device=dev,
+                           generator=gen).to(torch.uint16)
+    elif bpw == 3:
+        c2 = torch.randint(0, 256, (N, K // 8), dtype=torch.int32, device=dev,
+                           generator=gen).to(torch.uint8)
+    return c1, c2
+
+
+def _prefill_rows(e8, synth, cb, dev, stream, peaks):
+    """Prefill-sized fused decode GEMM (decode to a bf16 workspace + tcgen05 GEMM)
+    on the MLP up-projection and the four DiT block linears, 4096 tokens."""
+    import torch
+    rows = {}
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(5)
+    cases = [("mlp_up_14336_b3", synth.workloads()["mlp_up_14336_b3"].layers[0], 4096, 5)]
+    for lay in synth.workloads()["dit_3072_b4"].layers:
+        cases.append(("dit_3072_b4." + lay.name, lay, 4096, 10))
+    for name, lay, M, xseed in cases:
+        N, K, bpw = lay.N, lay.K, lay.bpw
+        codes = [_random_codes(torch, dev, N, K, bpw, gen) for _ in range(2)]
+        Xh = synth.activations_bf16(M, K, xseed)
+        X = torch.from_numpy(Xh.view(np.int16)).to(dev).view(torch.bfloat16)
+        Y = torch.empty((M, N), dtype=torch.float32, device=dev)
+        ws = torch.empty(e8.e8_workspace_bytes(e8.E8_GEMM_DECODED_W, M, N, K, bpw),
+                         dtype=torch.uint8, device=dev)
+
+        def g(i, X=X, Y=Y, ws=ws, codes=codes, N=N, K=K, bpw=bpw):
+            c1, c2 = codes[i % 2]
+            e8.e8_gemm(cb, X, c1, c2, N, K, bpw, 1, 0.02, mode=e8.E8_GEMM_DECODED_W, Y=Y,
+                       workspace=ws, stream=stream)
+
+        n = 20
+        t = _time_graphs(g, n, 4, stream) / 1e3 / n
+        flop = 2.0 * M * N * K
+        byt = N * K * bpw / 8 + M * K * 2 + M * N * 4
+        roof = max(flop / (peaks["bf16_tflops"] * 1e12), byt / (peaks["hbm_gbs"] * 1e9))
+        rows["prefill_" + name] = {"TFLOP_s": round(flop / t / 1e12, 1), "us": round(t * 1e6, 1),
+                                   "M": M, "N": N, "K": K, "bpw": bpw,
+                                   "roofline_frac": round(roof / t, 4),
+                                   "bound": "tensor" if flop / (peaks["bf16_tflops"] * 1e12) >=
+                                   byt / (peaks["hbm_gbs"] * 1e9) else "hbm"}
+        del codes, X, Y, ws
+    return rows
+
+
+def _decode_sweep_rows(e8, synth, cb, dev, stream, peaks):
+    """Decode to bf16 of one Llama-3-8B-shaped decoder layer (7 matrices) per rate;
+    the 32-layer figure is 32 times the layer."""
+    import torch
+    rows = {}
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(100)
+    for bpw in (2, 3, 4):
+        mats = synth.workloads()["llama3_8b_x32_b%d" % bpw].layers[:7]
+        data = []
+        for lay in mats:
+            codes = [_random_codes(torch, dev, lay.N, lay.K, bpw, gen) for _ in range(2)]
+            outs = [torch.empty((lay.N, lay.K), dtype=torch.bfloat16, device=dev)
+                    for _ in range(2)]
+            data.append((lay, codes, outs))
+
+        def d(i, data=data, bpw=bpw):
+            for lay, codes, outs in data:
+                c1, c2 = codes[i % 2]
+                e8.e8_decode_to_bf16(cb, c1, c2, lay.N, lay.K, bpw, lay.rht_seed, 0.02,
+                                     out=outs[i % 2], stream=stream)
+
+        n = 10
+        t = _time_graphs(d, n, 2, stream) / 1e3 / n
+        nw = sum(lay.N * lay.K for lay in mats)
+        byt = nw * (2 + bpw / 8)
+        rows["decode_llama3_8b_layer_b%d" % bpw] = {
+            "weights_per_s": nw / t, "us_per_layer": round(t * 1e6, 1),
+            "ms_32_layers": round(32 * t * 1e3, 3), "GB_s": round(byt / t / 1e9, 1),
+            "hbm_frac": round(byt / t / 1e9 / peaks["hbm_gbs"], 4)}
+        del data
+    return rows
+
+
 def _other_rows(e8, synth, cb, Wd, W, codes, X, N, K, bpw, rs, s, dev, stream, args, peaks):
     """Encode, decode-to-bf16 and the 1- and 4-token GEMM on the same layer."""
     import torch
@@ -411,6 +498,8 @@ def _other_rows(e8, synth, cb, Wd, W, codes, X, N, K, bpw, rs, s, dev, stream, a
     rows["decode_to_bf16"] = {"weights_per_s": N * K / t, "us": t * 1e6, "GB_s": byt / t / 1e9,
                               "hbm_frac": round(byt / t / 1e9 / peaks["hbm_gbs"], 4),
                               "bytes_per_weight": 2 + bpw / 8}
+    rows.update(_prefill_rows(e8, synth, cb, dev, stream, peaks))
+    rows.update(_decode_sweep_rows(e8, synth, cb, dev, stream, peaks))
     for Mx in (1, 4):
         Xm = X[:Mx].contiguous()
         Ym = torch.empty((Mx, N), dtype=torch.float32, device=dev)
