@@ -59,6 +59,8 @@ cudaError_t run_act_gemm(const e8_codebook* cb, const uint16_t* X, int64_t M,
   d.h8table = cb->h8table;
   d.hkeys = cb->hkeys;
   d.hvals = cb->hvals;
+  d.clist = cb->clist;
+  d.clist_len = cb->clist_len;
   d.status = cb->status;
   const int rows = (int)((2 * M + 15) / 16 * 16);
   if (!smem_variant && q8_eligible(M, K)) {
@@ -146,6 +148,8 @@ e8::DeviceCodebook dev_view(const e8_codebook* cb) {
   d.h8table = cb->h8table;
   d.hkeys = cb->hkeys;
   d.hvals = cb->hvals;
+  d.clist = cb->clist;
+  d.clist_len = cb->clist_len;
   d.status = cb->status;
   return d;
 }
@@ -201,6 +205,7 @@ int e8_codebook_build(e8_codebook** out, int device) {
     cudaFree(cb->h8table);
     cudaFree(cb->hkeys);
     cudaFree(cb->hvals);
+    cudaFree(cb->clist);
     cudaFree(cb->status);
     delete cb;
     if (prev >= 0) cudaSetDevice(prev);
@@ -213,6 +218,8 @@ int e8_codebook_build(e8_codebook** out, int device) {
     return fail(E8_ENOMEM);
   if (cudaMalloc(&cb->hvals, e8::kHashSlots * sizeof(uint32_t)) != cudaSuccess)
     return fail(E8_ENOMEM);
+  if (cudaMalloc(&cb->clist, e8::kCListCap * sizeof(int32_t)) != cudaSuccess)
+    return fail(E8_ENOMEM);
   if (cudaMalloc(&cb->status, 16) != cudaSuccess) return fail(E8_ENOMEM);
   cudaStream_t st;
   if (cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking) != cudaSuccess) return fail(E8_ECUDA);
@@ -221,6 +228,10 @@ int e8_codebook_build(e8_codebook** out, int device) {
   cudaMemsetAsync(cb->h8table, 0, kTableAlloc, st);
   int reps = e8::build_codebook_tables(cb->vecs, cb->table, cb->h8table, cb->hkeys, cb->hvals,
                                        &cb->max_probe, st);
+  // the kept norm-12 points with x1 = 0 and |x2| = 2: 888 positive
+  // representatives and the negations of all but the last
+  cb->clist_len = reps == 58680 ? e8::build_codebook_clist(cb->vecs, cb->clist, st) : -1;
+  if (cb->clist_len != 1775) reps = -1;
   cudaStreamDestroy(st);
   // the E8 shells of squared norm 2..12 hold 117360 vectors, half of them
   // positive representatives
@@ -241,6 +252,7 @@ void e8_codebook_free(e8_codebook* cb) {
   cudaFree(cb->h8table);
   cudaFree(cb->hkeys);
   cudaFree(cb->hvals);
+  cudaFree(cb->clist);
   cudaFree(cb->status);
   if (prev >= 0) cudaSetDevice(prev);
   delete cb;
@@ -276,7 +288,7 @@ size_t e8_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int bpw) {
   const size_t G = (size_t)N * (size_t)(K / 8);
   switch (op) {
     case E8_OP_ENCODE:
-      return 256 + G * sizeof(e8::WorkItem);
+      return 256 + 2 * G * sizeof(e8::WorkItem);
     case E8_GEMM_AUTO:
       return e8_workspace_bytes(e8_gemm_auto_mode(M, N, K, bpw), M, N, K, bpw);
     case E8_GEMM_ACT_RHT:

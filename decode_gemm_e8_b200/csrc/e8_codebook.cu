@@ -13,6 +13,7 @@
 // coordinates are enumerated by ascending nested loops, which is lexicographic.
 #include "e8_common.cuh"
 #include "e8_codebook.cuh"
+#include "e8_internal.h"
 
 namespace e8 {
 
@@ -167,6 +168,30 @@ __global__ void k_cb_h8(const uint32_t* table, uint32_t* h8, int* bad) {
   }
   if (!ok) atomicAdd(bad, 1);
   h8[q] = pack_vec(v);
+}
+
+__global__ void k_cb_clist(const int8_t* vecs, int32_t* clist, int* count) {
+  int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= kCbSize) return;
+  const int8_t* v = vecs + 8 * i;
+  int n = 0;
+  for (int j = 0; j < 8; ++j) n += v[j] * v[j];
+  if (n != 48 || v[0] != 0 || (v[1] != 4 && v[1] != -4)) return;
+  const int slot = atomicAdd(count, 1);
+  if (slot < kCListCap) clist[slot] = i;
+}
+
+int build_codebook_clist(const int8_t* d_vecs, int32_t* d_clist, cudaStream_t st) {
+  int* d_count = nullptr;
+  if (cudaMalloc(&d_count, sizeof(int)) != cudaSuccess) return -1;
+  cudaMemsetAsync(d_count, 0, sizeof(int), st);
+  k_cb_clist<<<kCbSize / 256, 256, 0, st>>>(d_vecs, d_clist, d_count);
+  int h = -1;
+  cudaMemcpyAsync(&h, d_count, sizeof(int), cudaMemcpyDeviceToHost, st);
+  cudaError_t e = cudaStreamSynchronize(st);
+  cudaFree(d_count);
+  if (e != cudaSuccess || cudaGetLastError() != cudaSuccess || h > kCListCap) return -1;
+  return h;
 }
 
 // Builds vecs, table, the transformed table and the hash on the current

@@ -94,6 +94,8 @@ struct DeviceCodebook {
   const uint32_t* h8table;   // [32769]
   const uint32_t* hkeys;     // [kHashSlots]
   const uint32_t* hvals;     // [kHashSlots]
+  const int32_t* clist;      // indices of the kept norm-12 points with x1 = 0, |x2| = 2
+  int clist_len;
   uint32_t* status;          // device status word
 };
 

@@ -175,6 +175,7 @@ __device__ __forceinline__ void push_work(const EncodeParams& p, const DeviceCod
   for (int i = 0; i < 8; ++i) w.u[i] = u[i];
   w.group = g;
   w.mask = mask;
+  w.cand = 0u;
 }
 
 __global__ void __launch_bounds__(256) k_encode(EncodeParams p, DeviceCodebook cb) {
@@ -311,28 +312,35 @@ __device__ __forceinline__ double approx_d2(const DeviceCodebook& cb, const floa
   return s;
 }
 
-// Exact argmin over candidates c in [0, n) of |u - (base + v_c)/den|^2 by one
-// warp; smallest index on ties.  All lanes return the same index.
+// Exact argmin of |u - (base + v_c)/den|^2 by one warp over the candidates c =
+// list[0..n) (or c in [0, n) when list is null), plus `extra` when >= 0;
+// smallest index on ties.  All lanes return the same index.
 __device__ int warp_exact_argmin(const DeviceCodebook& cb, const float (&u)[8],
-                                 const int (&base)[8], int den, int n) {
+                                 const int (&base)[8], int den, int n, const int32_t* list,
+                                 int extra) {
   const int lane = threadIdx.x & 31;
   const double inv_den = 1.0 / den;
+  const int total = n + (extra >= 0 ? 1 : 0);
+  auto cand = [&](int i) { return i < n ? (list ? (int)__ldg(list + i) : i) : extra; };
   double dmin = INFINITY;
   int Z[8];
-  for (int c = lane; c < n; c += 32) dmin = fmin(dmin, approx_d2(cb, u, base, c, inv_den, Z));
+  for (int i = lane; i < total; i += 32)
+    dmin = fmin(dmin, approx_d2(cb, u, base, cand(i), inv_den, Z));
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) dmin = fmin(dmin, __shfl_xor_sync(0xffffffffu, dmin, off));
   const double lim = dmin * (1.0 + 0x1p-40);
   // lane-local exact winner among the short list, then a warp tournament
   int best = -1;
   int Zw[8];
-  for (int c = lane; c < n; c += 32) {
+  for (int i = lane; i < total; i += 32) {
+    const int c = cand(i);
     double s = approx_d2(cb, u, base, c, inv_den, Z);
     if (!(s <= lim)) continue;
-    if (best < 0 || exact_cmp(u, Zw, Z, den) > 0) {
+    int cmp = best < 0 ? 1 : exact_cmp(u, Zw, Z, den);
+    if (cmp > 0 || (cmp == 0 && c < best)) {
       best = c;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) Zw[i] = Z[i];
+      for (int k = 0; k < 8; ++k) Zw[k] = Z[k];
     }
   }
 #pragma unroll
@@ -356,32 +364,59 @@ __device__ int warp_exact_argmin(const DeviceCodebook& cb, const float (&u)[8],
   return best < 0 ? 0 : best;
 }
 
-__global__ void __launch_bounds__(256) k_encode_slow(const WorkItem* work,
-                                                     const uint32_t* work_count,
-                                                     uint64_t work_cap, int bpw, uint16_t* idx1,
-                                                     void* idx2, DeviceCodebook cb) {
-  const uint64_t n = (uint64_t)min((unsigned long long)*work_count, (unsigned long long)work_cap);
+// One warp per work item: exact brute force over the whole candidate set, or
+// over the listed norm-12 points plus the item's best other candidate.  A
+// stage 1 settled here sends its stage 2 back (to `out`) for the class search.
+__global__ void __launch_bounds__(256) k_encode_slow(const WorkItem* in, const uint32_t* in_count,
+                                                     uint64_t cap, WorkItem* out,
+                                                     uint32_t* out_count, int bpw,
+                                                     uint16_t* idx1, void* idx2,
+                                                     DeviceCodebook cb) {
+  const uint64_t n = (uint64_t)min((unsigned long long)*in_count, (unsigned long long)cap);
   const uint64_t warp = ((uint64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const uint64_t nwarps = ((uint64_t)gridDim.x * blockDim.x) >> 5;
+  const int lane = threadIdx.x & 31;
   for (uint64_t w = warp; w < n; w += nwarps) {
-    const WorkItem& it = work[w];
+    const WorkItem& it = in[w];
     float u[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) u[i] = it.u[i];
     const int64_t g = it.group;
-    int i1 = idx1[g];
-    if (it.mask & 1u) {
+    const uint32_t mask = it.mask;
+    if (mask & kWorkStage1) {
       int zero[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-      i1 = warp_exact_argmin(cb, u, zero, 2, kCbSize);
-      if ((threadIdx.x & 31) == 0) idx1[g] = (uint16_t)i1;
+      const int i1 = (mask & kWorkStage1List)
+                         ? warp_exact_argmin(cb, u, zero, 2, cb.clist_len, cb.clist, (int)it.cand)
+                         : warp_exact_argmin(cb, u, zero, 2, kCbSize, nullptr, -1);
+      if (lane == 0) {
+        idx1[g] = (uint16_t)i1;
+        if (bpw > 2) {
+          const uint32_t slot = out ? atomicAdd(out_count, 1u) : 0xFFFFFFFFu;
+          if (slot < cap) {
+            WorkItem& o = out[slot];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) o.u[i] = u[i];
+            o.group = g;
+            o.mask = kWorkStage2;
+            o.cand = 0u;
+          } else {
+            atomicOr(cb.status, kDevWorklistOverflow);
+          }
+        }
+      }
+      continue;
     }
-    if (bpw > 2 && (it.mask & 2u)) {
+    if (bpw > 2 && (mask & kWorkStage2)) {
+      const int i1 = idx1[g];
       const int m = bpw == 3 ? 4 : 8;
       int base[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) base[i] = (m / 2) * (int)cb.vecs[8 * i1 + i];
-      int i2 = warp_exact_argmin(cb, u, base, m, bpw == 3 ? 256 : kCbSize);
-      if ((threadIdx.x & 31) == 0) {
+      const int i2 = (mask & kWorkStage2List)
+                         ? warp_exact_argmin(cb, u, base, m, cb.clist_len, cb.clist, (int)it.cand)
+                         : warp_exact_argmin(cb, u, base, m, bpw == 3 ? 256 : kCbSize, nullptr,
+                                             -1);
+      if (lane == 0) {
         if (bpw == 3) reinterpret_cast<uint8_t*>(idx2)[g] = (uint8_t)i2;
         else reinterpret_cast<uint16_t*>(idx2)[g] = (uint16_t)i2;
       }
@@ -418,13 +453,29 @@ cudaError_t launch_encode(const DeviceCodebook& cb, const float* W, int64_t N, i
   cudaError_t e = ensure_smem_limit(k_encode, kMaxDynSmem);
   if (e != cudaSuccess) return e;
   if (do_quantise) {
-    e = cudaMemsetAsync(work_count, 0, sizeof(uint32_t), st);
+    e = cudaMemsetAsync(work_count, 0, 4 * sizeof(uint32_t), st);
     if (e != cudaSuccess) return e;
   }
   k_encode<<<(unsigned)ctas, 256, smem, st>>>(p, cb);
   e = cudaGetLastError();
   if (e != cudaSuccess || !do_quantise) return e;
-  k_encode_slow<<<sm_count * 4, 256, 0, st>>>(work, work_count, work_cap, bpw, idx1, idx2, cb);
+  // undecided groups: class search (thread per group), then the warp brute
+  // force for what stays open; stage 2 of a group whose stage 1 needed the
+  // brute force takes a second round
+  WorkItem* r1 = work;
+  WorkItem* r2 = work + work_cap;
+  e = launch_encode_leader(cb, r1, work_count, work_cap, r2, work_count + 1, bpw, idx1, idx2,
+                           sm_count, st);
+  if (e != cudaSuccess) return e;
+  k_encode_slow<<<sm_count * 4, 256, 0, st>>>(r2, work_count + 1, work_cap, r1, work_count + 2,
+                                              bpw, idx1, idx2, cb);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (bpw == 2) return cudaSuccess;
+  e = launch_encode_leader(cb, r1, work_count + 2, work_cap, r2, work_count + 3, bpw, idx1, idx2,
+                           sm_count, st);
+  if (e != cudaSuccess) return e;
+  k_encode_slow<<<sm_count * 4, 256, 0, st>>>(r2, work_count + 3, work_cap, nullptr, nullptr, bpw,
+                                              idx1, idx2, cb);
   return cudaGetLastError();
 }
 

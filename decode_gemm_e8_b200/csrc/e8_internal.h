@@ -15,8 +15,10 @@ struct e8_codebook {
   uint32_t* h8table;
   uint32_t* hkeys;
   uint32_t* hvals;
+  int32_t* clist;     // indices of the kept norm-12 points with x1 = 0, |x2| = 2
   uint32_t* status;
   int max_probe;
+  int clist_len;
 };
 
 namespace e8 {
@@ -25,19 +27,35 @@ namespace e8 {
 struct WorkItem {
   float u[8];      // transformed, scaled weights of the group
   int64_t group;   // global group index (row * K/8 + column / 8)
-  uint32_t mask;   // bit 0: stage 1 undecided, bit 1: stage 2 undecided
-  uint32_t pad;
+  uint32_t mask;   // kWork* bits
+  uint32_t cand;   // with kWorkStage*List: best index outside the listed set
 };
 static_assert(sizeof(WorkItem) == 48, "WorkItem layout");
+enum : uint32_t {
+  kWorkStage1 = 1u,       // stage 1 undecided
+  kWorkStage2 = 2u,       // stage 2 undecided (or pending behind stage 1)
+  kWorkStage1List = 4u,   // stage 1: only the listed set and `cand` compete
+  kWorkStage2List = 8u,   // stage 2: likewise
+};
 
 int build_codebook_tables(int8_t* d_vecs, uint32_t* d_table, uint32_t* d_h8table,
                           uint32_t* d_hkeys, uint32_t* d_hvals, int* h_max_probe, cudaStream_t st);
+// Fills clist with the codebook indices of the norm-12 entries with x1 = 0 and
+// |x2| = 2 (doubled: 0 and 4); returns their number or -1.
+int build_codebook_clist(const int8_t* d_vecs, int32_t* d_clist, cudaStream_t st);
+constexpr int kCListCap = 2048;
 
 int encode_elems_per_cta(int nh);
+// Encoder workspace: four item counters (256 bytes), then two item regions of
+// `work_cap` items each.
 cudaError_t launch_encode(const DeviceCodebook& cb, const float* W, int64_t N, int64_t K, int bpw,
                           uint64_t seed, float gamma, uint16_t* idx1, void* idx2,
                           WorkItem* work, uint32_t* work_count, uint64_t work_cap, float* U,
                           int do_quantise, int sm_count, cudaStream_t st);
+cudaError_t launch_encode_leader(const DeviceCodebook& cb, const WorkItem* in,
+                                 const uint32_t* in_count, uint64_t cap, WorkItem* out,
+                                 uint32_t* out_count, int bpw, uint16_t* idx1, void* idx2,
+                                 int sm_count, cudaStream_t st);
 
 cudaError_t launch_decode(const DeviceCodebook& cb, const uint16_t* idx1, const void* idx2,
                           int64_t N, int64_t K, int bpw, uint64_t seed, float alpha,

@@ -112,6 +112,50 @@ def test_encode_planted_ties_and_lattice_points(gcb, cb):
             assert np.array_equal(g2, r2)
 
 
+def _e8_points_of_norm(rng, norm2, count):
+    """Random E8 points (real coordinates) of squared norm `norm2`, by rejection
+    from integer and half-integer vectors with even coordinate sum."""
+    out = []
+    while len(out) < count:
+        if rng.integers(2):
+            v = rng.integers(-3, 4, 8).astype(np.float64)
+        else:
+            v = rng.integers(-3, 3, 8).astype(np.float64) + 0.5
+        if v.sum() % 2 == 0 and (v * v).sum() == norm2:
+            out.append(v)
+    return np.array(out)
+
+
+def test_encode_near_truncated_shell(gcb, cb):
+    # groups near points of squared norm 12 (the shell the codebook keeps only
+    # in part), 14 and 16 (outside it), and between them, so that the nearest
+    # codebook point is decided by the kept part of the norm-12 shell
+    n = 256
+    rng = np.random.default_rng(12)
+    kept = cb[np.nonzero((cb.astype(np.int64) ** 2).sum(1) == 48)[0]].astype(np.float64) / 2
+    G = 8 * n // 8
+    parts = [kept[rng.integers(0, len(kept), G // 4)],
+             _e8_points_of_norm(rng, 12, G // 4),
+             _e8_points_of_norm(rng, 14, G // 8),
+             _e8_points_of_norm(rng, 16, G // 8)]
+    mid = _e8_points_of_norm(rng, 12, G // 4)
+    parts.append(0.5 * (mid + kept[rng.integers(0, len(kept), G // 4)]))
+    U = np.concatenate(parts)[:G]
+    U = U + rng.normal(0.0, 0.05, U.shape) * (np.arange(G) % 3 != 0)[:, None]
+    U = U.reshape(8, n)
+    from tests import indep
+    H = indep.sylvester(n).astype(np.float64)
+    d = orc.signs(4, n).astype(np.float64)
+    s = float(np.float32(1.0 / np.sqrt(n)))
+    W = (d[None, :] * (U @ H) / n).astype(np.float32)
+    for bpw in (2, 3, 4):
+        g1, g2, r1, r2 = _encode_both(gcb, W, bpw, 4, s)
+        assert np.array_equal(g1, r1)
+        if bpw > 2:
+            assert np.array_equal(g2, r2)
+    assert e8.e8_sync_status(gcb) == e8.E8_OK
+
+
 def test_encode_zero_and_nonfinite(gcb):
     W = np.zeros((4, 512), np.float32)
     W[1, 17] = np.nan
