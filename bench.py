@@ -329,7 +329,7 @@ def run_ours(args):
             "decoded_weights_per_s": N * K * args.steps * ws / sec,
             "roofline": {
                 "bound": "hbm",
-                "kernel": "k_act_gemm_q8 (fused decode + tcgen05 GEMM)",
+                "kernel": "k_gemm_q8 (fused decode + tcgen05 GEMM, stream-K over all SMs)",
                 "achieved": round(achieved, 1),
                 "peak": peaks["hbm_gbs"],
                 "unit": "GB/s",
@@ -362,8 +362,8 @@ def _traffic_from_profile():
     """DRAM bytes per launch of k_act_gemm from the committed ncu summary, or None
     when the kernel source changed since the counters were taken."""
     import hashlib
-    prof = os.path.join(ROOT, "profiles", "k_act_gemm_q8_llama4096_m16.md")
-    src = os.path.join(ROOT, "decode_gemm_e8_b200", "csrc", "e8_gemm_act.cu")
+    prof = os.path.join(ROOT, "profiles", "k_gemm_q8_llama4096_m16.md")
+    src = os.path.join(ROOT, "decode_gemm_e8_b200", "csrc", "e8_gemm_q8.cu")
     if not os.path.exists(prof):
         return None
     h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]

@@ -251,10 +251,11 @@ def e8_act_rht_q8(X, rht_seed: int, out=None, stream=None):
 
 def e8_gemm_xt(cb: Codebook, xq, M: int, idx1, idx2, N: int, K: int, bpw: int, scale: float,
                Y=None, stream=None):
-    """Fused decode + int8 GEMM on a buffer from e8_act_rht_q8."""
+    """Fused decode + int8 GEMM on a buffer from e8_act_rht_q8; the product is
+    added into Y (a new zero tensor when Y is None)."""
     import torch
     if Y is None:
-        Y = torch.empty((M, N), dtype=torch.float32, device=xq.device)
+        Y = torch.zeros((M, N), dtype=torch.float32, device=xq.device)
     _check(load_library().e8_gemm_xt(cb.handle, _ptr(xq), int(M), _ptr(idx1), _ptr(idx2), int(N),
                                      int(K), int(bpw), float(scale), _ptr(Y), _stream(stream)),
            "e8_gemm_xt")

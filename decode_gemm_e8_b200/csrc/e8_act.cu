@@ -249,153 +249,174 @@ cudaError_t launch_act_rht(const uint16_t* X, int64_t M, int64_t K, uint64_t see
 
 namespace e8 {
 
-// Activation transform for the int8 tensor-core path.  One CTA per token row
-// (all its Hadamard blocks, n_h in 256..4096): the row is transformed into
-// shared memory, its largest magnitude fixes the token's step s_m = max / 127,
-// and the row is written as two int8 pieces
+// Activation transform for the int8 tensor-core path.  One CTA of 512
+// threads per token row, 8 values per thread, the row in chunks of up to
+// 4096 positions (several Hadamard blocks when n_h < 4096).  Position
+// p = 256 w + 8 l + e (warp w, lane l, register e): the stages of the
+// three low bits run in registers, the next five by warp shuffles, and the
+// stages across warps (n_h > 256) after one exchange through shared memory,
+// where thread t takes the 8 positions g + 256 (8 (t & 1) + j), g = t >> 1,
+// three stages in registers and the last by a shuffle with its neighbour.
+// The row's largest magnitude fixes the token's step s_m = max / 127, and the
+// row is written as two int8 pieces
 //   q0 = rint(x / s_m),  q1 = rint((x - q0 s_m) * 128 / s_m),  |q1| <= 64,
 // so x = s_m (q0 + q1 / 128) + e with |e| <= s_m / 256.  Piece rows are
 // interleaved (row 2m = q0, row 2m + 1 = q1); colsum[row] = sum_k Xq[row][k]
 // lets the GEMM remove the +128 bias of its unsigned weight operand exactly.
-__global__ void __launch_bounds__(512) k_act_q8(const uint16_t* __restrict__ X, int64_t M,
-                                                int64_t K, int nh, uint64_t seed,
-                                                int8_t* __restrict__ Xq,
-                                                float* __restrict__ scales,
-                                                int32_t* __restrict__ colsum, int64_t rows) {
-  extern __shared__ __align__(16) float s_dyn[];
-  float* s_row = s_dyn;            // K floats
-  float* s_x = s_dyn + K;          // 4096-float transpose scratch
-  __shared__ float s_red[16];
-  __shared__ int s_ired[2][16];
-  grid_dep_wait();
+// Kept small (32 registers, K floats of shared memory) so that it can share an
+// SM with a CTA of the GEMM that follows it.
+__global__ void __launch_bounds__(512, 4) k_act_q8(const uint16_t* __restrict__ X, int M, int K,
+                                                   int nh, uint64_t seed,
+                                                   int8_t* __restrict__ Xq,
+                                                   float* __restrict__ scales,
+                                                   int32_t* __restrict__ colsum, int rows,
+                                                   float* __restrict__ Yz, int64_t yz_elems) {
+  extern __shared__ __align__(16) float s_row[];   // K floats
+  __shared__ float s_max[16];
+  __shared__ int s_sum[2][16];
+  // the GEMM that follows may start at once: it touches nothing that this
+  // kernel or its predecessor writes until its own wait for this grid
   grid_dep_launch();
+  grid_dep_wait();
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  const int64_t m = blockIdx.x;
-  if (m >= M) {
-    // padding rows: zero bytes and zero column sums
-    const int64_t pad_row = 2 * M + (m - M);
-    if (pad_row < rows) {
-      for (int64_t k = 16 * t; k < K; k += 16 * blockDim.x)
-        *reinterpret_cast<uint4*>(Xq + pad_row * K + k) = make_uint4(0u, 0u, 0u, 0u);
-      if (t == 0) colsum[pad_row] = 0;
+  const int m = blockIdx.x;
+  // the output that the following GEMM accumulates into starts at zero
+  if (Yz) {
+    const int64_t per = ((yz_elems + gridDim.x - 1) / gridDim.x + 3) & ~int64_t(3);
+    const int64_t z0 = (int64_t)m * per, z1 = z0 + per < yz_elems ? z0 + per : yz_elems;
+    for (int64_t i = z0 + 4 * t; i < z1; i += 4 * blockDim.x) {
+      if (i + 4 <= z1) {
+        *reinterpret_cast<float4*>(Yz + i) = make_float4(0.f, 0.f, 0.f, 0.f);
+      } else {
+        for (int64_t j = i; j < z1; ++j) Yz[j] = 0.0f;
+      }
     }
-    return;
   }
-  const bool owner = t < (nh >> 3);
-  for (int64_t kb = 0; kb < K; kb += nh) {
-    const int64_t k0 = kb + 8 * t;
-    float y[8];
-    {
-      uint4 raw = owner ? __ldg(reinterpret_cast<const uint4*>(X + m * K + k0))
-                        : make_uint4(0u, 0u, 0u, 0u);
+  // padding rows 2M .. rows-1: zero bytes, zero sums
+  for (int pr = 2 * M + m; pr < rows; pr += M) {
+    for (int k = 16 * t; k < K; k += 16 * 512)
+      *reinterpret_cast<uint4*>(Xq + (size_t)pr * K + k) = make_uint4(0u, 0u, 0u, 0u);
+    if (t == 0) colsum[pr] = 0;
+  }
+  const uint16_t* xrow = X + (size_t)m * K;
+  float mx = 0.0f;
+  for (int kb = 0; kb < K; kb += 4096) {
+    const int C = K - kb < 4096 ? K - kb : 4096;   // a multiple of 256
+    float* chunk = s_row + kb;
+    if (8 * t < C) {
+      const int k0 = kb + 8 * t;
+      float y[8];
+      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(xrow + k0));
       const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         y[2 * i] = bf16_lo_to_f32(rw[i]);
         y[2 * i + 1] = bf16_hi_to_f32(rw[i]);
       }
-    }
-    const uint64_t word = splitmix64_output(seed, (uint64_t)(k0 >> 6));
-    const uint32_t bits = (uint32_t)(word >> (k0 & 63));
+      const uint32_t bits =
+          (uint32_t)(splitmix64_output(seed, (uint64_t)(k0 >> 6)) >> (k0 & 63));
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-      y[i] = __uint_as_float(__float_as_uint(y[i]) ^ (((bits >> i) & 1u) << 31));
+      for (int i = 0; i < 8; ++i)
+        y[i] = __uint_as_float(__float_as_uint(y[i]) ^ (((bits >> i) & 1u) << 31));
+      // butterflies (a, b) -> (a + b, a - b), a the lower position
 #pragma unroll
-    for (int h = 1; h < 8; h <<= 1) {
+      for (int h = 1; h < 8; h <<= 1) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        if ((i & h) == 0) {
-          float a = y[i], c = y[i + h];
-          y[i] = a + c;
-          y[i + h] = a - c;
+        for (int i = 0; i < 8; ++i) {
+          if ((i & h) == 0) {
+            const float a = y[i], c = y[i + h];
+            y[i] = a + c;
+            y[i + h] = a - c;
+          }
         }
       }
-    }
 #pragma unroll
-    for (int h = 8; h < 256; h <<= 1) {
-      const int lm = h >> 3;
-      const bool upper = (lane & lm) != 0;
+      for (int lm = 1; lm < 32; lm <<= 1) {
+        const bool upper = (lane & lm) != 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float o = __shfl_xor_sync(0xffffffffu, y[i], lm);
-        y[i] = upper ? o - y[i] : y[i] + o;
+        for (int i = 0; i < 8; ++i) {
+          const float o = __shfl_xor_sync(0xffffffffu, y[i], lm);
+          y[i] = upper ? o - y[i] : y[i] + o;
+        }
       }
+      *reinterpret_cast<float4*>(chunk + 8 * t) = make_float4(y[0], y[1], y[2], y[3]);
+      *reinterpret_cast<float4*>(chunk + 8 * t + 4) = make_float4(y[4], y[5], y[6], y[7]);
     }
-    if (nh <= 256) {
-      if (owner) {
-        float4* d = reinterpret_cast<float4*>(s_row + k0);
-        d[0] = make_float4(y[0], y[1], y[2], y[3]);
-        d[1] = make_float4(y[4], y[5], y[6], y[7]);
-      }
-    } else {
-      if (owner) {
-        float4* d = reinterpret_cast<float4*>(s_x + 8 * t);
-        d[0] = make_float4(y[0], y[1], y[2], y[3]);
-        d[1] = make_float4(y[4], y[5], y[6], y[7]);
-      }
+    if (nh > 256) {
       __syncthreads();
-      if (t < 256) {
-        const int per = nh >> 8;
-        float z[16];
+      // stages across warps: h = 256 .. nh/2 on the positions g + 256 i
+      const int g = t >> 1, half = t & 1;
+      const int nw = C >> 8;                 // 256-position slices in the chunk
+      float y[8];
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          if (j < per) z[j] = s_x[t + 256 * j];
+      for (int j = 0; j < 8; ++j) {
+        const int i = 8 * half + j;
+        y[j] = i < nw ? chunk[g + 256 * i] : 0.0f;
+      }
 #pragma unroll
-        for (int h = 1; h < 16; h <<= 1) {
-          if (h >= per) break;
+      for (int h = 1; h < 8; h <<= 1) {
+        if (256 * h < nh) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            if (j < per && (j & h) == 0) {
-              float a = z[j], c = z[j + h];
-              z[j] = a + c;
-              z[j + h] = a - c;
+          for (int j = 0; j < 8; ++j) {
+            if ((j & h) == 0) {
+              const float a = y[j], c = y[j + h];
+              y[j] = a + c;
+              y[j + h] = a - c;
             }
           }
         }
-#pragma unroll
-        for (int j = 0; j < 16; ++j)
-          if (j < per) s_row[kb + t + 256 * j] = z[j];
       }
+      if (nh > 2048) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float o = __shfl_xor_sync(0xffffffffu, y[j], 1);
+          y[j] = half ? o - y[j] : y[j] + o;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int i = 8 * half + j;
+        if (i < nw) {
+          chunk[g + 256 * i] = y[j];
+          mx = fmaxf(mx, fabsf(y[j]));
+        }
+      }
+    } else if (8 * t < C) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) mx = fmaxf(mx, fabsf(chunk[8 * t + j]));
     }
-    __syncthreads();
   }
   // largest magnitude of the row
-  float mx = 0.0f;
-  for (int64_t k = t; k < K; k += blockDim.x) mx = fmaxf(mx, fabsf(s_row[k]));
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-  if (lane == 0) s_red[warp] = mx;
+  if (lane == 0) s_max[warp] = mx;
   __syncthreads();
-  if (t < 32) {
-    float v = t < (int)(blockDim.x >> 5) ? s_red[t] : 0.0f;
+  float amax = 0.0f;
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
-    if (t == 0) s_red[0] = v;
-  }
-  __syncthreads();
-  const float amax = s_red[0];
+  for (int w = 0; w < 16; ++w) amax = fmaxf(amax, s_max[w]);
   const float step = amax > 0.0f ? amax / 127.0f : 1.0f;
   const float inv = 1.0f / step;
   int sum0 = 0, sum1 = 0;
-  int8_t* q0row = Xq + (2 * m) * K;
-  int8_t* q1row = Xq + (2 * m + 1) * K;
-  for (int64_t k = 4 * t; k < K; k += 4 * blockDim.x) {
-    const float4 x4 = *reinterpret_cast<const float4*>(s_row + k);
-    const float xs[4] = {x4.x, x4.y, x4.z, x4.w};
-    uint32_t p0 = 0, p1 = 0;
+  int8_t* q0row = Xq + (size_t)(2 * m) * K;
+  int8_t* q1row = Xq + (size_t)(2 * m + 1) * K;
+  for (int k = 8 * t; k < K; k += 8 * 512) {
+    const float4 xa = *reinterpret_cast<const float4*>(s_row + k);
+    const float4 xb = *reinterpret_cast<const float4*>(s_row + k + 4);
+    const float xs[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+    uint32_t p0[2] = {0u, 0u}, p1[2] = {0u, 0u};
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 8; ++i) {
       const float a = fminf(fmaxf(rintf(xs[i] * inv), -127.0f), 127.0f);
       const float r = xs[i] - a * step;
       const float b = fminf(fmaxf(rintf(r * inv * 128.0f), -127.0f), 127.0f);
       const int ia = (int)a, ib = (int)b;
       sum0 += ia;
       sum1 += ib;
-      p0 |= (uint32_t)(ia & 0xFF) << (8 * i);
-      p1 |= (uint32_t)(ib & 0xFF) << (8 * i);
+      p0[i >> 2] |= (uint32_t)(ia & 0xFF) << (8 * (i & 3));
+      p1[i >> 2] |= (uint32_t)(ib & 0xFF) << (8 * (i & 3));
     }
-    *reinterpret_cast<uint32_t*>(q0row + k) = p0;
-    *reinterpret_cast<uint32_t*>(q1row + k) = p1;
+    *reinterpret_cast<uint2*>(q0row + k) = make_uint2(p0[0], p0[1]);
+    *reinterpret_cast<uint2*>(q1row + k) = make_uint2(p1[0], p1[1]);
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) {
@@ -403,32 +424,36 @@ __global__ void __launch_bounds__(512) k_act_q8(const uint16_t* __restrict__ X, 
     sum1 += __shfl_xor_sync(0xffffffffu, sum1, off);
   }
   if (lane == 0) {
-    s_ired[0][warp] = sum0;
-    s_ired[1][warp] = sum1;
+    s_sum[0][warp] = sum0;
+    s_sum[1][warp] = sum1;
   }
   __syncthreads();
-  if (t == 0) {
-    int a = 0, b = 0;
-    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
-      a += s_ired[0][w];
-      b += s_ired[1][w];
-    }
-    colsum[2 * m] = a;
-    colsum[2 * m + 1] = b;
-    scales[m] = step;
+  if (t < 32) {
+    int a = lane < 16 ? s_sum[0][lane] : s_sum[1][lane - 16];
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
+    if (lane == 0) colsum[2 * m] = a;
+    if (lane == 16) colsum[2 * m + 1] = a;
+    if (lane == 0) scales[m] = step;
   }
 }
 
 cudaError_t launch_act_q8(const uint16_t* X, int64_t M, int64_t K, uint64_t seed, int8_t* Xq,
                           float* scales, int32_t* colsum, int64_t rows, cudaStream_t st,
-                          int pdl) {
+                          int pdl, float* Yz, int64_t yz_elems) {
   const int nh = (int)hadamard_block(K);
-  if (nh < 256 || nh > 4096 || K > 32768) return cudaErrorInvalidValue;
-  const size_t smem = (size_t)(K + 4096) * sizeof(float);
+  if (nh < 256 || nh > 4096 || K > 32768 || M < 1 || M > 32 || rows < 2 * M || rows > 64)
+    return cudaErrorInvalidValue;
+  const size_t smem = (size_t)K * sizeof(float);
   cudaError_t e = ensure_smem_limit(k_act_q8, kMaxDynSmem);
   if (e != cudaSuccess) return e;
+  // the same shared-memory carveout as the GEMM that follows, so that the two
+  // can share an SM (an SM runs CTAs of one carveout at a time)
+  e = cudaFuncSetAttribute(k_act_q8, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared);
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(M + (rows - 2 * M)));
+  cfg.gridDim = dim3((unsigned)M);
   cfg.blockDim = dim3(512);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
@@ -437,7 +462,8 @@ cudaError_t launch_act_q8(const uint16_t* X, int64_t M, int64_t K, uint64_t seed
   attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, k_act_q8, X, M, K, nh, seed, Xq, scales, colsum, rows);
+  e = cudaLaunchKernelEx(&cfg, k_act_q8, X, (int)M, (int)K, nh, seed, Xq, scales, colsum,
+                         (int)rows, Yz, yz_elems);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -83,7 +83,8 @@ cudaError_t run_act_gemm(const e8_codebook* cb, const uint16_t* X, int64_t M,
     a.early_codes = 1;  // which writes only the activation buffer
     cudaError_t e = launch_act_q8(X, M, K, seed, reinterpret_cast<int8_t*>(buf),
                                   reinterpret_cast<float*>(buf + l.scales_off),
-                                  reinterpret_cast<int32_t*>(buf + l.colsum_off), rows, st, 1);
+                                  reinterpret_cast<int32_t*>(buf + l.colsum_off), rows, st, 1, Y,
+                                  M * N);
     if (e != cudaSuccess) return e;
     return launch_act_gemm_q8(d, a, cb->sm_count, st);
   }
@@ -457,8 +458,8 @@ int e8_gemm_xt(const e8_codebook* cb, const void* xq, int64_t M, const uint16_t*
   a.bpw = bpw;
   a.alpha = alpha_of(scale, e8::hadamard_block(K), bpw);
   a.Y = Y;
-  a.pdl = 1;          // only the library's table is read before the previous kernel ends
-  a.early_codes = 0;  // the previous kernel is the caller's and may write the codes
+  a.pdl = 1;          // table and codes are read before the previous kernel ends
+  a.early_codes = 1;
   return cuda_status(e8::launch_act_gemm_q8(dev_view(cb), a, cb->sm_count, (cudaStream_t)stream));
 }
 

@@ -375,433 +375,6 @@ static cudaError_t launch_act_gemm_generic(const DeviceCodebook& cb, const ActGe
   return cudaGetLastError();
 }
 
-// ===========================================================================
-// int8 tensor-core variant for up to 32 tokens: the small-batch hot path.
-//
-// The transformed activations arrive as two int8 pieces per token (rows 2m
-// and 2m + 1 of Xq, see k_act_q8) with a per-token step s_m, so that
-//   xt_m = s_m (q0_m + q1_m / 128)   (error below s_m / 256).
-// The weight operand is z + 128 as unsigned bytes (|z| <= 30), decoded on chip
-// straight into tensor memory; tcgen05.mma kind::i8 (K = 32 per instruction)
-// accumulates exactly in int32, and the epilogue removes the bias with the
-// per-row column sums of Xq:
-//   y[m][n] = alpha s_m ((D[n][2m] - 128 cs[2m]) + (D[n][2m+1] - 128 cs[2m+1]) / 128).
-// Structure: warp 0 TMA producer (index tiles with a 64-byte swizzle, Xq tiles
-// with a 128-byte swizzle), warp 1 tensor-memory allocation + one MMA issuer,
-// 16 decode warps (four per tensor-memory lane quarter, 8 groups each per K
-// step of 256), programmatic dependent launch (table copy and index tiles
-// before waiting for the transform), split-K over a cluster with the partial
-// tiles pushed to their owner CTA by st.async.
-// ===========================================================================
-namespace agq {
-constexpr int ROWS = 128;
-constexpr int KSTEP = 256;
-constexpr int GROUPS = KSTEP / 8;
-constexpr int DEC_WARPS = 16;
-constexpr int THREADS = 64 + DEC_WARPS * 32;
-constexpr int I1_BYTES = ROWS * GROUPS * 2;
-constexpr int TABLE_BYTES = 131088;
-constexpr int STAGE0 = 132096;        // table, rounded up to 1 KB
-constexpr uint32_t D_COLS = 64;       // int32 accumulator columns (rows_b <= 64)
-constexpr uint32_t A_COLS = KSTEP / 4;  // 4 int8 per tensor-memory column
-constexpr uint32_t TMEM_COLS = 256;
-constexpr int BAR_LIMIT = kMaxDynSmem - 1024 - 256;
-constexpr int RECV_BYTES = ROWS * 8 * 16;
-}  // namespace agq
-
-struct Q8Plan {
-  int stages, b_bytes, i2_bytes, stage_bytes, recv_off, aux_off, bar_off, total;
-};
-
-__host__ __device__ inline Q8Plan q8_plan(int rows_b, int bpw) {
-  using namespace agq;
-  Q8Plan p;
-  p.b_bytes = rows_b * KSTEP;
-  p.i2_bytes = bpw == 2 ? 0 : (bpw == 3 ? ROWS * GROUPS : ROWS * GROUPS * 2);
-  p.stage_bytes = (p.b_bytes + I1_BYTES + p.i2_bytes + 1023) & ~1023;
-  // after the stages: the reduction's receive area (128 rows x 8 float4) and the
-  // per-token steps and row sums (32 + 64 words), so peers can push partial
-  // tiles while this CTA is still in its main loop
-  p.stages = (BAR_LIMIT - STAGE0 - RECV_BYTES - 512) / p.stage_bytes;
-  if (p.stages > 3) p.stages = 3;
-  p.recv_off = STAGE0 + p.stages * p.stage_bytes;
-  p.aux_off = p.recv_off + RECV_BYTES;
-  p.bar_off = p.aux_off + 512;
-  p.total = 1024 + p.bar_off + 256;
-  return p;
-}
-
-// Offset of group-part `part` (8 groups) of row r in a 64-byte-swizzled index tile.
-__device__ __forceinline__ uint32_t sw64_off(int r, int part) {
-  return (uint32_t)(r * 64 + ((part ^ ((r >> 1) & 3)) << 4));
-}
-
-// Byte offset, inside the pair table, of the entry of codebook index i.
-__device__ __forceinline__ uint32_t table_off(uint32_t i) { return ((i + 1u) >> 1) << 2; }
-
-__device__ __forceinline__ void mma_ts_i8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                          uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// kind::i8 instruction descriptor: A unsigned 8-bit, B signed 8-bit, D int32, K-major.
-__host__ __device__ constexpr uint32_t idesc_u8s8_s32(uint32_t M, uint32_t N) {
-  return (2u << 4) | (0u << 7) | (1u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
-}
-
-// 32 lanes x 32 bit, 16 consecutive columns per thread.
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
-      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
-      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
-      "r"(v[15])
-      : "memory");
-}
-
-template <int BPW>
-__global__ void __launch_bounds__(agq::THREADS, 1)
-    k_act_gemm_q8(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmI1,
-                  const __grid_constant__ CUtensorMap tmI2, DeviceCodebook cb, int M, int N, int K,
-                  int rows_b, float alpha, const float* __restrict__ tok_scale,
-                  const int32_t* __restrict__ colsum, float* __restrict__ Y, int early_codes) {
-  using namespace agq;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
-  const Q8Plan plan = q8_plan(rows_b, BPW);
-  const int S = plan.stages;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + plan.bar_off);
-  uint64_t* full_code = bars;       // [3]
-  uint64_t* full_b = bars + 3;      // [3]
-  uint64_t* full_a = bars + 6;      // [3]
-  uint64_t* empty = bars + 9;       // [3]
-  uint64_t* acc_full = bars + 12;
-  uint64_t* table_full = bars + 13;
-  uint64_t* drain = bars + 14;
-  uint64_t* red_full = bars + 15;   // partial tiles pushed by the cluster peers
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
-  volatile uint32_t* abort_flag = tmem_slot + 1;
-  const uint32_t table_s = smem_u32(smem);
-  uint8_t* stage0 = smem + STAGE0;
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t crank = cluster_ctarank();
-  uint32_t ncl;
-  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(ncl));
-  const int n0 = (int)(blockIdx.x / ncl) * ROWS;
-  const int ksteps = K / KSTEP;
-  const int ks_begin = (int)((int64_t)crank * ksteps / ncl);
-  const int nks = (int)((int64_t)(crank + 1) * ksteps / ncl) - ks_begin;
-  const uint32_t code_tx = (uint32_t)(I1_BYTES + plan.i2_bytes);
-  const int chunks = (M + 3) >> 2;          // float4 chunks of a partial row
-  const int R = ROWS / (int)ncl;            // rows of the tile this CTA reduces
-  uint32_t* status = cb.status;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(&full_code[s], 1);
-      mbar_init(&full_b[s], 1);
-      mbar_init(&full_a[s], DEC_WARPS);
-      mbar_init(&empty[s], 1);
-    }
-    mbar_init(acc_full, 1);
-    mbar_init(table_full, 1);
-    mbar_init(drain, 1);
-    mbar_init(red_full, 1);
-    fence_mbar_init();
-    mbar_arrive_expect_tx(red_full, (uint32_t)((ncl - 1) * R * chunks * 16));
-    *abort_flag = 0u;
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, TMEM_COLS);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-  // publishes the initialised receive barrier to the cluster; the matching
-  // wait comes right before the first push into a peer
-  cluster_arrive();
-
-  if (warp == 0) {
-    if (lane == 0) {
-      tma_prefetch_desc(&tmB);
-      tma_prefetch_desc(&tmI1);
-      if (BPW > 2) tma_prefetch_desc(&tmI2);
-      mbar_arrive_expect_tx(table_full, TABLE_BYTES);
-      bulk_load(smem, cb.table, TABLE_BYTES, table_full);
-      const int pre = early_codes ? (nks < S ? nks : S) : 0;
-      for (int i = 0; i < pre; ++i) {
-        uint8_t* si1 = stage0 + i * plan.stage_bytes + plan.b_bytes;
-        const int g0 = (ks_begin + i) * GROUPS;
-        mbar_arrive_expect_tx(&full_code[i], code_tx);
-        tma_load_2d(si1, &tmI1, &full_code[i], g0, n0);
-        if (BPW > 2) tma_load_2d(si1 + I1_BYTES, &tmI2, &full_code[i], g0, n0);
-      }
-      grid_dep_wait();
-      uint32_t issued = 0;
-      for (int i = 0; i < nks; ++i) {
-        const int s = i % S;
-        const uint32_t round = (uint32_t)(i / S);
-        if (round > 0 &&
-            !mbar_wait_sleep(&empty[s], (round - 1u) & 1u, abort_flag, status, kDevTimeoutEmpty))
-          break;
-        uint8_t* sb = stage0 + s * plan.stage_bytes;
-        uint8_t* si1 = sb + plan.b_bytes;
-        const int k0 = (ks_begin + i) * KSTEP;
-        if (i >= pre) {
-          mbar_arrive_expect_tx(&full_code[s], code_tx);
-          tma_load_2d(si1, &tmI1, &full_code[s], k0 / 8, n0);
-          if (BPW > 2) tma_load_2d(si1 + I1_BYTES, &tmI2, &full_code[s], k0 / 8, n0);
-        }
-        mbar_arrive_expect_tx(&full_b[s], (uint32_t)plan.b_bytes);
-        tma_load_2d(sb, &tmB, &full_b[s], k0, 0);
-        tma_load_2d(sb + rows_b * 128, &tmB, &full_b[s], k0 + 128, 0);
-        ++issued;
-      }
-      if (ld_shared_volatile(abort_flag)) {
-        uint64_t t0 = global_timer_ns();
-        while (!mbar_try_wait(table_full, 0))
-          if (global_timer_ns() - t0 > 100000000ull) break;
-        for (uint32_t j = 0; j < (uint32_t)S && j < issued; ++j) {
-          const uint32_t idx = issued - 1 - j;
-          t0 = global_timer_ns();
-          while (!(mbar_try_wait(&full_b[idx % S], (idx / S) & 1u) &&
-                   mbar_try_wait(&full_code[idx % S], (idx / S) & 1u)))
-            if (global_timer_ns() - t0 > 100000000ull) break;
-        }
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      const uint32_t idesc = idesc_u8s8_s32(ROWS, (uint32_t)rows_b);
-      // slice j (32 int8 of K) of stage s: box (j >> 2) of 128 bytes of K, + (j & 3) * 32 bytes
-      const uint64_t bd0 = smem_desc(smem_u32(stage0), 16, 1024, 2);
-      const uint32_t box16 = (uint32_t)(rows_b * 128) >> 4;
-      const uint32_t stage16 = (uint32_t)plan.stage_bytes >> 4;
-      bool ok = true;
-      for (int i = 0; i < nks && ok; ++i) {
-        const int s = i % S;
-        const uint32_t ph = (uint32_t)(i / S) & 1u;
-        if (!mbar_wait_sleep(&full_a[s], ph, abort_flag, status, kDevTimeoutFull) ||
-            !mbar_wait_sleep(&full_b[s], ph, abort_flag, status, kDevTimeoutFull)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint64_t bds = bd0 + (uint64_t)((uint32_t)s * stage16);
-        const uint32_t a0 = tmem_base + D_COLS + (uint32_t)s * A_COLS;
-#pragma unroll
-        for (int j = 0; j < KSTEP / 32; ++j) {
-          const uint64_t bd = bds + (uint64_t)((uint32_t)(j >> 2) * box16 + (uint32_t)(j & 3) * 2u);
-          mma_ts_i8(tmem_base, a0 + (uint32_t)(j * 8), bd, idesc, (i > 0 || j > 0) ? 1u : 0u);
-        }
-        mma_commit(&empty[s]);
-      }
-      if (ok) mma_commit(acc_full);
-      mma_commit(drain);
-      uint64_t t0 = global_timer_ns();
-      while (!mbar_try_wait(drain, 0))
-        if (global_timer_ns() - t0 > 200000000ull) break;
-    }
-  } else {
-    // ------------------------------------------------------------ decoders
-    const int q = warp & 3;
-    const int part = (warp - 2) >> 2;
-    const int r = q * 32 + lane;
-    const uint32_t lane_bits = (uint32_t)(q * 32) << 16;
-    bool ok = mbar_wait_sleep(table_full, 0, abort_flag, status, kDevTimeoutFull);
-    for (int i = 0; i < nks && ok; ++i) {
-      const int s = i % S;
-      const uint32_t ph = (uint32_t)(i / S) & 1u;
-      if (!mbar_wait_sleep(&full_code[s], ph, abort_flag, status, kDevTimeoutFull)) break;
-      tc_fence_after();
-      const uint32_t si1 = smem_u32(stage0 + s * plan.stage_bytes + plan.b_bytes);
-      const uint4 c1 = lds128(si1 + sw64_off(r, part));
-      const uint32_t w1[4] = {c1.x, c1.y, c1.z, c1.w};
-      uint32_t w2[4] = {0u, 0u, 0u, 0u};
-      if (BPW == 4) {
-        const uint4 c2 = lds128(si1 + I1_BYTES + sw64_off(r, part));
-        w2[0] = c2.x; w2[1] = c2.y; w2[2] = c2.z; w2[3] = c2.w;
-      } else if (BPW == 3) {
-        // 32 one-byte indices per row, 32-byte swizzle: chunk (part >> 1), half (part & 1)
-        const uint32_t off = (uint32_t)(r * 32 + ((((part >> 1) ^ ((r >> 2) & 1))) << 4) +
-                                        (part & 1) * 8);
-        const uint2 c2 = lds64(si1 + I1_BYTES + off);
-        w2[0] = __byte_perm(c2.x, 0u, 0x4140);
-        w2[1] = __byte_perm(c2.x, 0u, 0x4342);
-        w2[2] = __byte_perm(c2.y, 0u, 0x4140);
-        w2[3] = __byte_perm(c2.y, 0u, 0x4342);
-      }
-      uint32_t v[16];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const uint32_t a = (w1[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
-        const uint32_t bb = (w2[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
-        const uint32_t ea = lds32(table_s + table_off(a));
-        const uint32_t eb = BPW > 2 ? lds32(table_s + table_off(bb)) : 0u;
-        decode_group_q8<BPW>(a, bb, ea, eb, v[2 * j], v[2 * j + 1]);
-      }
-      tmem_st16(tmem_base + lane_bits + D_COLS + (uint32_t)s * A_COLS + (uint32_t)(part * 16), v);
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&full_a[s]);
-    }
-  }
-
-  // ------------------------------------------------------------ epilogue ---
-  // Warps 2-5 hold row r of the int32 accumulator (TMEM lane r).  They first
-  // stage the per-token steps and row sums (written by the transform kernel)
-  // in shared memory, then wait for the accumulator.
-  float* s_sc = reinterpret_cast<float*>(smem + plan.aux_off);      // [32]
-  int32_t* s_cs = reinterpret_cast<int32_t*>(smem + plan.aux_off + 128);  // [64]
-  float4* recv = reinterpret_cast<float4*>(smem + plan.recv_off);
-  float y[32];
-  const bool epi = warp >= 2 && warp < 6;
-  const int er = (warp & 3) * 32 + lane;
-  if (epi) {
-    if (warp == 2) {
-      s_sc[lane] = lane < M ? __ldg(tok_scale + lane) : 0.0f;
-      s_cs[lane] = lane < rows_b ? __ldg(colsum + lane) : 0;
-      s_cs[32 + lane] = 32 + lane < rows_b ? __ldg(colsum + 32 + lane) : 0;
-    }
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    const bool have = nks > 0 && mbar_wait_sleep(acc_full, 0, abort_flag, status, kDevTimeoutMma);
-    tc_fence_after();
-    uint32_t dv[D_COLS];
-#pragma unroll
-    for (int c = 0; c < (int)D_COLS; c += 16)
-      if (c < rows_b)
-        tmem_ld16(tmem_base + (uint32_t)c + ((uint32_t)((warp & 3) * 32) << 16),
-                  *reinterpret_cast<uint32_t(*)[16]>(dv + c));
-    tmem_ld_wait();
-    // the +128 bias of the weight bytes contributes 128 * (row sum of Xq) over the
-    // whole K; the cluster's partial tiles are summed, so rank 0 alone removes it
-    const int corr = crank == 0 ? 128 : 0;
-#pragma unroll
-    for (int m = 0; m < 32; ++m) {
-      if (have && m < M) {
-        const int d0 = (int)dv[2 * m] - corr * s_cs[2 * m];
-        const int d1 = (int)dv[2 * m + 1] - corr * s_cs[2 * m + 1];
-        y[m] = s_sc[m] * ((float)d0 + (float)d1 * (1.0f / 128.0f));
-      } else {
-        y[m] = 0.0f;
-      }
-    }
-  }
-  // Reduce-scatter: row r goes to the CTA owning rows [owner*R, owner*R + R),
-  // slot [source rank][row - owner*R] of its receive area.
-  cluster_wait();
-  if (epi) {
-    const int owner = er / R;
-    const int slot = ((int)crank * R + (er - owner * R)) * chunks;
-    if (owner == (int)crank) {
-#pragma unroll
-      for (int c = 0; c < 8; ++c)
-        if (c < chunks) recv[slot + c] = make_float4(y[4 * c], y[4 * c + 1], y[4 * c + 2], y[4 * c + 3]);
-    } else {
-      const uint32_t raddr = mapa_shared(smem_u32(recv + slot), (uint32_t)owner);
-      const uint32_t rbar = mapa_shared(smem_u32(red_full), (uint32_t)owner);
-#pragma unroll
-      for (int c = 0; c < 8; ++c)
-        if (c < chunks)
-          st_async_v4(raddr + 16u * c, rbar,
-                      make_float4(y[4 * c], y[4 * c + 1], y[4 * c + 2], y[4 * c + 3]));
-    }
-  }
-  tc_fence_before();
-  __syncthreads();   // local rows written, every tensor-memory read done
-  {
-    const int r0 = (int)crank * R;
-    if (threadIdx.x < R * chunks) {
-      const bool got = mbar_wait_sleep(red_full, 0, abort_flag, status, kDevTimeoutCluster);
-      const int row = threadIdx.x % R, c = threadIdx.x / R;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int src = 0; src < (int)ncl; ++src) {
-        const float4 v4 = recv[(src * R + row) * chunks + c];
-        acc.x += v4.x; acc.y += v4.y; acc.z += v4.z; acc.w += v4.w;
-      }
-      const int n = n0 + r0 + row;
-      if (got && n < N) {
-        const float o[4] = {acc.x, acc.y, acc.z, acc.w};
-#pragma unroll
-        for (int t = 0; t < 4; ++t)
-          if (4 * c + t < M) Y[(size_t)(4 * c + t) * N + n] = alpha * o[t];
-      }
-    }
-  }
-  if (warp == 1) {
-    __syncwarp();
-    tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
-  }
-}
-
-template <int BPW>
-static cudaError_t launch_q8(const DeviceCodebook& cb, const ActQ8Args& a, int sm_count,
-                             cudaStream_t st) {
-  using namespace agq;
-  CUtensorMap tb, ti1, ti2;
-  if (!make_tmap_2d(&tb, a.Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.rows_b,
-                    (uint64_t)a.K, (uint32_t)a.rows_b, 128, CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorInvalidValue;
-  if (!make_tmap_2d(&ti1, a.idx1, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)a.N,
-                    (uint64_t)(a.K / 8), ROWS, GROUPS, CU_TENSOR_MAP_SWIZZLE_64B))
-    return cudaErrorInvalidValue;
-  if (BPW == 4) {
-    if (!make_tmap_2d(&ti2, a.idx2, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)a.N,
-                      (uint64_t)(a.K / 8), ROWS, GROUPS, CU_TENSOR_MAP_SWIZZLE_64B))
-      return cudaErrorInvalidValue;
-  } else if (BPW == 3) {
-    if (!make_tmap_2d(&ti2, a.idx2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.N,
-                      (uint64_t)(a.K / 8), ROWS, GROUPS, CU_TENSOR_MAP_SWIZZLE_32B))
-      return cudaErrorInvalidValue;
-  } else {
-    ti2 = ti1;
-  }
-  const Q8Plan plan = q8_plan(a.rows_b, BPW);
-  if (plan.stages < 2 || plan.total > kMaxDynSmem) return cudaErrorInvalidValue;
-  const int tiles = (int)((a.N + ROWS - 1) / ROWS);
-  const int ksteps = (int)(a.K / KSTEP);
-  int csize = 1;
-  while (csize < 8 && tiles * csize * 2 <= sm_count && csize * 2 <= ksteps) csize *= 2;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(tiles * csize));
-  cfg.blockDim = dim3(THREADS);
-  cfg.dynamicSmemBytes = (size_t)plan.total;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)csize;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = a.pdl ? 1 : 0;
-  cfg.attrs = attr;
-  cfg.numAttrs = 2;
-  cudaError_t e = ensure_smem_limit(k_act_gemm_q8<BPW>, kMaxDynSmem);
-  if (e != cudaSuccess) return e;
-  e = cudaLaunchKernelEx(&cfg, k_act_gemm_q8<BPW>, tb, ti1, ti2, cb, (int)a.M, (int)a.N,
-                         (int)a.K, a.rows_b, a.alpha, a.scales, a.colsum, a.Y, a.early_codes);
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
-}
-
-cudaError_t launch_act_gemm_q8(const DeviceCodebook& cb, const ActQ8Args& a, int sm_count,
-                               cudaStream_t st) {
-  if (a.bpw == 2) return launch_q8<2>(cb, a, sm_count, st);
-  if (a.bpw == 3) return launch_q8<3>(cb, a, sm_count, st);
-  return launch_q8<4>(cb, a, sm_count, st);
-}
-
 cudaError_t launch_act_gemm(const DeviceCodebook& cb, const ActGemmArgs& a, int sm_count,
                             cudaStream_t st) {
   return launch_act_gemm_generic(cb, a, sm_count, st);

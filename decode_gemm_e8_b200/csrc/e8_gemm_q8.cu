@@ -1,0 +1,595 @@
+// Fused decode + GEMM for small batches (up to 32 tokens), int8 tensor cores.
+//
+//   Y[m][n] = alpha * sum_k (FWHT D x_m)_k z_nk                 (activation-side RHT)
+//
+// z_n = m (c1 + beta c2) is the integer codebook vector of each 8-weight group
+// of row n ("glq 0.1.1", "How it works", item 1, and the "Bit widths" table),
+// |z| <= 30.  The transformed activations arrive as two int8 pieces per token
+// (rows 2m and 2m + 1 of Xq, written by k_act_q8) with a per-token step s_m:
+//   xt_m = s_m (q0_m + q1_m / 128).
+// The weight operand is z + 128 as unsigned bytes, decoded on chip straight
+// into tensor memory; tcgen05.mma kind::i8 accumulates exactly in int32 and
+// the epilogue removes the +128 bias with the row sums of Xq:
+//   y[m][n] = alpha s_m ((D[n][2m] - 128 cs[2m]) + (D[n][2m+1] - 128 cs[2m+1]) / 128).
+//
+// Work split (stream-K): the (128-row tile, 128-wide K unit) pairs are laid out
+// tile by tile and every CTA of a one-per-SM grid takes a contiguous run of
+// them, so all SMs get the same number of units within one.  A run covers at
+// most a few tiles; the partial tile of each is added into Y (zeroed by the
+// transform kernel that precedes this one) by a TMA bulk reduce-add, so the
+// order of the few partial sums of an output is not fixed.
+//
+// Roles (one CTA per SM):
+//   warp 0      TMA producer: the codebook pair table (once), the index tiles
+//               (a ring released by the decoders as soon as they hold the
+//               indices in registers; filled before waiting for the transform
+//               kernel) and the Xq tiles (a ring released by the MMA)
+//   warp 1      tensor-memory allocation; one thread issues tcgen05.mma
+//               (M = 128 weight rows, N = rows_b, K = 32) and the commits
+//   warps 2-17  decoders, two groups of eight taking alternate units: each
+//               thread owns one weight row (its TMEM lane) and 8 of the 16
+//               groups of a unit: index loads, pair-table gathers, combine,
+//               tcgen05.st of 16 columns into the unit's operand stage
+//   warps 18-21 epilogue, one per TMEM lane quarter: accumulator -> shared
+//               memory -> bulk reduce-add into Y
+// The tensor cores are used only for the X W^T contraction.
+#include "e8_common.cuh"
+#include "e8_codebook.cuh"
+#include "e8_internal.h"
+#include "e8_tmap.h"
+
+namespace e8 {
+
+namespace sk {
+constexpr int ROWS = 128;                 // weight rows per tile (MMA M)
+constexpr int KU = 128;                   // K of one work unit
+constexpr int GROUPS = KU / 8;            // groups of a row in one unit
+constexpr int DEC_GROUPS = 2;
+constexpr int DEC_WARPS = 8 * DEC_GROUPS;
+constexpr int EPI_WARP0 = 2 + DEC_WARPS;
+constexpr int THREADS = 32 * (EPI_WARP0 + 4);
+constexpr int TABLE_BYTES = 131088;       // 32769 u32 entries, padded to 16 bytes
+constexpr int I1_BYTES = ROWS * GROUPS * 2;
+constexpr uint32_t ACC_COLS = 64;         // int32 accumulator columns per buffer
+constexpr uint32_t A_COLS = KU / 4;       // 4 int8 weights per TMEM column
+constexpr int MAX_STAGES = 8;
+constexpr int AUX_BYTES = 512;            // per-token steps [32] and row sums [64]
+constexpr int BAR_BYTES = 512;
+// shared memory left free on the SM for a CTA of the activation transform
+// (K = 4096: 16 KB), so that it can run next to this kernel's CTA
+constexpr int CORESIDENT_RESERVE = 18 * 1024;
+}  // namespace sk
+
+// Shared memory: the pair table at offset 0 of the dynamic window (so its
+// address folds into the gather instructions), then, from the next 1 KB
+// boundary: the Xq ring (sx stages), the index-tile ring (sc stages), the
+// staging tile of the output (16 or 32 tokens x 128 fp32), the per-token steps
+// and row sums, and the barriers.  Offsets below are relative to that
+// boundary.  The decoded operands live in a ring of sa tensor-memory stages.
+struct SkPlan {
+  int sa, sx, sc, b_bytes, code_bytes, i2_bytes, code_off, y_off, aux_off, bar_off, total;
+  uint32_t tmem_cols;
+};
+
+__host__ __device__ inline SkPlan sk_plan(int rows_b, int bpw) {
+  using namespace sk;
+  SkPlan p;
+  p.b_bytes = rows_b * KU;                                  // multiple of 2 KB
+  p.i2_bytes = bpw == 2 ? 0 : (bpw == 3 ? ROWS * GROUPS : ROWS * GROUPS * 2);
+  p.code_bytes = I1_BYTES + p.i2_bytes;                     // multiple of 1 KB
+  const int y_bytes = (rows_b <= 32 ? 16 : 32) * ROWS * 4;
+  const int budget = kMaxDynSmem - TABLE_BYTES - 1024 - AUX_BYTES - BAR_BYTES -
+                     CORESIDENT_RESERVE - y_bytes;
+  p.sa = MAX_STAGES;                                        // 2 x 64 + 8 x 32 TMEM columns
+  // Xq tiles are requested after the transform kernel ends and take ~1 us to
+  // land, so the Xq ring holds a CTA's whole run where it can (7 units of
+  // 128 at 4096 x 4096); the index ring gets the rest, at least 4 stages
+  for (p.sx = 7; p.sx > 2; --p.sx)
+    if (budget - p.sx * p.b_bytes >= 4 * p.code_bytes) break;
+  p.sc = (budget - p.sx * p.b_bytes) / p.code_bytes;
+  if (p.sc > MAX_STAGES) p.sc = MAX_STAGES;
+  p.code_off = p.sx * p.b_bytes;
+  p.y_off = p.code_off + p.sc * p.code_bytes;
+  p.aux_off = p.y_off + y_bytes;
+  p.bar_off = p.aux_off + AUX_BYTES;
+  p.total = TABLE_BYTES + 1024 + p.bar_off + BAR_BYTES;
+  p.tmem_cols = 512u;
+  return p;
+}
+
+// Byte offset, inside the pair table, of the entry of codebook index i
+// (slot (i + 1) >> 1), for the index in the low / high 16 bits of w.
+__device__ __forceinline__ uint32_t sk_off_lo(uint32_t w) {
+  return (((w & 0xFFFFu) << 1) + 2u) & 0x3FFFCu;
+}
+__device__ __forceinline__ uint32_t sk_off_hi(uint32_t w) { return ((w >> 15) + 2u) & 0x3FFFCu; }
+__device__ __forceinline__ uint32_t sk_entry(const uint8_t* table, uint32_t off) {
+  return *reinterpret_cast<const uint32_t*>(table + off);
+}
+
+// Offset of the 16-byte half `h` of row r in a 32-byte-swizzled index tile.
+__device__ __forceinline__ uint32_t sw32_off(int r, int h) {
+  return (uint32_t)(r * 32 + ((h ^ ((r >> 2) & 1)) << 4));
+}
+
+__device__ __forceinline__ void sk_mma_i8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// kind::i8 instruction descriptor: A unsigned 8-bit, B signed 8-bit, D int32,
+// both operands K-major.
+__host__ __device__ constexpr uint32_t sk_idesc(uint32_t M, uint32_t N) {
+  return (2u << 4) | (0u << 7) | (1u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+
+__device__ __forceinline__ void sk_tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15])
+      : "memory");
+}
+
+// No memory clobber: nothing later in the thread depends on the sum, and the
+// shared-memory loads feeding the next adds may then be hoisted past it.
+__device__ __forceinline__ void red_add_f32(float* p, float v) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v));
+}
+
+// Element-wise fp32 add of a shared-memory tile into global memory by the TMA
+// unit (box of the tensor map; elements outside the tensor are skipped).
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, uint32_t smem_src,
+                                                  int32_t x, int32_t y) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%1, %2}], [%3];"
+      ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_src)
+      : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Units [begin, end) of CTA c when U units are spread over G CTAs.
+__device__ __forceinline__ int sk_unit_begin(int c, int U, int G) {
+  return (int)(((int64_t)c * U) / G);
+}
+
+// CW: accumulator columns read by the epilogue (32 for up to 16 tokens, else 64).
+// tmY: Y [M][N] fp32, box 128 x M (valid when use_tma_y; else fp32 atomics).
+template <int BPW, int CW>
+__global__ void __launch_bounds__(sk::THREADS, 1)
+    k_gemm_q8(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmI1,
+              const __grid_constant__ CUtensorMap tmI2, const __grid_constant__ CUtensorMap tmY,
+              DeviceCodebook cb, int M, int N, int K, int rows_b, float alpha,
+              const float* __restrict__ tok_scale, const int32_t* __restrict__ colsum,
+              float* __restrict__ Y, int use_tma_y, int early_codes) {
+  using namespace sk;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  const uint8_t* table = smem_raw;
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + TABLE_BYTES + 1023) & ~uintptr_t(1023));
+  const SkPlan plan = sk_plan(rows_b, BPW);
+  const int SA = plan.sa, SX = plan.sx, SC = plan.sc;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + plan.bar_off);
+  uint64_t* full_code = bars;                     // [SC] index tiles landed
+  uint64_t* code_empty = bars + MAX_STAGES;       // [SC] decoders hold the indices
+  uint64_t* full_a = bars + 2 * MAX_STAGES;       // [SA] operand decoded + Xq landed
+  uint64_t* a_empty = bars + 3 * MAX_STAGES;      // [SA] MMAs of the stage done
+  uint64_t* acc_full = bars + 4 * MAX_STAGES;     // [2]
+  uint64_t* acc_empty = acc_full + 2;             // [2]
+  uint64_t* table_full = acc_full + 4;
+  uint64_t* drain = acc_full + 5;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 6);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+  float* s_sc = reinterpret_cast<float*>(smem + plan.aux_off);             // [32]
+  int32_t* s_cs = reinterpret_cast<int32_t*>(smem + plan.aux_off + 128);   // [64]
+  float* s_y = reinterpret_cast<float*>(smem + plan.y_off);                // [M][128]
+  uint8_t* xq_ring = smem;
+  uint8_t* code_ring = smem + plan.code_off;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kunits = K / KU;
+  const int tiles = (N + ROWS - 1) / ROWS;
+  const int U = tiles * kunits;
+  const int u_begin = sk_unit_begin((int)blockIdx.x, U, (int)gridDim.x);
+  const int nu = sk_unit_begin((int)blockIdx.x + 1, U, (int)gridDim.x) - u_begin;
+  const int first_tile = u_begin / kunits;
+  const uint32_t code_tx = (uint32_t)plan.code_bytes;
+  uint32_t* status = cb.status;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < SC; ++s) {
+      mbar_init(&full_code[s], 1);
+      mbar_init(&code_empty[s], 8);
+    }
+    for (int s = 0; s < SA; ++s) {
+      mbar_init(&full_a[s], 9);   // eight decoder warps + the Xq tile
+      mbar_init(&a_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);
+    }
+    mbar_init(table_full, 1);
+    mbar_init(drain, 1);
+    fence_mbar_init();
+    *abort_flag = 0u;
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, plan.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint32_t tmem_a = tmem_base + 2 * ACC_COLS;
+  // the next kernel of the stream may be launched now: it waits for this grid
+  // before it touches anything this grid reads or writes
+  if (threadIdx.x == 0) grid_dep_launch();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmB);
+      tma_prefetch_desc(&tmI1);
+      if (BPW > 2) tma_prefetch_desc(&tmI2);
+      if (use_tma_y) tma_prefetch_desc(&tmY);
+      // the pair table in eight 16 KB pieces plus the last entry, starting at a
+      // CTA-dependent piece so that the SMs do not all read the same L2 lines
+      mbar_arrive_expect_tx(table_full, TABLE_BYTES);
+      for (int j = 0; j < 8; ++j) {
+        const int c = (j + (int)blockIdx.x) & 7;
+        bulk_load(smem_raw + c * 16384, reinterpret_cast<const uint8_t*>(cb.table) + c * 16384,
+                  16384, table_full);
+      }
+      bulk_load(smem_raw + 8 * 16384, reinterpret_cast<const uint8_t*>(cb.table) + 8 * 16384, 16,
+                table_full);
+      auto load_codes = [&](int i, int s) {
+        const int u = u_begin + i;
+        uint8_t* dst = code_ring + s * plan.code_bytes;
+        mbar_arrive_expect_tx(&full_code[s], code_tx);
+        tma_load_2d(dst, &tmI1, &full_code[s], (u % kunits) * GROUPS, (u / kunits) * ROWS);
+        if (BPW > 2)
+          tma_load_2d(dst + I1_BYTES, &tmI2, &full_code[s], (u % kunits) * GROUPS,
+                      (u / kunits) * ROWS);
+      };
+      // Index tiles do not depend on the preceding kernel: before waiting for
+      // it, load those of the first SC + SA units (the decoders of units
+      // below SA wait for nothing but their tiles, so the waits for free
+      // stages here cannot depend on the MMAs).
+      int cn = 0;                    // next unit whose index tiles to load
+      int cs = 0;
+      uint32_t cph = 0;
+      bool ok = true;
+      auto next_codes = [&](int limit) {
+        while (ok && cn < limit) {
+          if (cn >= SC &&
+              !mbar_wait_sleep(&code_empty[cs], cph ^ 1u, abort_flag, status, kDevTimeoutEmpty)) {
+            ok = false;
+            break;
+          }
+          load_codes(cn, cs);
+          ++cn;
+          if (++cs == SC) {
+            cs = 0;
+            cph ^= 1u;
+          }
+        }
+      };
+      if (early_codes) next_codes(nu < SC + SA ? nu : SC + SA);
+      grid_dep_wait();
+      int sa = 0;                    // operand stage of unit i
+      uint32_t aph = 0;
+      int ja = 0;                    // operand stage of unit i - SX, whose MMAs free
+      uint32_t jph = 0;              // the Xq stage of unit i
+      for (int i = 0; i < nu && ok; ++i) {
+        next_codes(i + SC < nu ? i + SC : nu);
+        if (!ok) break;
+        if (i >= SX) {
+          if (!mbar_wait_sleep(&a_empty[ja], jph, abort_flag, status, kDevTimeoutEmpty)) break;
+          if (++ja == SA) {
+            ja = 0;
+            jph ^= 1u;
+          }
+        }
+        const int u = u_begin + i;
+        mbar_arrive_expect_tx(&full_a[sa], (uint32_t)plan.b_bytes);
+        tma_load_2d(xq_ring + (i % SX) * plan.b_bytes, &tmB, &full_a[sa], (u % kunits) * KU, 0);
+        if (++sa == SA) {
+          sa = 0;
+          aph ^= 1u;
+        }
+      }
+      (void)aph;
+      if (ld_shared_volatile(abort_flag)) {
+        // let the copies in flight land before the CTA exits (bounded waits:
+        // a stage's barrier may never complete once the other roles stopped)
+        uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(table_full, 0))
+          if (global_timer_ns() - t0 > 100000000ull) break;
+        t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 1000000ull) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // this single thread's loop is latency-bound (each barrier test costs
+      // ~100 cycles): everything per unit is incremental, and a stage is
+      // released only when the producer will refill it
+      const uint32_t idesc = sk_idesc(ROWS, (uint32_t)rows_b);
+      const uint64_t bd0 = smem_desc(smem_u32(xq_ring), 16, 1024, 2);
+      const uint32_t stage16 = (uint32_t)plan.b_bytes >> 4;
+      int seg = 0;
+      int s = 0;                     // operand stage (tensor memory)
+      uint32_t ph = 0;
+      int sxi = 0;                   // Xq stage
+      int ku = u_begin - first_tile * kunits;
+      uint64_t bds = bd0;
+      uint32_t a0 = tmem_a;
+      for (int i = 0; i < nu; ++i) {
+        const bool first = (i == 0 || ku == 0);
+        const bool last = (i == nu - 1 || ku == kunits - 1);
+        if (first && i > 0) ++seg;
+        const int b = seg & 1;
+        if (first && seg >= 2 &&
+            !mbar_wait_sleep(&acc_empty[b], (uint32_t)((seg - 2) >> 1) & 1u, abort_flag, status,
+                             kDevTimeoutMma))
+          break;
+        if (!mbar_wait_sleep(&full_a[s], ph, abort_flag, status, kDevTimeoutFull)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + (uint32_t)b * ACC_COLS;
+#pragma unroll
+        for (int j = 0; j < KU / 32; ++j)
+          sk_mma_i8(d, a0 + (uint32_t)(j * 8), bds + (uint64_t)(j * 2), idesc,
+                    (first && j == 0) ? 0u : 1u);
+        // the stage is reused by unit i + SX (Xq) and unit i + SA (operand)
+        if (i + SX < nu) mma_commit(&a_empty[s]);
+        if (last) mma_commit(&acc_full[b]);
+        if (++ku == kunits) ku = 0;
+        if (++s == SA) {
+          s = 0;
+          ph ^= 1u;
+          a0 = tmem_a;
+        } else {
+          a0 += A_COLS;
+        }
+        if (++sxi == SX) {
+          sxi = 0;
+          bds = bd0;
+        } else {
+          bds += stage16;
+        }
+      }
+      mma_commit(drain);
+      uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(drain, 0))
+        if (global_timer_ns() - t0 > 200000000ull) break;
+    }
+  } else if (warp < EPI_WARP0) {
+    // ------------------------------------------------------------ decoders
+    const int dw = warp - 2;
+    const int q = warp & 3;
+    const int p = dw >> 2;
+    const int dg = p >> 1, h = p & 1;
+    const int r = q * 32 + lane;
+    const uint32_t lane_bits = (uint32_t)(q * 32) << 16;
+    bool ok = mbar_wait_sleep(table_full, 0, abort_flag, status, kDevTimeoutFull);
+    int cs = dg % SC, as = dg % SA;
+    uint32_t cph = 0, aph = 0;
+    for (int i = dg; i < nu && ok; i += DEC_GROUPS) {
+      if (!mbar_wait_sleep(&full_code[cs], cph, abort_flag, status, kDevTimeoutFull)) break;
+      const uint8_t* si1 = code_ring + cs * plan.code_bytes;
+      const uint4 c1 = *reinterpret_cast<const uint4*>(si1 + sw32_off(r, h));
+      uint4 c2 = make_uint4(0u, 0u, 0u, 0u);
+      if (BPW == 4) {
+        c2 = *reinterpret_cast<const uint4*>(si1 + I1_BYTES + sw32_off(r, h));
+      } else if (BPW == 3) {
+        const uint2 c = *reinterpret_cast<const uint2*>(si1 + I1_BYTES + r * 16 + h * 8);
+        c2 = make_uint4(__byte_perm(c.x, 0u, 0x4140), __byte_perm(c.x, 0u, 0x4342),
+                        __byte_perm(c.y, 0u, 0x4140), __byte_perm(c.y, 0u, 0x4342));
+      }
+      // the indices are in registers: the index-tile stage can be refilled
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&code_empty[cs]);
+      // the operand stage must have been read by the MMAs of unit i - SA
+      if (i >= SA &&
+          !mbar_wait_sleep(&a_empty[as], aph ^ 1u, abort_flag, status, kDevTimeoutMma))
+        break;
+      tc_fence_after();
+      const uint32_t w1[4] = {c1.x, c1.y, c1.z, c1.w};
+      const uint32_t w2[4] = {c2.x, c2.y, c2.z, c2.w};
+      uint32_t v[16];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t ea0 = sk_entry(table, sk_off_lo(w1[k]));
+        const uint32_t ea1 = sk_entry(table, sk_off_hi(w1[k]));
+        const uint32_t eb0 = BPW > 2 ? sk_entry(table, sk_off_lo(w2[k])) : 0u;
+        const uint32_t eb1 = BPW > 2 ? sk_entry(table, sk_off_hi(w2[k])) : 0u;
+        decode_group_q8<BPW>(w1[k] & 0xFFFFu, w2[k] & 0xFFFFu, ea0, eb0, v[4 * k], v[4 * k + 1]);
+        decode_group_q8<BPW>(w1[k] >> 16, w2[k] >> 16, ea1, eb1, v[4 * k + 2], v[4 * k + 3]);
+      }
+      sk_tmem_st16(tmem_a + lane_bits + (uint32_t)as * A_COLS + (uint32_t)(h * 16), v);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&full_a[as]);
+      cs += DEC_GROUPS;
+      if (cs >= SC) {
+        cs -= SC;
+        cph ^= 1u;
+      }
+      as += DEC_GROUPS;
+      if (as >= SA) {
+        as -= SA;
+        aph ^= 1u;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    const bool issuer = warp == EPI_WARP0 && lane == 0;
+    grid_dep_wait();   // steps, row sums and the zeroed Y come from the transform
+    if (warp == EPI_WARP0) {
+      s_sc[lane] = lane < M ? alpha * __ldg(tok_scale + lane) : 0.0f;
+      s_cs[lane] = lane < rows_b ? __ldg(colsum + lane) : 0;
+      s_cs[32 + lane] = 32 + lane < rows_b ? __ldg(colsum + 32 + lane) : 0;
+    }
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    const int nseg = nu > 0 ? (u_begin + nu - 1) / kunits - first_tile + 1 : 0;
+    // every epilogue thread runs the same sequence of named barriers, also
+    // after a failed wait (it then only skips the work)
+    bool ok = true;
+    for (int seg = 0; seg < nseg; ++seg) {
+      const int b = seg & 1;
+      ok = ok && mbar_wait_sleep(&acc_full[b], (uint32_t)(seg >> 1) & 1u, abort_flag, status,
+                                 kDevTimeoutMma);
+      tc_fence_after();
+      const int tile = first_tile + seg;
+      const int n = tile * ROWS + r;
+      // the segment holding K unit 0 of its tile removes the bias of the whole row
+      const int corr = tile * kunits >= u_begin ? 128 : 0;
+      // 32 accumulator columns (16 tokens) per pass
+#pragma unroll
+      for (int c0 = 0; c0 < CW; c0 += 32) {
+        if (!ok) break;
+        uint32_t dv[32];
+        const uint32_t ta = tmem_base + (uint32_t)b * ACC_COLS + (uint32_t)c0 +
+                            ((uint32_t)(q * 32) << 16);
+        tmem_ld16(ta, *reinterpret_cast<uint32_t(*)[16]>(dv));
+        if (c0 + 16 < rows_b) {
+          tmem_ld16(ta + 16, *reinterpret_cast<uint32_t(*)[16]>(dv + 16));
+        } else {
+#pragma unroll
+          for (int j = 16; j < 32; ++j) dv[j] = 0u;
+        }
+        tmem_ld_wait();
+        if (use_tma_y) {
+          // tokens past M have zero steps and row sums: staged as zeros (the
+          // bulk reduce covers only M rows), no branch in the loop
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int m = (c0 >> 1) + j;
+            const int d0 = (int)dv[2 * j] - corr * s_cs[2 * m];
+            const int d1 = (int)dv[2 * j + 1] - corr * s_cs[2 * m + 1];
+            s_y[m * ROWS + r] = s_sc[m] * ((float)d0 + (float)d1 * (1.0f / 128.0f));
+          }
+        } else if (n < N) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int m = (c0 >> 1) + j;
+            const int d0 = (int)dv[2 * j] - corr * s_cs[2 * m];
+            const int d1 = (int)dv[2 * j + 1] - corr * s_cs[2 * m + 1];
+            if (m < M)
+              red_add_f32(Y + (size_t)m * N + n,
+                          s_sc[m] * ((float)d0 + (float)d1 * (1.0f / 128.0f)));
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0 && ok) mbar_arrive(&acc_empty[b]);
+      if (use_tma_y) {
+        // the staged tile [M][128] goes to Y[0..M)[tile * 128 ..) by one bulk
+        // reduce-add; the stage is reused only after the unit has read it
+        fence_proxy_async_smem();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (issuer && ok) {
+          tma_reduce_add_2d(&tmY, smem_u32(s_y), tile * ROWS, 0);
+          bulk_wait_read_all();
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+      }
+    }
+    if (issuer && use_tma_y) bulk_wait_all();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, plan.tmem_cols);
+  }
+}
+
+template <int BPW>
+static cudaError_t launch_gemm_q8(const DeviceCodebook& cb, const ActQ8Args& a, int sm_count,
+                                  cudaStream_t st) {
+  using namespace sk;
+  if (a.rows_b < 16 || a.rows_b > 64 || (a.rows_b % 16) != 0 || a.M < 1 || a.M > 32 ||
+      2 * a.M > a.rows_b || (a.K % KU) != 0)
+    return cudaErrorInvalidValue;
+  CUtensorMap tb, ti1, ti2, ty;
+  if (!make_tmap_2d(&tb, a.Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.rows_b,
+                    (uint64_t)a.K, (uint32_t)a.rows_b, KU, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&ti1, a.idx1, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)a.N,
+                    (uint64_t)(a.K / 8), ROWS, GROUPS, CU_TENSOR_MAP_SWIZZLE_32B))
+    return cudaErrorInvalidValue;
+  if (BPW == 4) {
+    if (!make_tmap_2d(&ti2, a.idx2, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)a.N,
+                      (uint64_t)(a.K / 8), ROWS, GROUPS, CU_TENSOR_MAP_SWIZZLE_32B))
+      return cudaErrorInvalidValue;
+  } else if (BPW == 3) {
+    if (!make_tmap_2d(&ti2, a.idx2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.N,
+                      (uint64_t)(a.K / 8), ROWS, GROUPS, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorInvalidValue;
+  } else {
+    ti2 = ti1;
+  }
+  // Y by bulk reduce-add when its rows are 16-byte multiples (else fp32 atomics)
+  int use_tma_y = (a.N % 4) == 0 &&
+                  make_tmap_2d(&ty, a.Y, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)a.M,
+                               (uint64_t)a.N, (uint32_t)a.M, ROWS, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (!use_tma_y) ty = tb;
+  const SkPlan plan = sk_plan(a.rows_b, BPW);
+  if (plan.sa < 2 || plan.sc < 2 || plan.total > kMaxDynSmem) return cudaErrorInvalidValue;
+  const int64_t units = ((a.N + ROWS - 1) / ROWS) * (a.K / KU);
+  if (units > INT32_MAX) return cudaErrorInvalidValue;
+  const int grid = (int)(units < sm_count ? units : sm_count);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = (size_t)plan.total;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = a.pdl ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  auto kern = a.rows_b <= 32 ? k_gemm_q8<BPW, 32> : k_gemm_q8<BPW, 64>;
+  cudaError_t e = ensure_smem_limit(kern, kMaxDynSmem);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared);
+  if (e != cudaSuccess) return e;
+  e = cudaLaunchKernelEx(&cfg, kern, tb, ti1, ti2, ty, cb, (int)a.M, (int)a.N, (int)a.K,
+                         a.rows_b, a.alpha, a.scales, a.colsum, a.Y, use_tma_y, a.early_codes);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_act_gemm_q8(const DeviceCodebook& cb, const ActQ8Args& a, int sm_count,
+                               cudaStream_t st) {
+  if (a.bpw == 2) return launch_gemm_q8<2>(cb, a, sm_count, st);
+  if (a.bpw == 3) return launch_gemm_q8<3>(cb, a, sm_count, st);
+  return launch_gemm_q8<4>(cb, a, sm_count, st);
+}
+
+}  // namespace e8

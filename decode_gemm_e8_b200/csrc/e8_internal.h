@@ -85,7 +85,9 @@ cudaError_t launch_act_gemm(const DeviceCodebook& cb, const ActGemmArgs& a, int 
                             cudaStream_t st);
 
 // int8 path for up to 32 tokens: Xq int8 [rows_b][K] (token m: rows 2m, 2m + 1),
-// per-token steps and per-row column sums from launch_act_q8.
+// per-token steps and per-row column sums from launch_act_q8.  The kernel adds
+// its partial tiles into Y, which must hold zeros when it starts (the
+// transform kernel zeroes it when given Y).
 struct ActQ8Args {
   const int8_t* Xq;
   const float* scales;   // [M]
@@ -102,9 +104,11 @@ struct ActQ8Args {
 };
 cudaError_t launch_act_gemm_q8(const DeviceCodebook& cb, const ActQ8Args& a, int sm_count,
                                cudaStream_t st);
+// When Yz is not null the kernel also zeroes Yz[0, yz_elems) (the fp32 output
+// that launch_act_gemm_q8 accumulates into), after the preceding kernel ends.
 cudaError_t launch_act_q8(const uint16_t* X, int64_t M, int64_t K, uint64_t seed, int8_t* Xq,
                           float* scales, int32_t* colsum, int64_t rows, cudaStream_t st,
-                          int pdl);
+                          int pdl, float* Yz = nullptr, int64_t yz_elems = 0);
 
 // Layout of the int8 activation buffer: Xq [rows][K] int8, then the per-token
 // steps (fp32 [M]) and the per-row column sums (int32 [rows]), each part

@@ -131,7 +131,11 @@ int e8_act_rht(const uint16_t* X, int64_t M, int64_t K, uint64_t rht_seed, uint1
  * In the DECODED_W and SIMT modes the product uses W_dec itself; in the
  * ACT_RHT modes it uses the unrounded decoded weights (relative Frobenius
  * difference to the W_dec product about 1.7e-3, from the bf16 rounding of
- * W_dec).  workspace: at least e8_workspace_bytes(mode, M, N, K, bpw) bytes. */
+ * W_dec).  In E8_GEMM_ACT_RHT with up to 32 tokens (the int8 path, see
+ * e8_gemm_xt) the K range of an output is split over several CTAs whose
+ * partial sums are added with fp32 atomics: the last bits of Y can differ
+ * between runs.  workspace: at least e8_workspace_bytes(mode, M, N, K, bpw)
+ * bytes. */
 int e8_gemm(const e8_codebook* cb, const uint16_t* X, int64_t M, const uint16_t* idx1,
             const void* idx2, int64_t N, int64_t K, int bpw, uint64_t rht_seed, float scale,
             float* Y, int mode, void* workspace, size_t ws_bytes, void* stream);
@@ -154,10 +158,13 @@ size_t e8_act_q8_bytes(int64_t M, int64_t K);
 
 /* Second half of E8_GEMM_ACT_RHT: the fused decode + int8 tensor-core GEMM on
  * a buffer written by e8_act_rht_q8 for the same M, K and rht_seed:
- * Y fp32 [M][N] = alpha * s_m * ((q0 + q1 / 128) . z) over each weight row, z
- * the integer codebook vectors decoded on chip.  One transform can serve every
- * weight matrix that shares K and rht_seed (for instance q, k and v).  Same
- * shape limits as e8_act_rht_q8.  No workspace. */
+ * Y fp32 [M][N] += alpha * s_m * ((q0 + q1 / 128) . z) over each weight row, z
+ * the integer codebook vectors decoded on chip.  The product is ADDED into Y
+ * (zero Y first for a plain product); the partial sums of one output, from
+ * the CTAs that split its K range, are added with fp32 atomics, so the last
+ * bits of Y can differ from run to run (relative differences of order 1e-7).
+ * One transform can serve every weight matrix that shares K and rht_seed (for
+ * instance q, k and v).  Same shape limits as e8_act_rht_q8.  No workspace. */
 int e8_gemm_xt(const e8_codebook* cb, const void* xq, int64_t M, const uint16_t* idx1,
                const void* idx2, int64_t N, int64_t K, int bpw, float scale, float* Y,
                void* stream);

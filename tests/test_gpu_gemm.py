@@ -20,6 +20,7 @@ pytestmark = pytest.mark.gpu
 
 BAR = 2e-3
 BAR_DECODED = 1e-4
+REPEAT = 1e-6   # run-to-run agreement of the int8 path (atomic partial sums)
 ACT_MODES = [e8.E8_GEMM_ACT_RHT, e8.E8_GEMM_ACT_RHT_SMEM]
 ALL_MODES = ACT_MODES + [e8.E8_GEMM_DECODED_W, e8.E8_GEMM_SIMT]
 
@@ -136,7 +137,7 @@ def test_act_rht_hi_lo(gcb):
     assert not Xt[2 * M:].any()
 
 
-def test_act_gemm_is_deterministic(gcb):
+def test_act_gemm_repeatable(gcb):
     wl = synth.workloads()["llama_4096_b4"]
     lay = wl.layers[0]
     W = lay.weights()
@@ -147,7 +148,10 @@ def test_act_gemm_is_deterministic(gcb):
                             mode=e8.E8_GEMM_ACT_RHT))
     b = gu.to_np(e8.e8_gemm(gcb, X, i1, i2, lay.N, lay.K, lay.bpw, lay.rht_seed, s,
                             mode=e8.E8_GEMM_ACT_RHT))
-    assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+    # the int8 path adds the partial tiles of an output with fp32 atomics in no
+    # fixed order; two runs agree to within a few rounding steps
+    assert gu.rel_fro(a, b) < REPEAT
+    assert np.max(np.abs(a - b)) <= 1e-5 * np.max(np.abs(a))
     assert e8.e8_sync_status(gcb) == e8.E8_OK
 
 
@@ -164,7 +168,11 @@ def test_gemm_xt_matches_gemm_and_graph_capture(gcb):
     assert e8.e8_gemm_xt_rows(16) == 32
     xq = e8.e8_act_rht_q8(X, lay.rht_seed)
     b = e8.e8_gemm_xt(gcb, xq, 16, i1, i2, lay.N, lay.K, lay.bpw, s)
-    assert np.array_equal(gu.to_np(a).view(np.uint32), gu.to_np(b).view(np.uint32))
+    # partial tiles are added with atomics: equal up to the order of a few fp32 adds
+    assert gu.rel_fro(gu.to_np(b), gu.to_np(a)) < REPEAT
+    # e8_gemm_xt adds into Y
+    b2 = e8.e8_gemm_xt(gcb, xq, 16, i1, i2, lay.N, lay.K, lay.bpw, s, Y=b.clone())
+    assert gu.rel_fro(gu.to_np(b2), 2.0 * gu.to_np(a)) < REPEAT
     # the same call captured in a CUDA graph and replayed
     Y = torch.empty_like(a)
     ws = torch.empty(e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT, 16, lay.N, lay.K, lay.bpw),
@@ -177,10 +185,10 @@ def test_gemm_xt_matches_gemm_and_graph_capture(gcb):
     with torch.cuda.graph(g, stream=st):
         e8.e8_gemm(gcb, X, i1, i2, lay.N, lay.K, lay.bpw, lay.rht_seed, s,
                    mode=e8.E8_GEMM_ACT_RHT, Y=Y, workspace=ws, stream=st)
-    Y.zero_()
+    Y.fill_(float("nan"))
     g.replay()
     torch.cuda.synchronize()
-    assert np.array_equal(gu.to_np(Y).view(np.uint32), gu.to_np(a).view(np.uint32))
+    assert gu.rel_fro(gu.to_np(Y), gu.to_np(a)) < REPEAT
     assert e8.e8_sync_status(gcb) == e8.E8_OK
 
 
