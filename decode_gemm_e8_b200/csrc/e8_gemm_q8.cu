@@ -47,10 +47,13 @@ constexpr int GROUPS = KU / 8;            // groups of a row in one unit
 constexpr int DEC_GROUPS = 2;
 constexpr int DEC_WARPS = 8 * DEC_GROUPS;
 constexpr int EPI_WARP0 = 2 + DEC_WARPS;
-constexpr int THREADS = 32 * (EPI_WARP0 + 4);
+constexpr int MMA2_WARP = EPI_WARP0 + 4;  // issuer of the odd units
+constexpr int THREADS = 32 * (MMA2_WARP + 1);
 constexpr int TABLE_BYTES = 131088;       // 32769 u32 entries, padded to 16 bytes
 constexpr int I1_BYTES = ROWS * GROUPS * 2;
 constexpr uint32_t ACC_COLS = 64;         // int32 accumulator columns per buffer
+// tensor memory: accumulators [issuer parity][segment buffer], then the operand ring
+constexpr uint32_t ACC_TOTAL = 4 * ACC_COLS;
 constexpr uint32_t A_COLS = KU / 4;       // 4 int8 weights per TMEM column
 constexpr int MAX_STAGES = 8;
 constexpr int AUX_BYTES = 512;            // per-token steps [32] and row sums [64]
@@ -80,7 +83,7 @@ __host__ __device__ inline SkPlan sk_plan(int rows_b, int bpw) {
   const int y_bytes = (rows_b <= 32 ? 16 : 32) * ROWS * 4;
   const int budget = kMaxDynSmem - TABLE_BYTES - 1024 - AUX_BYTES - BAR_BYTES -
                      CORESIDENT_RESERVE - y_bytes;
-  p.sa = MAX_STAGES;                                        // 2 x 64 + 8 x 32 TMEM columns
+  p.sa = MAX_STAGES;                                        // 4 x 64 + 8 x 32 TMEM columns
   // Xq tiles are requested after the transform kernel ends and take ~1 us to
   // land, so the Xq ring holds a CTA's whole run where it can (7 units of
   // 128 at 4096 x 4096); the index ring gets the rest, at least 4 stages
@@ -170,8 +173,10 @@ __device__ __forceinline__ int sk_unit_begin(int c, int U, int G) {
 
 // CW: accumulator columns read by the epilogue (32 for up to 16 tokens, else 64).
 // tmY: Y [M][N] fp32, box 128 x M (valid when use_tma_y; else fp32 atomics).
+// At most 64 registers, so that a CTA of the activation transform (512
+// threads x 32 registers) fits on the SM next to it.
 template <int BPW, int CW>
-__global__ void __launch_bounds__(sk::THREADS, 1)
+__global__ void __maxnreg__(64)
     k_gemm_q8(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmI1,
               const __grid_constant__ CUtensorMap tmI2, const __grid_constant__ CUtensorMap tmY,
               DeviceCodebook cb, int M, int N, int K, int rows_b, float alpha,
@@ -189,11 +194,11 @@ __global__ void __launch_bounds__(sk::THREADS, 1)
   uint64_t* code_empty = bars + MAX_STAGES;       // [SC] decoders hold the indices
   uint64_t* full_a = bars + 2 * MAX_STAGES;       // [SA] operand decoded + Xq landed
   uint64_t* a_empty = bars + 3 * MAX_STAGES;      // [SA] MMAs of the stage done
-  uint64_t* acc_full = bars + 4 * MAX_STAGES;     // [2]
+  uint64_t* acc_full = bars + 4 * MAX_STAGES;     // [2] both issuers done with a segment
   uint64_t* acc_empty = acc_full + 2;             // [2]
   uint64_t* table_full = acc_full + 4;
-  uint64_t* drain = acc_full + 5;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 6);
+  uint64_t* drain = acc_full + 5;                 // [2] one per issuer
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 7);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   float* s_sc = reinterpret_cast<float*>(smem + plan.aux_off);             // [32]
   int32_t* s_cs = reinterpret_cast<int32_t*>(smem + plan.aux_off + 128);   // [64]
@@ -221,11 +226,11 @@ __global__ void __launch_bounds__(sk::THREADS, 1)
       mbar_init(&a_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_full[b], 2);
       mbar_init(&acc_empty[b], 4);
+      mbar_init(&drain[b], 1);
     }
     mbar_init(table_full, 1);
-    mbar_init(drain, 1);
     fence_mbar_init();
     *abort_flag = 0u;
   }
@@ -237,7 +242,9 @@ __global__ void __launch_bounds__(sk::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const uint32_t tmem_a = tmem_base + 2 * ACC_COLS;
+  const uint32_t tmem_a = tmem_base + ACC_TOTAL;
+  const int nseg = nu > 0 ? (u_begin + nu - 1) / kunits - first_tile + 1 : 0;
+  const int ku_first = u_begin - first_tile * kunits;   // K unit of the run's first unit
   // the next kernel of the stream may be launched now: it waits for this grid
   // before it touches anything this grid reads or writes
   if (threadIdx.x == 0) grid_dep_launch();
@@ -326,58 +333,68 @@ __global__ void __launch_bounds__(sk::THREADS, 1)
         }
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == MMA2_WARP) {
     if (lane == 0) {
-      // this single thread's loop is latency-bound (each barrier test costs
-      // ~100 cycles): everything per unit is incremental, and a stage is
-      // released only when the producer will refill it
+      // Two issuers, one per decoder group: the even units accumulate into
+      // the parity-0 buffers, the odd units into the parity-1 buffers (the
+      // epilogue adds the two).  Each issuer's loop is latency-bound (a barrier
+      // test costs ~100 cycles); everything per unit is incremental, and a
+      // stage is released only when the producer or a decoder will reuse it.
+      const int par = warp == 1 ? 0 : 1;
       const uint32_t idesc = sk_idesc(ROWS, (uint32_t)rows_b);
       const uint64_t bd0 = smem_desc(smem_u32(xq_ring), 16, 1024, 2);
       const uint32_t stage16 = (uint32_t)plan.b_bytes >> 4;
-      int seg = 0;
-      int s = 0;                     // operand stage (tensor memory)
+      int s = par, sxi = par % SX;   // operand and Xq stages of the issuer's unit
       uint32_t ph = 0;
-      int sxi = 0;                   // Xq stage
-      int ku = u_begin - first_tile * kunits;
-      uint64_t bds = bd0;
-      uint32_t a0 = tmem_a;
-      for (int i = 0; i < nu; ++i) {
-        const bool first = (i == 0 || ku == 0);
-        const bool last = (i == nu - 1 || ku == kunits - 1);
-        if (first && i > 0) ++seg;
+      bool ok = true;
+      int lo = 0;                    // first local unit of the segment
+      for (int seg = 0; seg < nseg && ok; ++seg) {
+        const int len = kunits - (seg == 0 ? ku_first : 0);
+        const int hi = lo + len < nu ? lo + len : nu;
         const int b = seg & 1;
-        if (first && seg >= 2 &&
+        if (seg >= 2 &&
             !mbar_wait_sleep(&acc_empty[b], (uint32_t)((seg - 2) >> 1) & 1u, abort_flag, status,
-                             kDevTimeoutMma))
+                             kDevTimeoutMma)) {
+          ok = false;
           break;
-        if (!mbar_wait_sleep(&full_a[s], ph, abort_flag, status, kDevTimeoutFull)) break;
-        tc_fence_after();
-        const uint32_t d = tmem_base + (uint32_t)b * ACC_COLS;
+        }
+        const int i0 = lo + (((lo & 1) != par) ? 1 : 0);
+        if (i0 >= hi) {
+          // no unit of this parity in the segment
+          mbar_arrive(&acc_full[b]);
+          lo = hi;
+          continue;
+        }
+        const uint32_t d = tmem_base + (uint32_t)(par * 2 + b) * ACC_COLS;
+        for (int i = i0; i < hi; i += 2) {
+          if (!mbar_wait_sleep(&full_a[s], ph, abort_flag, status, kDevTimeoutFull)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = tmem_a + (uint32_t)s * A_COLS;
+          const uint64_t bds = bd0 + (uint64_t)((uint32_t)sxi * stage16);
 #pragma unroll
-        for (int j = 0; j < KU / 32; ++j)
-          sk_mma_i8(d, a0 + (uint32_t)(j * 8), bds + (uint64_t)(j * 2), idesc,
-                    (first && j == 0) ? 0u : 1u);
-        // the stage is reused by unit i + SX (Xq) and unit i + SA (operand)
-        if (i + SX < nu) mma_commit(&a_empty[s]);
-        if (last) mma_commit(&acc_full[b]);
-        if (++ku == kunits) ku = 0;
-        if (++s == SA) {
-          s = 0;
-          ph ^= 1u;
-          a0 = tmem_a;
-        } else {
-          a0 += A_COLS;
+          for (int j = 0; j < KU / 32; ++j)
+            sk_mma_i8(d, a0 + (uint32_t)(j * 8), bds + (uint64_t)(j * 2), idesc,
+                      (i == i0 && j == 0) ? 0u : 1u);
+          // the stage is reused by unit i + SX (Xq) and unit i + SA (operand)
+          if (i + SX < nu) mma_commit(&a_empty[s]);
+          s += 2;
+          if (s >= SA) {
+            s -= SA;
+            ph ^= 1u;
+          }
+          sxi += 2;
+          if (sxi >= SX) sxi -= SX;
         }
-        if (++sxi == SX) {
-          sxi = 0;
-          bds = bd0;
-        } else {
-          bds += stage16;
-        }
+        if (!ok) break;
+        mma_commit(&acc_full[b]);
+        lo = hi;
       }
-      mma_commit(drain);
+      mma_commit(&drain[par]);
       uint64_t t0 = global_timer_ns();
-      while (!mbar_try_wait(drain, 0))
+      while (!mbar_try_wait(&drain[par], 0))
         if (global_timer_ns() - t0 > 200000000ull) break;
     }
   } else if (warp < EPI_WARP0) {
@@ -451,12 +468,18 @@ __global__ void __launch_bounds__(sk::THREADS, 1)
       s_cs[32 + lane] = 32 + lane < rows_b ? __ldg(colsum + 32 + lane) : 0;
     }
     asm volatile("bar.sync 1, 128;" ::: "memory");
-    const int nseg = nu > 0 ? (u_begin + nu - 1) / kunits - first_tile + 1 : 0;
     // every epilogue thread runs the same sequence of named barriers, also
     // after a failed wait (it then only skips the work)
     bool ok = true;
+    int lo = 0;                      // first local unit of the segment
     for (int seg = 0; seg < nseg; ++seg) {
       const int b = seg & 1;
+      const int len = kunits - (seg == 0 ? ku_first : 0);
+      const int hi = lo + len < nu ? lo + len : nu;
+      // which issuers accumulated into the segment (units of parity 0 / 1)
+      const bool has0 = hi - lo >= 2 || (lo & 1) == 0;
+      const bool has1 = hi - lo >= 2 || (lo & 1) == 1;
+      lo = hi;
       ok = ok && mbar_wait_sleep(&acc_full[b], (uint32_t)(seg >> 1) & 1u, abort_flag, status,
                                  kDevTimeoutMma);
       tc_fence_after();
@@ -464,26 +487,30 @@ __global__ void __launch_bounds__(sk::THREADS, 1)
       const int n = tile * ROWS + r;
       // the segment holding K unit 0 of its tile removes the bias of the whole row
       const int corr = tile * kunits >= u_begin ? 128 : 0;
-      // 32 accumulator columns (16 tokens) per pass
+      const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+      const uint32_t t0a = tmem_base + (uint32_t)b * ACC_COLS + lane_off;         // parity 0
+      const uint32_t t1a = tmem_base + (uint32_t)(2 + b) * ACC_COLS + lane_off;   // parity 1
+      // 16 accumulator columns (8 tokens) per pass
 #pragma unroll
-      for (int c0 = 0; c0 < CW; c0 += 32) {
+      for (int c0 = 0; c0 < CW; c0 += 16) {
         if (!ok) break;
-        uint32_t dv[32];
-        const uint32_t ta = tmem_base + (uint32_t)b * ACC_COLS + (uint32_t)c0 +
-                            ((uint32_t)(q * 32) << 16);
-        tmem_ld16(ta, *reinterpret_cast<uint32_t(*)[16]>(dv));
-        if (c0 + 16 < rows_b) {
-          tmem_ld16(ta + 16, *reinterpret_cast<uint32_t(*)[16]>(dv + 16));
-        } else {
-#pragma unroll
-          for (int j = 16; j < 32; ++j) dv[j] = 0u;
+        uint32_t dv[16], dw[16];
+        if (c0 < rows_b) {
+          if (has0) tmem_ld16(t0a + (uint32_t)c0, dv);
+          if (has1) tmem_ld16(t1a + (uint32_t)c0, dw);
+          tmem_ld_wait();
         }
-        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const uint32_t x0 = (c0 < rows_b && has0) ? dv[j] : 0u;
+          const uint32_t x1 = (c0 < rows_b && has1) ? dw[j] : 0u;
+          dv[j] = x0 + x1;
+        }
         if (use_tma_y) {
           // tokens past M have zero steps and row sums: staged as zeros (the
           // bulk reduce covers only M rows), no branch in the loop
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
+          for (int j = 0; j < 8; ++j) {
             const int m = (c0 >> 1) + j;
             const int d0 = (int)dv[2 * j] - corr * s_cs[2 * m];
             const int d1 = (int)dv[2 * j + 1] - corr * s_cs[2 * m + 1];
@@ -491,7 +518,7 @@ __global__ void __launch_bounds__(sk::THREADS, 1)
           }
         } else if (n < N) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
+          for (int j = 0; j < 8; ++j) {
             const int m = (c0 >> 1) + j;
             const int d0 = (int)dv[2 * j] - corr * s_cs[2 * m];
             const int d1 = (int)dv[2 * j + 1] - corr * s_cs[2 * m + 1];
