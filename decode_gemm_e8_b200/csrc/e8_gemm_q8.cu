@@ -162,9 +162,6 @@ __device__ __forceinline__ void bulk_wait_read_all() {
 __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
 
 // Units [begin, end) of CTA c when U units are spread over G CTAs.
 __device__ __forceinline__ int sk_unit_begin(int c, int U, int G) {
@@ -421,6 +418,8 @@ __global__ void __maxnreg__(64)
                         __byte_perm(c.y, 0u, 0x4140), __byte_perm(c.y, 0u, 0x4342));
       }
       // the indices are in registers: the index-tile stage can be refilled
+      // once these shared-memory reads are ordered before the next bulk copy
+      fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&code_empty[cs]);
       // the operand stage must have been read by the MMAs of unit i - SA

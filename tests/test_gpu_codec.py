@@ -218,6 +218,36 @@ def test_decode_bit_exact(gcb, bpw, N, K):
     assert np.array_equal(gu.to_np(out), ref)
 
 
+@pytest.mark.parametrize("bpw", [2, 3, 4])
+@pytest.mark.parametrize("N,K", [(2, 4096), (16, 4096), (8, 3072), (4, 14336), (6, 12288),
+                                 (64, 1024), (8, 2048), (40, 6144)])
+def test_decode_bit_exact_slab_shapes(gcb, bpw, N, K):
+    # N K a multiple of 8192 and a Hadamard block of 1024..4096: the tensor-core
+    # decoder (two exact products per slab of 8192 weights)
+    assert (N * K) % 8192 == 0
+    i1, i2 = _random_codes(N, K, bpw, 7 * N + K + bpw)
+    s = 0.0211
+    out = e8.e8_decode_to_bf16(gcb, gu.to_dev(i1), None if i2 is None else gu.to_dev(i2), N, K,
+                               bpw, 1234 + N, s)
+    ref = orc.decode(i1, i2, N, K, bpw, 1234 + N, s)
+    assert np.array_equal(gu.to_np(out), ref)
+    assert e8.e8_sync_status(gcb) == e8.E8_OK
+
+
+def test_decode_extreme_codes(gcb, cb):
+    # the largest |z| (norm-12 points with a coordinate of 3, both signs, at
+    # both stages) and index 65535, on the tensor-core and the fallback paths
+    big = np.nonzero(np.abs(cb.astype(np.int64)).max(1) == 6)[0]
+    rng = np.random.default_rng(3)
+    for N, K in ((8, 4096), (3, 4096)):
+        G = N * K // 8
+        i1 = rng.choice(np.append(big, 65535), G).astype(np.uint16).reshape(N, K // 8)
+        i2 = rng.choice(np.append(big, 65535), G).astype(np.uint16).reshape(N, K // 8)
+        out = e8.e8_decode_to_bf16(gcb, gu.to_dev(i1), gu.to_dev(i2), N, K, 4, 99, 0.5)
+        ref = orc.decode(i1, i2, N, K, 4, 99, 0.5)
+        assert np.array_equal(gu.to_np(out), ref)
+
+
 @pytest.mark.parametrize("wl", ["llama_4096_b4", "mlp_up_14336_b3"])
 def test_encode_decode_full_size(gcb, wl):
     lay = synth.workloads()[wl].layers[0]
