@@ -362,8 +362,11 @@ static int decode_fast_plan(int64_t K, int* mask_off, int* bar_off, size_t* smem
 cudaError_t launch_decode(const DeviceCodebook& cb, const uint16_t* idx1, const void* idx2,
                           int64_t N, int64_t K, int bpw, uint64_t seed, float alpha,
                           uint16_t* Wdec, int sm_count, cudaStream_t st) {
-  if (decode_tc_eligible(N, K))
-    return launch_decode_tc(cb, idx1, idx2, N, K, bpw, seed, alpha, Wdec, sm_count, st);
+  {
+    const cudaError_t e =
+        launch_decode_tc(cb, idx1, idx2, N, K, bpw, seed, alpha, Wdec, sm_count, st);
+    if (e != cudaErrorNotSupported) return e;
+  }
   const int64_t nh = hadamard_block(K);
   if ((K % 128) == 0 && nh >= 256 && nh <= 4096 && K <= 32768 && N > 0) {
     DecodeFastParams f;

@@ -2,39 +2,45 @@
 // blocks of n_h = 1024, 2048 or 4096 ("glq 0.1.1", "How it works", items
 // 1-2: the inverse of the randomized Hadamard transform of the encoder).
 //
-//   z = m (c1 + beta c2)   integer 8-vector per group, |z| <= 30
+//   z = m (c1 + beta c2)   integer 8-vector per group
 //   t = FWHT_nh(z)         exact on integers
 //   w = bf16_rne(d * fl32(t * alpha))
 //
 // With n_h = 64 R and a block read as R rows of 64 (position 64 a + b), the
-// Sylvester matrix factors as H_nh = H_R (x) H_64, so t = H_R Z H_64.  Work
-// unit: a slab of 8192 consecutive weights = 128 rows of 64 (8192 / n_h whole
-// blocks).  Two products per slab, both exact:
-//   GEMM 1 (kind::i8):  U^T = diag(H_64, H_64) [Z rows r and r + 64 side by
-//     side], A = the block-diagonal H_64 pair (signed, tensor memory), B = the
-//     decoded bytes z + 128 (unsigned, shared memory, 64 rows of 128): the
-//     accumulator lane c + 64 h holds row c of U^T for slab rows 64 h .. 64 h
-//     + 63, i.e. U[r][c] = sum_b z[r][b] H_64[c][b] (plus 128 * 64 on c = 0,
-//     removed exactly); |U| <= 64 * 30 = 1920, exact in fp16.
-//   GEMM 2 (kind::f16):  T = diag(H_R, ..., H_R) [U^T rows], A = the 128/R
-//     copies of H_R on the diagonal (tensor memory), B = U^T in fp16 (shared
-//     memory, 64 rows of 128): lane d + R t holds row d of block t,
-//     T[d][c] = sum_a H_R[d][a] U_t[a][c], |T| <= 122880 < 2^24, exact in fp32.
-// So each lane of the second accumulator owns 64 consecutive weights: scaled,
-// signed, rounded and stored as 128 contiguous bytes.  The result equals the
+// natural-order Sylvester matrix factors as H_nh = H_R (x) H_8 (x) H_8:
+//   * H_8 inside each group of 8: the decoders gather from the transformed
+//     pair table, which holds H_8 v / 4, so one group decodes straight to
+//     H_8 z / 4 (integers, |.| <= 20);
+//   * H_8 across the 8 groups of a row of 64: three butterfly stages in the
+//     decoder thread that owns the row, in fp16 (exact: |U / 4| <= 160), give
+//     U / 4 with U = Z H_64 (H_64 = H_8 (x) H_8);
+//   * H_R across the R rows of a block: one tensor-core product per slab of
+//     8192 weights (128 rows of 64), kind::f16 with fp32 accumulation,
+//     T / 4 = diag(H_R, ..., H_R) (U / 4): A = the 128 / R copies of H_R on
+//     the diagonal (tensor memory), B = the slab's U / 4 as written by the
+//     decoders, row after row (shared memory, N-major); |T / 4| <= 10240,
+//     exact in fp32.
+// Lane m of the accumulator owns slab weights 64 m .. 64 m + 63, and
+// fl32((T / 4) (4 alpha)) = fl32(t alpha) exactly, so the result equals the
 // sequential definition bit for bit (the only roundings are the two of w).
+// Each warp of the readout stages its 32 x 32 bf16 piece of the slab in a
+// 64-byte-swizzled tile and writes it with one TMA store.
 //
 // Roles (one CTA per SM, persistent over slabs):
-//   warp 0      producer: bulk copies of the slab's index words (ring of 4)
-//   warp 1      tensor-memory allocation; one thread issues both GEMMs
-//   warps 2-9   decoders: pair-table gathers -> z + 128 bytes (ring of 2)
-//   warps 10-13 first readout: U^T -> fp16 operand of GEMM 2 (ring of 2)
-//   warps 14-17 second readout: T -> scale, sign, bf16, global stores
+//   warp 0      producer: table, then bulk copies of each slab's index words
+//   warp 1      tensor-memory allocation; one elected lane issues the product
+//   warps 2-9   decoders, two groups of four taking alternate slabs; thread r
+//               of a group decodes row r of the slab
+//   warps 10-17 readout: T -> scale, sign, bf16, TMA store
+// The product of slab i waits on one barrier: the decoder warps that wrote
+// its operand stage and the readout warps that emptied its accumulator
+// buffer (slab i - 3) arrive on the same one.
 #include <cuda_fp16.h>
 
 #include "e8_common.cuh"
 #include "e8_codebook.cuh"
 #include "e8_internal.h"
+#include "e8_tmap.h"
 
 namespace e8 {
 
@@ -42,33 +48,31 @@ namespace dtc {
 constexpr int SLAB = 8192;                  // weights per slab
 constexpr int GROUPS = SLAB / 8;
 constexpr int TABLE_BYTES = 131088;
-constexpr int CODE_STAGES = 4;
+constexpr int STAGES = 3;                   // index words, operand and accumulator rings
 constexpr int CODE_BYTES = GROUPS * 4;      // idx1 (2 KB) + idx2 (up to 2 KB)
-constexpr int B1_BYTES = 64 * 128;          // 64 rows x 128 bytes (u8)
-constexpr int B2_BYTES = 64 * 256;          // 64 rows x 128 fp16, two 128-byte panels
-constexpr int DEC_WARPS = 8;
-constexpr int THREADS = 32 * 18;
+constexpr int B_BYTES = 128 * 128;          // 128 rows x 64 fp16, 128-byte swizzled
+constexpr int YW_BYTES = 32 * 64;           // one readout warp's 32 x 32 bf16 tile
+constexpr int SIGN_CHUNKS = 512;            // sign words kept in shared memory (K <= 32768)
+constexpr int DEC_WARP0 = 2;
+constexpr int DEC_WARPS = 8;                // two groups of four
+constexpr int RD_WARP0 = DEC_WARP0 + DEC_WARPS;
+constexpr int RD_WARPS = 8;
+constexpr int THREADS = 32 * (RD_WARP0 + RD_WARPS);
 // tensor memory columns
-constexpr uint32_t A1_COL = 0;              // diag(H64, H64), s8: 32 columns
-constexpr uint32_t A2_COL = 32;             // diag(H_R ...), f16: 64 columns
-constexpr uint32_t D1_COL = 128;            // two buffers of 64
-constexpr uint32_t D2_COL = 256;            // two buffers of 64
+constexpr uint32_t A_COL = 0;               // diag(H_R ...), f16: 64 columns
+constexpr uint32_t D_COL = 64;              // three buffers of 64
+constexpr uint32_t TMEM_COLS = 256;
 // shared memory (after the table, from the next 1 KB boundary)
 constexpr int CODE_OFF = 0;
-constexpr int B1_OFF = CODE_OFF + CODE_STAGES * CODE_BYTES;   // 16 KB
-constexpr int B2_OFF = B1_OFF + 2 * B1_BYTES;                 // 32 KB
-constexpr int BAR_OFF = B2_OFF + 2 * B2_BYTES;                // 64 KB
+constexpr int B_OFF = CODE_OFF + STAGES * CODE_BYTES;         // 12 KB
+constexpr int Y_OFF = B_OFF + STAGES * B_BYTES;               // 60 KB
+constexpr int SIGN_OFF = Y_OFF + RD_WARPS * 2 * YW_BYTES;     // 92 KB
+constexpr int BAR_OFF = SIGN_OFF + SIGN_CHUNKS * 8;           // 96 KB
 constexpr int SMEM_TOTAL = TABLE_BYTES + 1024 + BAR_OFF + 256;
+static_assert(SMEM_TOTAL <= kMaxDynSmem, "shared memory budget");
+static_assert(B_OFF % 1024 == 0 && Y_OFF % 1024 == 0, "swizzled tiles sit on 1 KB boundaries");
 }  // namespace dtc
 
-__device__ __forceinline__ void dtc_mma_i8_ts(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc,
-                                              uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d),
-      "r"(a), "l"(b), "r"(idesc), "r"(acc)
-      : "memory");
-}
 __device__ __forceinline__ void dtc_mma_f16_ts(uint32_t d, uint32_t a, uint64_t b,
                                                uint32_t idesc, uint32_t acc) {
   asm volatile(
@@ -77,12 +81,9 @@ __device__ __forceinline__ void dtc_mma_f16_ts(uint32_t d, uint32_t a, uint64_t 
       "r"(a), "l"(b), "r"(idesc), "r"(acc)
       : "memory");
 }
-// kind::i8: A signed, B unsigned, D int32, K-major; kind::f16: A, B fp16, D fp32.
-__host__ __device__ constexpr uint32_t dtc_idesc_i8(uint32_t M, uint32_t N) {
-  return (2u << 4) | (1u << 7) | (0u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
-}
-__host__ __device__ constexpr uint32_t dtc_idesc_f16(uint32_t M, uint32_t N) {
-  return (1u << 4) | (0u << 7) | (0u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
+// kind::f16: A, B fp16, D fp32; A K-major, B N-major (bit 16).
+__host__ __device__ constexpr uint32_t dtc_idesc_f16_bn(uint32_t M, uint32_t N) {
+  return (1u << 4) | (0u << 7) | (0u << 10) | (1u << 16) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
 __device__ __forceinline__ void dtc_st32(uint32_t taddr, const uint32_t (&v)[32]) {
@@ -119,70 +120,106 @@ __device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t col) {
   return row * 128u + ((((col >> 4) ^ (row & 7u)) << 4) | (col & 15u));
 }
 
+// The 32 sign bits v of 32 consecutive weights, rearranged for pairs: bit
+// 15 - j holds v bit 2 j and bit 31 - j holds v bit 2 j + 1, so that
+// (W << j) & 0x80008000 is the sign mask of the bf16 pair j.  Even bits are
+// gathered into the low half and odd bits into the high half by four
+// delta swaps, then the word is bit-reversed and its halves exchanged.
+__device__ __forceinline__ uint32_t pair_sign_word(uint32_t v) {
+  uint32_t t;
+  t = (v ^ (v >> 1)) & 0x22222222u;
+  v ^= t ^ (t << 1);
+  t = (v ^ (v >> 2)) & 0x0C0C0C0Cu;
+  v ^= t ^ (t << 2);
+  t = (v ^ (v >> 4)) & 0x00F000F0u;
+  v ^= t ^ (t << 4);
+  t = (v ^ (v >> 8)) & 0x0000FF00u;
+  v ^= t ^ (t << 8);
+  const uint32_t b = __brev(v);
+  return (b >> 16) | (b << 16);
+}
+
 struct DecodeTcParams {
   const uint16_t* idx1;
   const void* idx2;
   int64_t slabs;          // N * K / 8192
-  int K, nh, R;           // R = nh / 64
+  int K, nh, log2R;       // R = nh / 64
   uint64_t seed;
   float alpha;
-  uint16_t* out;
-  const uint32_t* table;  // pair table (global)
+  const uint32_t* table;  // transformed pair table H_8 v / 4 (global)
   uint32_t* status;
 };
 
+// Bulk copies of one slab's index words into a stage of the ring.
 template <int BPW>
-__global__ void __launch_bounds__(dtc::THREADS, 1) k_decode_tc(DecodeTcParams p) {
+__device__ __forceinline__ void load_codes(const DecodeTcParams& p, uint8_t* dst, uint64_t* bar,
+                                           int64_t slab) {
+  constexpr uint32_t i2b = BPW == 4 ? 2048u : (BPW == 3 ? 1024u : 0u);
+  mbar_arrive_expect_tx(bar, 2048u + i2b);
+  bulk_load(dst, p.idx1 + slab * dtc::GROUPS, 2048u, bar);
+  if (BPW > 2)
+    bulk_load(dst + 2048, static_cast<const uint8_t*>(p.idx2) + slab * (int64_t)i2b, i2b, bar);
+}
+
+template <int BPW>
+__global__ void __launch_bounds__(dtc::THREADS, 1)
+    k_decode_tc(const DecodeTcParams p, const __grid_constant__ CUtensorMap tmOut) {
   using namespace dtc;
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  const uint8_t* table = smem_raw;
+  const uint8_t* table = smem_raw;   // transformed pair table: H_8 v / 4
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + TABLE_BYTES + 1023) & ~uintptr_t(1023));
   uint8_t* codes = smem + CODE_OFF;
-  uint8_t* b1 = smem + B1_OFF;
-  uint8_t* b2 = smem + B2_OFF;
+  uint8_t* bst = smem + B_OFF;
+  uint8_t* ytile = smem + Y_OFF;
+  uint32_t* sgn = reinterpret_cast<uint32_t*>(smem + SIGN_OFF);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
-  uint64_t* code_full = bars;         // [4] index words landed
-  uint64_t* code_empty = bars + 4;    // [4] decoders hold them in registers
-  uint64_t* b1_full = bars + 8;       // [2] z + 128 bytes of the slab written
-  uint64_t* b1_empty = bars + 10;     // [2] GEMM 1 done with them
-  uint64_t* d1_full = bars + 12;      // [2] U^T in tensor memory
-  uint64_t* d1_empty = bars + 14;     // [2] U^T read out
-  uint64_t* b2_full = bars + 16;      // [2] fp16 U^T written
-  uint64_t* b2_empty = bars + 18;     // [2] GEMM 2 done with it
-  uint64_t* d2_full = bars + 20;      // [2] T in tensor memory
-  uint64_t* d2_empty = bars + 22;     // [2] T read out
-  uint64_t* table_full = bars + 24;
-  uint64_t* drain = bars + 25;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 26);
+  uint64_t* code_full = bars;                 // [3] index words landed
+  uint64_t* code_empty = bars + STAGES;       // [3] decoders hold them in registers
+  uint64_t* b_full = bars + 2 * STAGES;       // [3] operand written + accumulator buffer free
+  uint64_t* b_empty = bars + 3 * STAGES;      // [3] product done with the operand
+  uint64_t* d_full = bars + 4 * STAGES;       // [3] product in tensor memory
+  uint64_t* table_full = bars + 5 * STAGES;
+  uint64_t* drain = table_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   uint32_t* status = p.status;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t nsl = (p.slabs - (int64_t)blockIdx.x + gridDim.x - 1) / gridDim.x;
+  const int chunks = p.K >> 6;
+  const bool sgn_in_smem = chunks <= SIGN_CHUNKS;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < CODE_STAGES; ++s) {
+    for (int s = 0; s < STAGES; ++s) {
       mbar_init(&code_full[s], 1);
-      mbar_init(&code_empty[s], DEC_WARPS);
-    }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&b1_full[s], DEC_WARPS);
-      mbar_init(&b1_empty[s], 1);
-      mbar_init(&d1_full[s], 1);
-      mbar_init(&d1_empty[s], 4);
-      mbar_init(&b2_full[s], 4);
-      mbar_init(&b2_empty[s], 1);
-      mbar_init(&d2_full[s], 1);
-      mbar_init(&d2_empty[s], 4);
+      mbar_init(&code_empty[s], DEC_WARPS / 2);
+      mbar_init(&b_full[s], DEC_WARPS / 2 + RD_WARPS);
+      mbar_init(&b_empty[s], 1);
+      mbar_init(&d_full[s], 1);
+      // the accumulator buffers start free
+      for (int w = 0; w < RD_WARPS; ++w) mbar_arrive(&b_full[s]);
     }
     mbar_init(table_full, 1);
     mbar_init(drain, 1);
     fence_mbar_init();
     *abort_flag = 0u;
+    // the 128 KB table and the first index words stream in while the
+    // constants are built
+    mbar_arrive_expect_tx(table_full, TABLE_BYTES);
+    for (int j = 0; j < 8; ++j) {
+      const int c = (j + (int)blockIdx.x) & 7;
+      bulk_load(smem_raw + c * 16384, reinterpret_cast<const uint8_t*>(p.table) + c * 16384,
+                16384, table_full);
+    }
+    bulk_load(smem_raw + 8 * 16384, reinterpret_cast<const uint8_t*>(p.table) + 8 * 16384, 16,
+              table_full);
+    for (int64_t i = 0; i < nsl && i < STAGES; ++i)
+      load_codes<BPW>(p, codes + i * CODE_BYTES, &code_full[i], (int64_t)blockIdx.x + i * gridDim.x);
+    tma_prefetch_desc(&tmOut);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 512);
+    tmem_alloc(tmem_slot, TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -190,42 +227,32 @@ __global__ void __launch_bounds__(dtc::THREADS, 1) k_decode_tc(DecodeTcParams p)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  // the constant operands: diag(H64, H64) as s8 and diag(H_R, ...) as fp16,
-  // one row per tensor-memory lane
-  if (warp >= 10 && warp < 14) {
+  if (warp >= RD_WARP0) {
+    // diag(H_R, ...) as fp16, one row per tensor-memory lane: columns 0-31
+    // (k = 0..63) by warps 10-13, 32-63 by warps 14-17.  H[d][a0 | b] =
+    // H[d][a0] H[d][b] for b < 2 <= lowest set bit of a0: each word is the
+    // row's first two entries, negated by H[d][a0].
     const uint32_t q = warp & 3, m = q * 32 + lane;
     const uint32_t lane_bits = (q * 32) << 16;
+    const int part = (warp - RD_WARP0) >> 2;
+    const uint32_t lr = (uint32_t)p.log2R, d = m & ((1u << lr) - 1u);
+    const uint32_t base2 = 0x3C00u | ((d & 1u) ? 0xBC000000u : 0x3C000000u);
     uint32_t v[32];
 #pragma unroll
     for (int w = 0; w < 32; ++w) {
-      uint32_t x = 0u;
-#pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        const uint32_t k = 4 * w + b;
-        const uint32_t e = (m >> 6) == (k >> 6) ? (had_neg(m & 63, k & 63) ? 0xFFu : 0x01u) : 0u;
-        x |= e << (8 * b);
-      }
-      v[w] = x;
+      const uint32_t k0 = 64u * part + 2u * w;
+      v[w] = (k0 >> lr) != (m >> lr) ? 0u : (had_neg(d, k0) ? base2 ^ 0x80008000u : base2);
     }
-    dtc_st32(tmem_base + lane_bits + A1_COL, v);
-    const uint32_t R = (uint32_t)p.R;
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-#pragma unroll
-      for (int w = 0; w < 32; ++w) {
-        uint32_t x = 0u;
-#pragma unroll
-        for (int b = 0; b < 2; ++b) {
-          const uint32_t k = 64 * half + 2 * w + b;
-          const uint32_t e =
-              m / R == k / R ? (had_neg(m % R, k % R) ? 0xBC00u : 0x3C00u) : 0u;
-          x |= e << (16 * b);
-        }
-        v[w] = x;
-      }
-      dtc_st32(tmem_base + lane_bits + A2_COL + 32 * half, v);
-    }
+    dtc_st32(tmem_base + lane_bits + A_COL + 32 * part, v);
     tmem_st_wait();
+    if (sgn_in_smem) {
+      // the sign words of every 64-column chunk of a row, in pair form
+      for (int g = threadIdx.x - 32 * RD_WARP0; g < chunks; g += 32 * RD_WARPS) {
+        const uint64_t word = splitmix64_output(p.seed, (uint64_t)g);
+        sgn[2 * g] = pair_sign_word((uint32_t)word);
+        sgn[2 * g + 1] = pair_sign_word((uint32_t)(word >> 32));
+      }
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -234,31 +261,17 @@ __global__ void __launch_bounds__(dtc::THREADS, 1) k_decode_tc(DecodeTcParams p)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      mbar_arrive_expect_tx(table_full, TABLE_BYTES);
-      for (int j = 0; j < 8; ++j) {
-        const int c = (j + (int)blockIdx.x) & 7;
-        bulk_load(smem_raw + c * 16384, reinterpret_cast<const uint8_t*>(p.table) + c * 16384,
-                  16384, table_full);
-      }
-      bulk_load(smem_raw + 8 * 16384, reinterpret_cast<const uint8_t*>(p.table) + 8 * 16384, 16,
-                table_full);
-      const uint32_t i2b = BPW == 4 ? 2048u : (BPW == 3 ? 1024u : 0u);
+      // slabs 0 .. STAGES - 1 were issued before the role split
       int s = 0;
-      uint32_t ph = 0;
-      int64_t issued = 0;
-      for (int64_t i = 0; i < nsl; ++i) {
-        if (i >= CODE_STAGES &&
-            !mbar_wait_sleep(&code_empty[s], ph ^ 1u, abort_flag, status, kDevTimeoutEmpty))
+      uint32_t ph = 1;
+      int64_t issued = nsl < STAGES ? nsl : STAGES;
+      for (int64_t i = STAGES; i < nsl; ++i) {
+        if (!mbar_wait_sleep(&code_empty[s], ph ^ 1u, abort_flag, status, kDevTimeoutEmpty))
           break;
-        const int64_t slab = (int64_t)blockIdx.x + i * gridDim.x;
-        uint8_t* dst = codes + s * CODE_BYTES;
-        mbar_arrive_expect_tx(&code_full[s], 2048u + i2b);
-        bulk_load(dst, p.idx1 + slab * GROUPS, 2048u, &code_full[s]);
-        if (BPW > 2)
-          bulk_load(dst + 2048, static_cast<const uint8_t*>(p.idx2) + slab * (int64_t)i2b, i2b,
-                    &code_full[s]);
+        load_codes<BPW>(p, codes + s * CODE_BYTES, &code_full[s],
+                        (int64_t)blockIdx.x + i * gridDim.x);
         ++issued;
-        if (++s == CODE_STAGES) {
+        if (++s == STAGES) {
           s = 0;
           ph ^= 1u;
         }
@@ -268,205 +281,206 @@ __global__ void __launch_bounds__(dtc::THREADS, 1) k_decode_tc(DecodeTcParams p)
         uint64_t t0 = global_timer_ns();
         while (!mbar_try_wait(table_full, 0))
           if (global_timer_ns() - t0 > 100000000ull) break;
-        for (int64_t j = issued > CODE_STAGES ? issued - CODE_STAGES : 0; j < issued; ++j) {
+        for (int64_t j = issued > STAGES ? issued - STAGES : 0; j < issued; ++j) {
           t0 = global_timer_ns();
-          while (!mbar_try_wait(&code_full[j % CODE_STAGES], (uint32_t)(j / CODE_STAGES) & 1u))
+          while (!mbar_try_wait(&code_full[j % STAGES], (uint32_t)(j / STAGES) & 1u))
             if (global_timer_ns() - t0 > 100000000ull) break;
         }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc1 = dtc_idesc_i8(128, 64);
-      const uint32_t idesc2 = dtc_idesc_f16(128, 64);
-      const uint64_t bd1 = smem_desc(smem_u32(b1), 16, 1024, 2);
-      const uint64_t bd2 = smem_desc(smem_u32(b2), 16, 1024, 2);
-      bool ok = true;
-      for (int64_t i = 0; i <= nsl && ok; ++i) {
-        if (i < nsl) {
-          // GEMM 1 of slab i
-          const int s = (int)(i & 1);
-          const uint32_t ph = (uint32_t)(i >> 1) & 1u;
-          if (!mbar_wait_sleep(&b1_full[s], ph, abort_flag, status, kDevTimeoutFull) ||
-              (i >= 2 &&
-               !mbar_wait_sleep(&d1_empty[s], ph ^ 1u, abort_flag, status, kDevTimeoutMma))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t d = tmem_base + D1_COL + 64u * (uint32_t)s;
-          const uint64_t bd = bd1 + (uint64_t)((uint32_t)(s * B1_BYTES) >> 4);
+    // The whole warp runs the loop (warp-uniform operands); one elected lane
+    // issues.  K = 128 slab rows: eight steps of 16 rows = 2 KB of the
+    // operand stage each.
+    const uint32_t idesc = dtc_idesc_f16_bn(128, 64);
+    const uint64_t bd0 = smem_desc(smem_u32(bst), 16, 1024, 2);
+    int s = 0;
+    uint32_t ph = 0;
+    for (int64_t i = 0; i < nsl; ++i) {
+      if (!warp_wait(&b_full[s], ph, abort_flag, status, kDevTimeoutFull)) break;
+      tc_fence_after();
+      const uint32_t d = tmem_base + D_COL + 64u * (uint32_t)s;
+      const uint64_t bd = bd0 + (uint64_t)(((uint32_t)s * B_BYTES) >> 4);
+      if (elect_one()) {
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            dtc_mma_i8_ts(d, tmem_base + A1_COL + 8u * j, bd + (uint64_t)(2 * j), idesc1,
-                          j > 0 ? 1u : 0u);
-          mma_commit(&b1_empty[s]);
-          mma_commit(&d1_full[s]);
-        }
-        if (i >= 1) {
-          // GEMM 2 of slab i - 1
-          const int64_t k = i - 1;
-          const int s = (int)(k & 1);
-          const uint32_t ph = (uint32_t)(k >> 1) & 1u;
-          if (!mbar_wait_sleep(&b2_full[s], ph, abort_flag, status, kDevTimeoutFull) ||
-              (k >= 2 &&
-               !mbar_wait_sleep(&d2_empty[s], ph ^ 1u, abort_flag, status, kDevTimeoutMma))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t d = tmem_base + D2_COL + 64u * (uint32_t)s;
-          const uint64_t bd = bd2 + (uint64_t)((uint32_t)(s * B2_BYTES) >> 4);
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            dtc_mma_f16_ts(d, tmem_base + A2_COL + 8u * j,
-                           bd + (uint64_t)((j >> 2) * (8192 >> 4) + (j & 3) * 2), idesc2,
-                           j > 0 ? 1u : 0u);
-          mma_commit(&b2_empty[s]);
-          mma_commit(&d2_full[s]);
-        }
+        for (int j = 0; j < 8; ++j)
+          dtc_mma_f16_ts(d, tmem_base + A_COL + 8u * j, bd + (uint64_t)(j * (2048 >> 4)), idesc,
+                         j > 0 ? 1u : 0u);
+        mma_commit(&b_empty[s]);
+        mma_commit(&d_full[s]);
       }
-      mma_commit(drain);
-      uint64_t t0 = global_timer_ns();
-      while (!mbar_try_wait(drain, 0))
-        if (global_timer_ns() - t0 > 200000000ull) break;
+      __syncwarp();
+      if (++s == STAGES) {
+        s = 0;
+        ph ^= 1u;
+      }
     }
-  } else if (warp < 2 + DEC_WARPS) {
+    if (elect_one()) {
+      mma_commit(drain);
+      const uint64_t t1 = global_timer_ns();
+      while (!mbar_try_wait(drain, 0))
+        if (global_timer_ns() - t1 > 200000000ull) break;
+    }
+    __syncwarp();
+  } else if (warp < RD_WARP0) {
     // ------------------------------------------------------------ decoders
-    const int t = threadIdx.x - 64;     // 0 .. 255: groups 4t .. 4t + 3 of the slab
-    const uint32_t r = (uint32_t)t >> 1;               // slab row (64 weights)
-    const uint32_t rb = r & 63u, hcol = (r >> 6) * 64u;
-    bool ok = mbar_wait_sleep(table_full, 0, abort_flag, status, kDevTimeoutFull);
-    int cs = 0;
-    uint32_t cph = 0;
-    for (int64_t i = 0; i < nsl && ok; ++i) {
-      if (!mbar_wait_sleep(&code_full[cs], cph, abort_flag, status, kDevTimeoutFull)) break;
-      const uint8_t* cw = codes + cs * CODE_BYTES;
-      const uint2 w1 = *reinterpret_cast<const uint2*>(cw + 8 * t);
-      uint2 w2 = make_uint2(0u, 0u);
+    // group `grp` takes slabs grp, grp + 2, ...; thread r decodes slab row r
+    // (groups 8 r .. 8 r + 7) and finishes its 64-point transform
+    const int grp = (warp - DEC_WARP0) >> 2;
+    const uint32_t r = (uint32_t)(threadIdx.x - 32 * DEC_WARP0) & 127u;
+    const __half2 bias2 = __half2half2(__ushort_as_half((unsigned short)0x6880u));   // 2304
+    bool ok = warp_wait(table_full, 0, abort_flag, status, kDevTimeoutFull);
+    for (int64_t i = grp; i < nsl && ok; i += 2) {
+      const int s = (int)(i % STAGES);
+      const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
+      if (!warp_wait(&code_full[s], ph, abort_flag, status, kDevTimeoutFull)) break;
+      const uint8_t* cw = codes + s * CODE_BYTES;
+      const uint4 c1 = *reinterpret_cast<const uint4*>(cw + 16 * r);
+      uint4 c2 = make_uint4(0u, 0u, 0u, 0u);
       if (BPW == 4) {
-        w2 = *reinterpret_cast<const uint2*>(cw + 2048 + 8 * t);
+        c2 = *reinterpret_cast<const uint4*>(cw + 2048 + 16 * r);
       } else if (BPW == 3) {
-        const uint32_t c = *reinterpret_cast<const uint32_t*>(cw + 2048 + 4 * t);
-        w2 = make_uint2(__byte_perm(c, 0u, 0x4140), __byte_perm(c, 0u, 0x4342));
+        const uint2 c = *reinterpret_cast<const uint2*>(cw + 2048 + 8 * r);
+        c2 = make_uint4(__byte_perm(c.x, 0u, 0x4140), __byte_perm(c.x, 0u, 0x4342),
+                        __byte_perm(c.y, 0u, 0x4140), __byte_perm(c.y, 0u, 0x4342));
       }
       // the index words are in registers; order these shared-memory reads
       // before the producer's next bulk-copy write into the stage
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&code_empty[cs]);
-      const int s = (int)(i & 1);
-      if (i >= 2) {
-        if (!mbar_wait_sleep(&b1_empty[s], ((uint32_t)(i >> 1) & 1u) ^ 1u, abort_flag, status,
-                             kDevTimeoutMma))
-          break;
-        // the tensor cores' reads of the stage (async proxy) before these writes
-        fence_proxy_async_smem();
-      }
-      uint8_t* bt = b1 + s * B1_BYTES;
-      const uint32_t ww1[2] = {w1.x, w1.y}, ww2[2] = {w2.x, w2.y};
+      if (lane == 0) mbar_arrive(&code_empty[s]);
+      // decode: group g -> four fp16 pairs 1024 + (H_8 z / 4 + 128), in
+      // coordinate order
+      __half2 x[8][4];
+      const uint32_t w1[4] = {c1.x, c1.y, c1.z, c1.w}, w2[4] = {c2.x, c2.y, c2.z, c2.w};
 #pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const uint32_t ea0 = *reinterpret_cast<const uint32_t*>(table + ((((ww1[k] & 0xFFFFu) << 1) + 2u) & 0x3FFFCu));
-        const uint32_t ea1 = *reinterpret_cast<const uint32_t*>(table + (((ww1[k] >> 15) + 2u) & 0x3FFFCu));
-        const uint32_t eb0 = BPW > 2 ? *reinterpret_cast<const uint32_t*>(table + ((((ww2[k] & 0xFFFFu) << 1) + 2u) & 0x3FFFCu)) : 0u;
-        const uint32_t eb1 = BPW > 2 ? *reinterpret_cast<const uint32_t*>(table + (((ww2[k] >> 15) + 2u) & 0x3FFFCu)) : 0u;
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t ea0 = *reinterpret_cast<const uint32_t*>(table + ((((w1[k] & 0xFFFFu) << 1) + 2u) & 0x3FFFCu));
+        const uint32_t ea1 = *reinterpret_cast<const uint32_t*>(table + (((w1[k] >> 15) + 2u) & 0x3FFFCu));
+        const uint32_t eb0 = BPW > 2 ? *reinterpret_cast<const uint32_t*>(table + ((((w2[k] & 0xFFFFu) << 1) + 2u) & 0x3FFFCu)) : 0u;
+        const uint32_t eb1 = BPW > 2 ? *reinterpret_cast<const uint32_t*>(table + (((w2[k] >> 15) + 2u) & 0x3FFFCu)) : 0u;
         uint32_t lo0, hi0, lo1, hi1;
-        decode_group_q8<BPW>(ww1[k] & 0xFFFFu, ww2[k] & 0xFFFFu, ea0, eb0, lo0, hi0);
-        decode_group_q8<BPW>(ww1[k] >> 16, ww2[k] >> 16, ea1, eb1, lo1, hi1);
-        // groups 4t + 2k and 4t + 2k + 1: bytes 8 ((t & 1) * 4 + 2k) .. of row r
-        const uint32_t col = hcol + 8u * (((uint32_t)t & 1u) * 4u + 2u * k);
-        *reinterpret_cast<uint2*>(bt + sw128(rb, col)) = make_uint2(lo0, hi0);
-        *reinterpret_cast<uint2*>(bt + sw128(rb, col + 8u)) = make_uint2(lo1, hi1);
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&b1_full[s]);
-      if (++cs == CODE_STAGES) {
-        cs = 0;
-        cph ^= 1u;
-      }
-    }
-  } else if (warp < 14) {
-    // ------------------------------------------------------------ readout 1
-    const uint32_t q = warp & 3, m = q * 32 + lane;
-    const uint32_t c = m & 63u, h = m >> 6;
-    const uint32_t lane_bits = (q * 32) << 16;
-    const int bias = c == 0 ? 128 * 64 : 0;
-    for (int64_t i = 0; i < nsl; ++i) {
-      const int s = (int)(i & 1);
-      const uint32_t ph = (uint32_t)(i >> 1) & 1u;
-      if (!mbar_wait_sleep(&d1_full[s], ph, abort_flag, status, kDevTimeoutMma)) break;
-      if (i >= 2) {
-        if (!mbar_wait_sleep(&b2_empty[s], ph ^ 1u, abort_flag, status, kDevTimeoutMma)) break;
-        fence_proxy_async_smem();
-      }
-      tc_fence_after();
-      uint32_t u[32], u2[32];
-      dtc_ld32(tmem_base + lane_bits + D1_COL + 64u * (uint32_t)s, u);
-      dtc_ld32(tmem_base + lane_bits + D1_COL + 64u * (uint32_t)s + 32u, u2);
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&d1_empty[s]);
-      // row c of panel h of the fp16 operand: 64 values, 128 bytes
-      uint8_t* row = b2 + s * B2_BYTES + h * 8192u;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        uint32_t pk[4];
+        decode_group_q8<BPW>(w1[k] & 0xFFFFu, w2[k] & 0xFFFFu, ea0, eb0, lo0, hi0);
+        decode_group_q8<BPW>(w1[k] >> 16, w2[k] >> 16, ea1, eb1, lo1, hi1);
+        const uint32_t wd[4] = {lo0, hi0, lo1, hi1};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int x = 8 * j + 2 * e;
-          const int a = (int)(x < 32 ? u[x] : u2[x - 32]) - bias;
-          const int b = (int)(x + 1 < 32 ? u[x + 1] : u2[x - 31]) - bias;
-          __half2 hv = __floats2half2_rn((float)a, (float)b);
-          pk[e] = *reinterpret_cast<uint32_t*>(&hv);
+          const uint32_t a = __byte_perm(wd[e], 0x64646464u, 0x4140);
+          const uint32_t b = __byte_perm(wd[e], 0x64646464u, 0x4342);
+          x[2 * k + (e >> 1)][2 * (e & 1)] = *reinterpret_cast<const __half2*>(&a);
+          x[2 * k + (e >> 1)][2 * (e & 1) + 1] = *reinterpret_cast<const __half2*>(&b);
         }
-        *reinterpret_cast<uint4*>(row + sw128(c, 16u * j)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      // H_8 across the groups, natural order, exact in fp16.  First stage
+      // with the bias 2 x 1152 removed: (A + (B - 2304)) and (A - B), both
+      // intermediates integers below 2048 in magnitude.
+#pragma unroll
+      for (int g = 0; g < 8; g += 2)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const __half2 a = x[g][e], b = x[g + 1][e];
+          x[g][e] = __hadd2(a, __hsub2(b, bias2));
+          x[g + 1][e] = __hsub2(a, b);
+        }
+#pragma unroll
+      for (int h = 2; h < 8; h <<= 1)
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          if (g & h) continue;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const __half2 a = x[g][e], b = x[g + h][e];
+            x[g][e] = __hadd2(a, b);
+            x[g + h][e] = __hsub2(a, b);
+          }
+        }
+      // the product of slab i - 3 has read this operand stage
+      if (i >= STAGES && !warp_wait(&b_empty[s], ph ^ 1u, abort_flag, status, kDevTimeoutMma))
+        break;
+      // row r of the N-major operand: U[r][8 g' + k'] for g' = 0..7, one
+      // 16-byte chunk per g', 128-byte swizzled
+      uint8_t* brow = bst + s * B_BYTES + r * 128u;
+#pragma unroll
+      for (int g = 0; g < 8; ++g) {
+        uint4 v;
+        v.x = *reinterpret_cast<const uint32_t*>(&x[g][0]);
+        v.y = *reinterpret_cast<const uint32_t*>(&x[g][1]);
+        v.z = *reinterpret_cast<const uint32_t*>(&x[g][2]);
+        v.w = *reinterpret_cast<const uint32_t*>(&x[g][3]);
+        *reinterpret_cast<uint4*>(brow + (((uint32_t)g ^ (r & 7u)) << 4)) = v;
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&b2_full[s]);
+      if (lane == 0) mbar_arrive(&b_full[s]);
     }
   } else {
-    // ------------------------------------------------------------ readout 2
-    const uint32_t q = warp & 3, m = q * 32 + lane;
+    // ------------------------------------------------------------ readout
+    // lane m of the accumulator, columns 32 hh .. 32 hh + 31: slab weights
+    // 64 m + 32 hh .., staged as row `lane` of this warp's 32 x 32 tile
+    // (64-byte swizzled: chunk j of row l at ((j ^ ((l >> 1) & 3)) << 4))
+    const uint32_t q = warp & 3, wi = (uint32_t)(warp - RD_WARP0), hh = wi >> 2;
+    const uint32_t m = q * 32 + lane;
     const uint32_t lane_bits = (q * 32) << 16;
-    const int R = p.R;
-    const int tb = (int)m / R, d = (int)m % R;
+    const uint32_t K = (uint32_t)p.K;
+    const float alpha4 = 4.0f * p.alpha;
+    // column of the slab's first weight, advanced by grid * 8192 mod K
+    const uint32_t step = (uint32_t)(((uint64_t)gridDim.x * SLAB) % K);
+    uint32_t base = (uint32_t)(((uint64_t)blockIdx.x * SLAB) % K);
+    const uint32_t offm = (64u * m) % K;
+    uint8_t* ybuf = ytile + wi * 2u * YW_BYTES;
+    uint32_t yoff[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) yoff[j] = lane * 64u + ((j ^ ((lane >> 1) & 3u)) << 4);
+    int s = 0;
+    uint32_t ph = 0;
     for (int64_t i = 0; i < nsl; ++i) {
-      const int s = (int)(i & 1);
-      const uint32_t ph = (uint32_t)(i >> 1) & 1u;
-      if (!mbar_wait_sleep(&d2_full[s], ph, abort_flag, status, kDevTimeoutMma)) break;
+      if (!warp_wait(&d_full[s], ph, abort_flag, status, kDevTimeoutMma)) break;
       tc_fence_after();
-      uint32_t y[32], y2[32];
-      dtc_ld32(tmem_base + lane_bits + D2_COL + 64u * (uint32_t)s, y);
-      dtc_ld32(tmem_base + lane_bits + D2_COL + 64u * (uint32_t)s + 32u, y2);
+      uint32_t y[32];
+      dtc_ld32(tmem_base + lane_bits + D_COL + 64u * (uint32_t)s + 32u * hh, y);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&d2_empty[s]);
-      const int64_t slab = (int64_t)blockIdx.x + i * gridDim.x;
-      const int64_t e0 = slab * SLAB + (int64_t)tb * p.nh + 64 * d;
-      const int64_t col = e0 % p.K;
-      const uint64_t word = splitmix64_output(p.seed, (uint64_t)(col >> 6));
-      uint4* dst = reinterpret_cast<uint4*>(p.out + e0);
+      if (lane == 0) mbar_arrive(&b_full[s]);   // accumulator buffer free for slab i + 3
+      uint32_t pos = base + offm;
+      if (pos >= K) pos -= K;
+      uint32_t W;
+      if (sgn_in_smem) {
+        W = sgn[2 * (pos >> 6) + hh];
+      } else {
+        const uint64_t word = splitmix64_output(p.seed, (uint64_t)(pos >> 6));
+        W = pair_sign_word((uint32_t)(word >> (32 * hh)));
+      }
+      uint32_t pk[16];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        uint32_t pk[4];
+      for (int e = 0; e < 16; ++e) {
+        const float a = __fmul_rn(__uint_as_float(y[2 * e]), alpha4);
+        const float b = __fmul_rn(__uint_as_float(y[2 * e + 1]), alpha4);
+        pk[e] = pack_bf16x2(a, b) ^ ((W << e) & 0x80008000u);
+      }
+      // the store of slab i - 2 has read this stage
+      uint8_t* yt = ybuf + (uint32_t)(i & 1) * YW_BYTES;
+      if (i >= 2 && lane == 0) bulk_wait_read_1();
+      __syncwarp();
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int x = 8 * j + 2 * e;
-          float a = __fmul_rn(__uint_as_float(x < 32 ? y[x] : y2[x - 32]), p.alpha);
-          float b = __fmul_rn(__uint_as_float(x + 1 < 32 ? y[x + 1] : y2[x - 31]), p.alpha);
-          a = __uint_as_float(__float_as_uint(a) ^ ((uint32_t)(word >> x) & 1u) << 31);
-          b = __uint_as_float(__float_as_uint(b) ^ ((uint32_t)(word >> (x + 1)) & 1u) << 31);
-          pk[e] = pack_bf16x2(a, b);
-        }
-        dst[j] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      for (int j = 0; j < 4; ++j)
+        *reinterpret_cast<uint4*>(yt + yoff[j]) =
+            make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        const int64_t slab = (int64_t)blockIdx.x + i * gridDim.x;
+        tma_store_2d(&tmOut, smem_u32(yt), (int32_t)(32 * hh), (int32_t)(slab * 128 + 32 * q));
+      }
+      base += step;
+      if (base >= K) base -= K;
+      if (++s == STAGES) {
+        s = 0;
+        ph ^= 1u;
       }
     }
+    if (lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -474,45 +488,55 @@ __global__ void __launch_bounds__(dtc::THREADS, 1) k_decode_tc(DecodeTcParams p)
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, 512);
+    tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 
 template <int BPW>
-static cudaError_t launch_decode_tc_t(const DecodeTcParams& p, int grid, cudaStream_t st) {
+static cudaError_t launch_decode_tc_t(const DecodeTcParams& p, const CUtensorMap& tm, int grid,
+                                      cudaStream_t st) {
   cudaError_t e = ensure_smem_limit(k_decode_tc<BPW>, kMaxDynSmem);
   if (e != cudaSuccess) return e;
-  k_decode_tc<BPW><<<grid, dtc::THREADS, dtc::SMEM_TOTAL, st>>>(p);
+  k_decode_tc<BPW><<<grid, dtc::THREADS, dtc::SMEM_TOTAL, st>>>(p, tm);
   return cudaGetLastError();
 }
 
-// Shapes served: n_h in {1024, 2048, 4096} and N K a multiple of 8192.
-bool decode_tc_eligible(int64_t N, int64_t K) {
+// Shapes served: n_h in {1024, 2048, 4096}, N K a multiple of 8192 with
+// N K / 64 rows addressable by the store, 16-byte aligned buffers.
+bool decode_tc_eligible(int64_t N, int64_t K, const void* idx1, const void* idx2,
+                        const void* out) {
   const int64_t nh = hadamard_block(K);
+  auto al = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
   return N > 0 && (nh == 1024 || nh == 2048 || nh == 4096) && ((N * K) % dtc::SLAB) == 0 &&
-         K <= (int64_t)1 << 30;
+         K <= ((int64_t)1 << 30) && N * K / 64 < ((int64_t)1 << 31) && al(idx1) &&
+         (idx2 == nullptr || al(idx2)) && al(out);
 }
 
 cudaError_t launch_decode_tc(const DeviceCodebook& cb, const uint16_t* idx1, const void* idx2,
                              int64_t N, int64_t K, int bpw, uint64_t seed, float alpha,
                              uint16_t* Wdec, int sm_count, cudaStream_t st) {
-  if (!decode_tc_eligible(N, K)) return cudaErrorInvalidValue;
+  if (!decode_tc_eligible(N, K, idx1, bpw > 2 ? idx2 : nullptr, Wdec))
+    return cudaErrorNotSupported;
+  CUtensorMap tm;
+  if (!make_tmap_2d(&tm, Wdec, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)(N * K / 64), 64,
+                    32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+    return cudaErrorNotSupported;
   DecodeTcParams p;
   p.idx1 = idx1;
   p.idx2 = idx2;
   p.slabs = N * K / dtc::SLAB;
   p.K = (int)K;
   p.nh = (int)hadamard_block(K);
-  p.R = p.nh / 64;
+  p.log2R = 0;
+  while ((64 << p.log2R) < p.nh) ++p.log2R;
   p.seed = seed;
   p.alpha = alpha;
-  p.out = Wdec;
-  p.table = cb.table;
+  p.table = cb.h8table;
   p.status = cb.status;
   const int grid = (int)(p.slabs < sm_count ? p.slabs : sm_count);
-  if (bpw == 2) return launch_decode_tc_t<2>(p, grid, st);
-  if (bpw == 3) return launch_decode_tc_t<3>(p, grid, st);
-  return launch_decode_tc_t<4>(p, grid, st);
+  if (bpw == 2) return launch_decode_tc_t<2>(p, tm, grid, st);
+  if (bpw == 3) return launch_decode_tc_t<3>(p, tm, grid, st);
+  return launch_decode_tc_t<4>(p, tm, grid, st);
 }
 
 }  // namespace e8

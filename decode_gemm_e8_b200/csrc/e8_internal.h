@@ -60,9 +60,12 @@ cudaError_t launch_encode_leader(const DeviceCodebook& cb, const WorkItem* in,
 cudaError_t launch_decode(const DeviceCodebook& cb, const uint16_t* idx1, const void* idx2,
                           int64_t N, int64_t K, int bpw, uint64_t seed, float alpha,
                           uint16_t* Wdec, int sm_count, cudaStream_t st);
-// Tensor-core decoder (n_h = 1024, 2048, 4096; N K a multiple of 8192); same
-// contract and bit-identical result as launch_decode.
-bool decode_tc_eligible(int64_t N, int64_t K);
+// Tensor-core decoder (n_h = 1024, 2048, 4096; N K a multiple of 8192;
+// 16-byte aligned buffers); same contract and bit-identical result as
+// launch_decode.  Returns cudaErrorNotSupported, launching nothing, for other
+// shapes.
+bool decode_tc_eligible(int64_t N, int64_t K, const void* idx1, const void* idx2,
+                        const void* out);
 cudaError_t launch_decode_tc(const DeviceCodebook& cb, const uint16_t* idx1, const void* idx2,
                              int64_t N, int64_t K, int bpw, uint64_t seed, float alpha,
                              uint16_t* Wdec, int sm_count, cudaStream_t st);
