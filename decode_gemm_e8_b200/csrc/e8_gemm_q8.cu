@@ -24,8 +24,9 @@
 //               (a ring released by the decoders as soon as they hold the
 //               indices in registers; filled before waiting for the transform
 //               kernel) and the Xq tiles (a ring released by the MMA)
-//   warp 1      tensor-memory allocation; one thread issues tcgen05.mma
-//               (M = 128 weight rows, N = rows_b, K = 32) and the commits
+//   warps 1, 22 tensor-memory allocation (warp 1); one elected lane of each
+//               issues tcgen05.mma (M = 128 weight rows, N = rows_b, K = 32)
+//               and the commits for the even / odd units
 //   warps 2-17  decoders, two groups of eight taking alternate units: each
 //               thread owns one weight row (its TMEM lane) and 8 of the 16
 //               groups of a unit: index loads, pair-table gathers, combine,
@@ -325,69 +326,75 @@ __global__ void __maxnreg__(64)
       }
     }
   } else if (warp == 1 || warp == MMA2_WARP) {
-    if (lane == 0) {
-      // Two issuers, one per decoder group: the even units accumulate into
-      // the parity-0 buffers, the odd units into the parity-1 buffers (the
-      // epilogue adds the two).  Each issuer's loop is latency-bound (a barrier
-      // test costs ~100 cycles); everything per unit is incremental, and a
-      // stage is released only when the producer or a decoder will reuse it.
-      const int par = warp == 1 ? 0 : 1;
-      const uint32_t idesc = sk_idesc(ROWS, (uint32_t)rows_b);
-      const uint64_t bd0 = smem_desc(smem_u32(xq_ring), 16, 1024, 2);
-      const uint32_t stage16 = (uint32_t)plan.b_bytes >> 4;
-      int s = par, sxi = par % SX;   // operand and Xq stages of the issuer's unit
-      uint32_t ph = 0;
-      bool ok = true;
-      int lo = 0;                    // first local unit of the segment
-      for (int seg = 0; seg < nseg && ok; ++seg) {
-        const int len = kunits - (seg == 0 ? ku_first : 0);
-        const int hi = lo + len < nu ? lo + len : nu;
-        const int b = seg & 1;
-        if (seg >= 2 &&
-            !mbar_wait_sleep(&acc_empty[b], (uint32_t)((seg - 2) >> 1) & 1u, abort_flag, status,
-                             kDevTimeoutMma)) {
+    // Two issuers, one per decoder group: the even units accumulate into the
+    // parity-0 buffers, the odd units into the parity-1 buffers (the epilogue
+    // adds the two).  The whole warp runs the loop (warp-uniform operands);
+    // the elected lane issues the MMAs and the commits, so that every commit
+    // tracks all MMAs before it.  A stage is released only when the producer
+    // or a decoder will reuse it.
+    const int par = warp == 1 ? 0 : 1;
+    const uint32_t idesc = sk_idesc(ROWS, (uint32_t)rows_b);
+    const uint64_t bd0 = smem_desc(smem_u32(xq_ring), 16, 1024, 2);
+    const uint32_t stage16 = (uint32_t)plan.b_bytes >> 4;
+    int s = par, sxi = par % SX;   // operand and Xq stages of the issuer's unit
+    uint32_t ph = 0;
+    bool ok = true;
+    int lo = 0;                    // first local unit of the segment
+    for (int seg = 0; seg < nseg && ok; ++seg) {
+      const int len = kunits - (seg == 0 ? ku_first : 0);
+      const int hi = lo + len < nu ? lo + len : nu;
+      const int b = seg & 1;
+      if (seg >= 2 && !warp_wait(&acc_empty[b], (uint32_t)((seg - 2) >> 1) & 1u, abort_flag,
+                                 status, kDevTimeoutMma)) {
+        ok = false;
+        break;
+      }
+      const int i0 = lo + (((lo & 1) != par) ? 1 : 0);
+      if (i0 >= hi) {
+        // no unit of this parity in the segment
+        if (elect_one()) mbar_arrive(&acc_full[b]);
+        __syncwarp();
+        lo = hi;
+        continue;
+      }
+      const uint32_t d = tmem_base + (uint32_t)(par * 2 + b) * ACC_COLS;
+      for (int i = i0; i < hi; i += 2) {
+        if (!warp_wait(&full_a[s], ph, abort_flag, status, kDevTimeoutFull)) {
           ok = false;
           break;
         }
-        const int i0 = lo + (((lo & 1) != par) ? 1 : 0);
-        if (i0 >= hi) {
-          // no unit of this parity in the segment
-          mbar_arrive(&acc_full[b]);
-          lo = hi;
-          continue;
-        }
-        const uint32_t d = tmem_base + (uint32_t)(par * 2 + b) * ACC_COLS;
-        for (int i = i0; i < hi; i += 2) {
-          if (!mbar_wait_sleep(&full_a[s], ph, abort_flag, status, kDevTimeoutFull)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t a0 = tmem_a + (uint32_t)s * A_COLS;
-          const uint64_t bds = bd0 + (uint64_t)((uint32_t)sxi * stage16);
+        tc_fence_after();
+        const uint32_t a0 = tmem_a + (uint32_t)s * A_COLS;
+        const uint64_t bds = bd0 + (uint64_t)((uint32_t)sxi * stage16);
+        if (elect_one()) {
 #pragma unroll
           for (int j = 0; j < KU / 32; ++j)
             sk_mma_i8(d, a0 + (uint32_t)(j * 8), bds + (uint64_t)(j * 2), idesc,
                       (i == i0 && j == 0) ? 0u : 1u);
           // the stage is reused by unit i + SX (Xq) and unit i + SA (operand)
           if (i + SX < nu) mma_commit(&a_empty[s]);
-          s += 2;
-          if (s >= SA) {
-            s -= SA;
-            ph ^= 1u;
-          }
-          sxi += 2;
-          if (sxi >= SX) sxi -= SX;
         }
-        if (!ok) break;
-        mma_commit(&acc_full[b]);
-        lo = hi;
+        __syncwarp();
+        s += 2;
+        if (s >= SA) {
+          s -= SA;
+          ph ^= 1u;
+        }
+        sxi += 2;
+        if (sxi >= SX) sxi -= SX;
       }
+      if (!ok) break;
+      if (elect_one()) mma_commit(&acc_full[b]);
+      __syncwarp();
+      lo = hi;
+    }
+    if (elect_one()) {
       mma_commit(&drain[par]);
-      uint64_t t0 = global_timer_ns();
+      const uint64_t t0 = global_timer_ns();
       while (!mbar_try_wait(&drain[par], 0))
         if (global_timer_ns() - t0 > 200000000ull) break;
     }
+    __syncwarp();
   } else if (warp < EPI_WARP0) {
     // ------------------------------------------------------------ decoders
     const int dw = warp - 2;
