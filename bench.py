@@ -195,6 +195,9 @@ def run_ours(args):
     build.build()
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
+    if args.profile == "decode":
+        _profile_decode(e8, dev)
+        return
     peaks = _peaks()
     lay = synth.workloads()[WORKLOAD].layers[0]
     N, K, bpw = lay.N, lay.K, lay.bpw
@@ -374,6 +377,25 @@ def _traffic_from_profile():
     if not m_h or not m_t or m_h.group(1) != h:
         return None
     return int(m_t.group(1))
+
+
+def _profile_decode(e8, dev):
+    """Three bf16 decodes of a 14336 x 4096 matrix at 4 bpw (about 150 MB on the
+    device, more than L2), for ncu captures of the tensor-core decoder."""
+    import torch
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(11)
+    N, K, bpw = 14336, 4096, 4
+    c1, c2 = _random_codes(torch, dev, N, K, bpw, gen)
+    cb = e8.Codebook(dev.index)
+    out = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+    for _ in range(3):
+        e8.e8_decode_to_bf16(cb, c1, c2, N, K, bpw, 7, 0.02, out=out)
+    torch.cuda.synchronize()
+    if e8.e8_sync_status(cb) != 0:
+        raise RuntimeError("decoder reported a device error")
+    print("profile decodes done", flush=True)
+    cb.free()
 
 
 def _random_codes(torch, dev, N, K, bpw, gen):
@@ -597,8 +619,10 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-load", action="store_true",
                     help="skip the load phase that precedes the timed region (clock record)")
-    ap.add_argument("--profile", action="store_true",
-                    help="run 8 eager steps of the headline call and exit (ncu captures)")
+    ap.add_argument("--profile", nargs="?", const="gemm", choices=["gemm", "decode"],
+                    help="run 8 eager steps of the headline call (gemm) or 3 bf16 decodes "
+                         "of the 14336 x 4096 MLP up-projection at 4 bpw (decode), then exit "
+                         "(ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
