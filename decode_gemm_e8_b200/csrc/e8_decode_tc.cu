@@ -143,7 +143,7 @@ struct DecodeTcParams {
   const uint16_t* idx1;
   const void* idx2;
   int64_t slabs;          // N * K / 8192
-  int K, nh, log2R;       // R = nh / 64
+  int K, log2R;           // R = n_h / 64
   uint64_t seed;
   float alpha;
   const uint32_t* table;  // transformed pair table H_8 v / 4 (global)
@@ -526,9 +526,9 @@ cudaError_t launch_decode_tc(const DeviceCodebook& cb, const uint16_t* idx1, con
   p.idx2 = idx2;
   p.slabs = N * K / dtc::SLAB;
   p.K = (int)K;
-  p.nh = (int)hadamard_block(K);
+  const int64_t nh = hadamard_block(K);
   p.log2R = 0;
-  while ((64 << p.log2R) < p.nh) ++p.log2R;
+  while ((int64_t(64) << p.log2R) < nh) ++p.log2R;
   p.seed = seed;
   p.alpha = alpha;
   p.table = cb.h8table;

@@ -223,7 +223,7 @@ def test_decode_bit_exact(gcb, bpw, N, K):
                                  (64, 1024), (8, 2048), (40, 6144)])
 def test_decode_bit_exact_slab_shapes(gcb, bpw, N, K):
     # N K a multiple of 8192 and a Hadamard block of 1024..4096: the tensor-core
-    # decoder (two exact products per slab of 8192 weights)
+    # decoder (in-thread H8 stages and one exact product per slab of 8192 weights)
     assert (N * K) % 8192 == 0
     i1, i2 = _random_codes(N, K, bpw, 7 * N + K + bpw)
     s = 0.0211
