@@ -139,6 +139,13 @@ def _max_over_ranks(x: float, ws: int, device):
     return float(t.item())
 
 
+def _rank_layer_seeds(lay, rank: int):
+    """(weight seed, RHT seed) of the layer rank `rank` quantises and multiplies:
+    rank 0 takes the workload's own seeds, every other rank a distinct layer of
+    the same shape (weak scaling: no data-path collective)."""
+    return (lay.w_seed if rank == 0 else (lay.w_seed, rank)), lay.rht_seed + 7919 * rank
+
+
 def _barrier(ws):
     if ws > 1:
         import torch.distributed as dist
@@ -204,9 +211,9 @@ def run_ours(args):
     M = args.M
     cb = e8.Codebook(local)
     # every rank quantises its own layer (weak scaling); rank 0 is the seeded workload
-    W = synth.gaussian_weights(N, K, lay.std, lay.w_seed if rank == 0 else (lay.w_seed, rank))
+    w_seed, rs = _rank_layer_seeds(lay, rank)
+    W = synth.gaussian_weights(N, K, lay.std, w_seed)
     s = synth.suggest_scale(W, bpw)
-    rs = lay.rht_seed + 7919 * rank
     Wd = torch.from_numpy(W).to(dev)
     i1, i2 = e8.e8_encode(cb, Wd, bpw, rs, s)
     torch.cuda.synchronize()
