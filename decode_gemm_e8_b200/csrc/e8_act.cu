@@ -277,27 +277,36 @@ __global__ void __launch_bounds__(512, 4) k_act_q8(const uint16_t* __restrict__ 
   // the GEMM that follows may start at once: it touches nothing that this
   // kernel or its predecessor writes until its own wait for this grid
   grid_dep_launch();
-  grid_dep_wait();
+  // With K <= 4096 each thread quantises at most 8 values: the row is read,
+  // transformed and quantised before the wait for the preceding kernel (a
+  // kernel that releases its dependents early writes nothing that this one
+  // reads: X comes from a finished kernel), and only the stores wait for it,
+  // so that this work overlaps the tail of the preceding GEMM.
+  const bool early = K <= 4096;
+  if (!early) grid_dep_wait();
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int m = blockIdx.x;
-  // the output that the following GEMM accumulates into starts at zero
-  if (Yz) {
-    const int64_t per = ((yz_elems + gridDim.x - 1) / gridDim.x + 3) & ~int64_t(3);
-    const int64_t z0 = (int64_t)m * per, z1 = z0 + per < yz_elems ? z0 + per : yz_elems;
-    for (int64_t i = z0 + 4 * t; i < z1; i += 4 * blockDim.x) {
-      if (i + 4 <= z1) {
-        *reinterpret_cast<float4*>(Yz + i) = make_float4(0.f, 0.f, 0.f, 0.f);
-      } else {
-        for (int64_t j = i; j < z1; ++j) Yz[j] = 0.0f;
+  auto zero_outputs = [&]() {
+    // the output that the following GEMM accumulates into starts at zero
+    if (Yz) {
+      const int64_t per = ((yz_elems + gridDim.x - 1) / gridDim.x + 3) & ~int64_t(3);
+      const int64_t z0 = (int64_t)m * per, z1 = z0 + per < yz_elems ? z0 + per : yz_elems;
+      for (int64_t i = z0 + 4 * t; i < z1; i += 4 * blockDim.x) {
+        if (i + 4 <= z1) {
+          *reinterpret_cast<float4*>(Yz + i) = make_float4(0.f, 0.f, 0.f, 0.f);
+        } else {
+          for (int64_t j = i; j < z1; ++j) Yz[j] = 0.0f;
+        }
       }
     }
-  }
-  // padding rows 2M .. rows-1: zero bytes, zero sums
-  for (int pr = 2 * M + m; pr < rows; pr += M) {
-    for (int k = 16 * t; k < K; k += 16 * 512)
-      *reinterpret_cast<uint4*>(Xq + (size_t)pr * K + k) = make_uint4(0u, 0u, 0u, 0u);
-    if (t == 0) colsum[pr] = 0;
-  }
+    // padding rows 2M .. rows-1: zero bytes, zero sums
+    for (int pr = 2 * M + m; pr < rows; pr += M) {
+      for (int k = 16 * t; k < K; k += 16 * 512)
+        *reinterpret_cast<uint4*>(Xq + (size_t)pr * K + k) = make_uint4(0u, 0u, 0u, 0u);
+      if (t == 0) colsum[pr] = 0;
+    }
+  };
+  if (!early) zero_outputs();
   const uint16_t* xrow = X + (size_t)m * K;
   float mx = 0.0f;
   for (int kb = 0; kb < K; kb += 4096) {
@@ -399,6 +408,7 @@ __global__ void __launch_bounds__(512, 4) k_act_q8(const uint16_t* __restrict__ 
   int sum0 = 0, sum1 = 0;
   int8_t* q0row = Xq + (size_t)(2 * m) * K;
   int8_t* q1row = Xq + (size_t)(2 * m + 1) * K;
+  uint2 e0 = make_uint2(0u, 0u), e1 = make_uint2(0u, 0u);   // early: this thread's bytes
   for (int k = 8 * t; k < K; k += 8 * 512) {
     const float4 xa = *reinterpret_cast<const float4*>(s_row + k);
     const float4 xb = *reinterpret_cast<const float4*>(s_row + k + 4);
@@ -415,8 +425,13 @@ __global__ void __launch_bounds__(512, 4) k_act_q8(const uint16_t* __restrict__ 
       p0[i >> 2] |= (uint32_t)(ia & 0xFF) << (8 * (i & 3));
       p1[i >> 2] |= (uint32_t)(ib & 0xFF) << (8 * (i & 3));
     }
-    *reinterpret_cast<uint2*>(q0row + k) = make_uint2(p0[0], p0[1]);
-    *reinterpret_cast<uint2*>(q1row + k) = make_uint2(p1[0], p1[1]);
+    if (early) {
+      e0 = make_uint2(p0[0], p0[1]);
+      e1 = make_uint2(p1[0], p1[1]);
+    } else {
+      *reinterpret_cast<uint2*>(q0row + k) = make_uint2(p0[0], p0[1]);
+      *reinterpret_cast<uint2*>(q1row + k) = make_uint2(p1[0], p1[1]);
+    }
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) {
@@ -428,6 +443,14 @@ __global__ void __launch_bounds__(512, 4) k_act_q8(const uint16_t* __restrict__ 
     s_sum[1][warp] = sum1;
   }
   __syncthreads();
+  if (early) {
+    grid_dep_wait();
+    zero_outputs();
+    if (8 * t < K) {
+      *reinterpret_cast<uint2*>(q0row + 8 * t) = e0;
+      *reinterpret_cast<uint2*>(q1row + 8 * t) = e1;
+    }
+  }
   if (t < 32) {
     int a = lane < 16 ? s_sum[0][lane] : s_sum[1][lane - 16];
 #pragma unroll

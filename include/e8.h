@@ -137,12 +137,13 @@ int e8_act_rht(const uint16_t* X, int64_t M, int64_t K, uint64_t rht_seed, uint1
  * when N is not a multiple of 4): the last bits of Y can differ between runs.
  * workspace: at least e8_workspace_bytes(mode, M, N, K, bpw) bytes.
  * Ordering: the int8 path launches its kernels with programmatic dependent
- * launch; its GEMM kernel may read idx1, idx2 and the codebook before the
- * kernel that precedes the call on the stream has finished, if that kernel
- * releases its dependents early (griddepcontrol.launch_dependents).  Kernels
- * that do not release early (every kernel of this library that writes indices
- * included) are waited for in full.  X and Y are accessed only after the
- * preceding kernel has finished. */
+ * launch; its kernels may read X (K <= 4096), idx1, idx2 and the codebook
+ * before the kernel that precedes the call on the stream has finished, if
+ * that kernel releases its dependents early (griddepcontrol.launch_dependents).
+ * Kernels that do not release early (every kernel of this library that writes
+ * X-sized inputs or indices included) are waited for in full.  Y, the
+ * workspace and everything else are written only after the preceding kernel
+ * has finished. */
 int e8_gemm(const e8_codebook* cb, const uint16_t* X, int64_t M, const uint16_t* idx1,
             const void* idx2, int64_t N, int64_t K, int bpw, uint64_t rht_seed, float scale,
             float* Y, int mode, void* workspace, size_t ws_bytes, void* stream);
