@@ -48,7 +48,13 @@ namespace dtc {
 constexpr int SLAB = 8192;                  // weights per slab
 constexpr int GROUPS = SLAB / 8;
 constexpr int TABLE_BYTES = 131088;
-constexpr int STAGES = 3;                   // index words, operand and accumulator rings
+constexpr int STAGES = 3;                   // operand and accumulator rings
+// Index-word ring: an even number of stages, so that each stage serves one
+// decoder group only.  Bulk copies may land out of order; were a stage shared
+// by both groups, a group could reach its next use of the stage while the
+// other group's copy into it was still in flight, and the parity wait would
+// take the barrier two phases behind for the phase it waits for.
+constexpr int CSTAGES = 4;
 constexpr int CODE_BYTES = GROUPS * 4;      // idx1 (2 KB) + idx2 (up to 2 KB)
 constexpr int B_BYTES = 128 * 128;          // 128 rows x 64 fp16, 128-byte swizzled
 constexpr int YW_BYTES = 32 * 64;           // one readout warp's 32 x 32 bf16 tile
@@ -64,9 +70,9 @@ constexpr uint32_t D_COL = 64;              // three buffers of 64
 constexpr uint32_t TMEM_COLS = 256;
 // shared memory (after the table, from the next 1 KB boundary)
 constexpr int CODE_OFF = 0;
-constexpr int B_OFF = CODE_OFF + STAGES * CODE_BYTES;         // 12 KB
-constexpr int Y_OFF = B_OFF + STAGES * B_BYTES;               // 60 KB
-constexpr int SIGN_OFF = Y_OFF + RD_WARPS * 2 * YW_BYTES;     // 92 KB
+constexpr int B_OFF = CODE_OFF + CSTAGES * CODE_BYTES;        // 16 KB
+constexpr int Y_OFF = B_OFF + STAGES * B_BYTES;               // 64 KB
+constexpr int SIGN_OFF = Y_OFF + RD_WARPS * YW_BYTES;         // 80 KB
 constexpr int BAR_OFF = SIGN_OFF + SIGN_CHUNKS * 8;           // 96 KB
 constexpr int SMEM_TOTAL = TABLE_BYTES + 1024 + BAR_OFF + 256;
 static_assert(SMEM_TOTAL <= kMaxDynSmem, "shared memory budget");
@@ -174,12 +180,12 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
   uint8_t* ytile = smem + Y_OFF;
   uint32_t* sgn = reinterpret_cast<uint32_t*>(smem + SIGN_OFF);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
-  uint64_t* code_full = bars;                 // [3] index words landed
-  uint64_t* code_empty = bars + STAGES;       // [3] decoders hold them in registers
-  uint64_t* b_full = bars + 2 * STAGES;       // [3] operand written + accumulator buffer free
-  uint64_t* b_empty = bars + 3 * STAGES;      // [3] product done with the operand
-  uint64_t* d_full = bars + 4 * STAGES;       // [3] product in tensor memory
-  uint64_t* table_full = bars + 5 * STAGES;
+  uint64_t* code_full = bars;                 // [4] index words landed
+  uint64_t* code_empty = bars + CSTAGES;      // [4] decoders hold them in registers
+  uint64_t* b_full = bars + 2 * CSTAGES;      // [3] operand written + accumulator buffer free
+  uint64_t* b_empty = b_full + STAGES;        // [3] product done with the operand
+  uint64_t* d_full = b_empty + STAGES;        // [3] product in tensor memory
+  uint64_t* table_full = d_full + STAGES;
   uint64_t* drain = table_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile uint32_t* abort_flag = tmem_slot + 1;
@@ -191,9 +197,11 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
   const bool sgn_in_smem = chunks <= SIGN_CHUNKS;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < CSTAGES; ++s) {
       mbar_init(&code_full[s], 1);
       mbar_init(&code_empty[s], DEC_WARPS / 2);
+    }
+    for (int s = 0; s < STAGES; ++s) {
       mbar_init(&b_full[s], DEC_WARPS / 2 + RD_WARPS);
       mbar_init(&b_empty[s], 1);
       mbar_init(&d_full[s], 1);
@@ -214,7 +222,7 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
     }
     bulk_load(smem_raw + 8 * 16384, reinterpret_cast<const uint8_t*>(p.table) + 8 * 16384, 16,
               table_full);
-    for (int64_t i = 0; i < nsl && i < STAGES; ++i)
+    for (int64_t i = 0; i < nsl && i < CSTAGES; ++i)
       load_codes<BPW>(p, codes + i * CODE_BYTES, &code_full[i], (int64_t)blockIdx.x + i * gridDim.x);
     tma_prefetch_desc(&tmOut);
   }
@@ -261,17 +269,17 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      // slabs 0 .. STAGES - 1 were issued before the role split
+      // slabs 0 .. CSTAGES - 1 were issued before the role split
       int s = 0;
       uint32_t ph = 1;
-      int64_t issued = nsl < STAGES ? nsl : STAGES;
-      for (int64_t i = STAGES; i < nsl; ++i) {
+      int64_t issued = nsl < CSTAGES ? nsl : CSTAGES;
+      for (int64_t i = CSTAGES; i < nsl; ++i) {
         if (!mbar_wait_sleep(&code_empty[s], ph ^ 1u, abort_flag, status, kDevTimeoutEmpty))
           break;
         load_codes<BPW>(p, codes + s * CODE_BYTES, &code_full[s],
                         (int64_t)blockIdx.x + i * gridDim.x);
         ++issued;
-        if (++s == STAGES) {
+        if (++s == CSTAGES) {
           s = 0;
           ph ^= 1u;
         }
@@ -281,9 +289,9 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
         uint64_t t0 = global_timer_ns();
         while (!mbar_try_wait(table_full, 0))
           if (global_timer_ns() - t0 > 100000000ull) break;
-        for (int64_t j = issued > STAGES ? issued - STAGES : 0; j < issued; ++j) {
+        for (int64_t j = issued > CSTAGES ? issued - CSTAGES : 0; j < issued; ++j) {
           t0 = global_timer_ns();
-          while (!mbar_try_wait(&code_full[j % STAGES], (uint32_t)(j / STAGES) & 1u))
+          while (!mbar_try_wait(&code_full[j % CSTAGES], (uint32_t)(j / CSTAGES) & 1u))
             if (global_timer_ns() - t0 > 100000000ull) break;
         }
       }
@@ -332,10 +340,11 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
     const __half2 bias2 = __half2half2(__ushort_as_half((unsigned short)0x6880u));   // 2304
     bool ok = warp_wait(table_full, 0, abort_flag, status, kDevTimeoutFull);
     for (int64_t i = grp; i < nsl && ok; i += 2) {
-      const int s = (int)(i % STAGES);
-      const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
-      if (!warp_wait(&code_full[s], ph, abort_flag, status, kDevTimeoutFull)) break;
-      const uint8_t* cw = codes + s * CODE_BYTES;
+      const int cs = (int)(i % CSTAGES);
+      if (!warp_wait(&code_full[cs], (uint32_t)(i / CSTAGES) & 1u, abort_flag, status,
+                     kDevTimeoutFull))
+        break;
+      const uint8_t* cw = codes + cs * CODE_BYTES;
       const uint4 c1 = *reinterpret_cast<const uint4*>(cw + 16 * r);
       uint4 c2 = make_uint4(0u, 0u, 0u, 0u);
       if (BPW == 4) {
@@ -349,7 +358,9 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
       // before the producer's next bulk-copy write into the stage
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&code_empty[s]);
+      if (lane == 0) mbar_arrive(&code_empty[cs]);
+      const int s = (int)(i % STAGES);
+      const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
       // decode: group g -> four fp16 pairs 1024 + (H_8 z / 4 + 128), in
       // coordinate order
       __half2 x[8][4];
@@ -428,7 +439,7 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
     const uint32_t step = (uint32_t)(((uint64_t)gridDim.x * SLAB) % K);
     uint32_t base = (uint32_t)(((uint64_t)blockIdx.x * SLAB) % K);
     const uint32_t offm = (64u * m) % K;
-    uint8_t* ybuf = ytile + wi * 2u * YW_BYTES;
+    uint8_t* yt = ytile + wi * YW_BYTES;
     uint32_t yoff[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) yoff[j] = lane * 64u + ((j ^ ((lane >> 1) & 3u)) << 4);
@@ -459,9 +470,8 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
         const float b = __fmul_rn(__uint_as_float(y[2 * e + 1]), alpha4);
         pk[e] = pack_bf16x2(a, b) ^ ((W << e) & 0x80008000u);
       }
-      // the store of slab i - 2 has read this stage
-      uint8_t* yt = ybuf + (uint32_t)(i & 1) * YW_BYTES;
-      if (i >= 2 && lane == 0) bulk_wait_read_1();
+      // the store of slab i - 1 has read the tile
+      if (i >= 1 && lane == 0) bulk_wait_read_all();
       __syncwarp();
 #pragma unroll
       for (int j = 0; j < 4; ++j)

@@ -20,10 +20,12 @@
 // order of the few partial sums of an output is not fixed.
 //
 // Roles (one CTA per SM):
-//   warp 0      TMA producer: the codebook pair table (once), the index tiles
-//               (a ring released by the decoders as soon as they hold the
-//               indices in registers; filled before waiting for the transform
-//               kernel) and the Xq tiles (a ring released by the MMA)
+//   warp 0      TMA producer: the codebook pair table (once) and the index
+//               tiles (a ring released by the decoders as soon as they hold
+//               the indices in registers), without waiting for the transform
+//               kernel
+//   warp 23     TMA producer of the Xq tiles (a ring released by the MMA),
+//               after the transform kernel
 //   warps 1, 22 tensor-memory allocation (warp 1); one elected lane of each
 //               issues tcgen05.mma (M = 128 weight rows, N = rows_b, K = 32)
 //               and the commits for the even / odd units
@@ -49,7 +51,8 @@ constexpr int DEC_GROUPS = 2;
 constexpr int DEC_WARPS = 8 * DEC_GROUPS;
 constexpr int EPI_WARP0 = 2 + DEC_WARPS;
 constexpr int MMA2_WARP = EPI_WARP0 + 4;  // issuer of the odd units
-constexpr int THREADS = 32 * (MMA2_WARP + 1);
+constexpr int XQ_WARP = MMA2_WARP + 1;    // producer of the Xq tiles
+constexpr int THREADS = 32 * (XQ_WARP + 1);
 constexpr int TABLE_BYTES = 131088;       // 32769 u32 entries, padded to 16 bytes
 constexpr int I1_BYTES = ROWS * GROUPS * 2;
 constexpr uint32_t ACC_COLS = 64;         // int32 accumulator columns per buffer
@@ -57,6 +60,7 @@ constexpr uint32_t ACC_COLS = 64;         // int32 accumulator columns per buffe
 constexpr uint32_t ACC_TOTAL = 4 * ACC_COLS;
 constexpr uint32_t A_COLS = KU / 4;       // 4 int8 weights per TMEM column
 constexpr int MAX_STAGES = 8;
+static_assert(MAX_STAGES % 2 == 0, "each operand stage serves one decoder group and one issuer");
 constexpr int AUX_BYTES = 512;            // per-token steps [32] and row sums [64]
 constexpr int BAR_BYTES = 512;
 // shared memory left free on the SM for a CTA of the activation transform
@@ -92,6 +96,12 @@ __host__ __device__ inline SkPlan sk_plan(int rows_b, int bpw) {
     if (budget - p.sx * p.b_bytes >= 4 * p.code_bytes) break;
   p.sc = (budget - p.sx * p.b_bytes) / p.code_bytes;
   if (p.sc > MAX_STAGES) p.sc = MAX_STAGES;
+  // An even number of index stages keeps each stage with one decoder group
+  // (groups take alternate units).  Bulk copies may land out of order: were a
+  // stage shared, a group could reach its next use of it while the other
+  // group's copy into it was still in flight, and the parity wait would take
+  // the barrier two phases behind for the phase it waits for.
+  p.sc &= ~1;
   p.code_off = p.sx * p.b_bytes;
   p.y_off = p.code_off + p.sc * p.code_bytes;
   p.aux_off = p.y_off + y_bytes;
@@ -289,31 +299,10 @@ __global__ void __maxnreg__(64)
           }
         }
       };
-      if (early_codes) next_codes(nu < SC + SA ? nu : SC + SA);
-      grid_dep_wait();
-      int sa = 0;                    // operand stage of unit i
-      uint32_t aph = 0;
-      int ja = 0;                    // operand stage of unit i - SX, whose MMAs free
-      uint32_t jph = 0;              // the Xq stage of unit i
-      for (int i = 0; i < nu && ok; ++i) {
-        next_codes(i + SC < nu ? i + SC : nu);
-        if (!ok) break;
-        if (i >= SX) {
-          if (!mbar_wait_sleep(&a_empty[ja], jph, abort_flag, status, kDevTimeoutEmpty)) break;
-          if (++ja == SA) {
-            ja = 0;
-            jph ^= 1u;
-          }
-        }
-        const int u = u_begin + i;
-        mbar_arrive_expect_tx(&full_a[sa], (uint32_t)plan.b_bytes);
-        tma_load_2d(xq_ring + (i % SX) * plan.b_bytes, &tmB, &full_a[sa], (u % kunits) * KU, 0);
-        if (++sa == SA) {
-          sa = 0;
-          aph ^= 1u;
-        }
-      }
-      (void)aph;
+      // every index tile, as the decoders free stages; the Xq tiles, which
+      // come from the preceding kernel, have a producer of their own
+      if (!early_codes) grid_dep_wait();
+      next_codes(nu);
       if (ld_shared_volatile(abort_flag)) {
         // let the copies in flight land before the CTA exits (bounded waits:
         // a stage's barrier may never complete once the other roles stopped)
@@ -395,6 +384,34 @@ __global__ void __maxnreg__(64)
         if (global_timer_ns() - t0 > 200000000ull) break;
     }
     __syncwarp();
+  } else if (warp == XQ_WARP) {
+    // ------------------------------------------------------------ Xq tiles
+    if (lane == 0) {
+      grid_dep_wait();
+      int sa = 0;                    // operand stage of unit i
+      for (int i = 0; i < nu; ++i) {
+        // the Xq stage of unit i was last read by the MMAs of unit i - SX, and
+        // the operand stage's barrier must have completed the phase of unit
+        // i - SA before this unit's arrival (the two issuers' MMAs, of
+        // alternate units, complete in no fixed order)
+        if (i >= SX && !mbar_wait_sleep(&a_empty[(i - SX) % SA], (uint32_t)((i - SX) / SA) & 1u,
+                                        abort_flag, status, kDevTimeoutEmpty))
+          break;
+        if (i >= SA && !mbar_wait_sleep(&a_empty[(i - SA) % SA], (uint32_t)((i - SA) / SA) & 1u,
+                                        abort_flag, status, kDevTimeoutEmpty))
+          break;
+        const int u = u_begin + i;
+        mbar_arrive_expect_tx(&full_a[sa], (uint32_t)plan.b_bytes);
+        tma_load_2d(xq_ring + (i % SX) * plan.b_bytes, &tmB, &full_a[sa], (u % kunits) * KU, 0);
+        if (++sa == SA) sa = 0;
+      }
+      if (ld_shared_volatile(abort_flag)) {
+        // let the copies in flight land before the CTA exits
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 1000000ull) {
+        }
+      }
+    }
   } else if (warp < EPI_WARP0) {
     // ------------------------------------------------------------ decoders
     const int dw = warp - 2;
