@@ -92,15 +92,19 @@ def _check(rc: int, where: str):
 
 
 def _ptr(t):
-    if t is None:
-        return None
-    return ctypes.c_void_p(t.data_ptr())
+    # the argtypes declare c_void_p, which takes a plain integer address
+    return None if t is None else t.data_ptr()
 
 
 def _stream(stream=None):
     import torch
-    s = stream if stream is not None else torch.cuda.current_stream()
-    return ctypes.c_void_p(s.cuda_stream)
+    if stream is not None:
+        return stream.cuda_stream
+    try:
+        # the raw handle of the current stream, without building a Stream object
+        return torch._C._cuda_getCurrentRawStream(torch.cuda.current_device())
+    except AttributeError:
+        return torch.cuda.current_stream().cuda_stream
 
 
 class Codebook:
@@ -222,8 +226,9 @@ def e8_gemm(cb: Codebook, X, idx1, idx2, N: int, K: int, bpw: int, rht_seed: int
     dev = X.device
     if Y is None:
         Y = torch.empty((M, N), dtype=torch.float32, device=dev)
-    need = e8_workspace_bytes(mode, M, N, K, bpw)
-    ws = _workspace(need, dev, workspace)
+    # a caller's workspace is checked by the library (E8_EWORKSPACE if too small)
+    ws = workspace if workspace is not None else _workspace(
+        e8_workspace_bytes(mode, M, N, K, bpw), dev)
     _check(load_library().e8_gemm(cb.handle, _ptr(X), M, _ptr(idx1), _ptr(idx2), N, K, int(bpw),
                                   int(rht_seed) & (2**64 - 1), float(scale), _ptr(Y), int(mode),
                                   _ptr(ws), ws.numel(), _stream(stream)), "e8_gemm")

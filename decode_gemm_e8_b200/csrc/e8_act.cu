@@ -468,12 +468,9 @@ cudaError_t launch_act_q8(const uint16_t* X, int64_t M, int64_t K, uint64_t seed
   if (nh < 256 || nh > 4096 || K > 32768 || M < 1 || M > 32 || rows < 2 * M || rows > 64)
     return cudaErrorInvalidValue;
   const size_t smem = (size_t)K * sizeof(float);
-  cudaError_t e = ensure_smem_limit(k_act_q8, kMaxDynSmem);
-  if (e != cudaSuccess) return e;
   // the same shared-memory carveout as the GEMM that follows, so that the two
   // can share an SM (an SM runs CTAs of one carveout at a time)
-  e = cudaFuncSetAttribute(k_act_q8, cudaFuncAttributePreferredSharedMemoryCarveout,
-                           cudaSharedmemCarveoutMaxShared);
+  cudaError_t e = ensure_smem_limit(k_act_q8, kMaxDynSmem, true);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)M);

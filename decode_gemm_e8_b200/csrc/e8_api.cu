@@ -13,7 +13,7 @@
 
 namespace e8 {
 
-cudaError_t ensure_smem_limit_ptr(const void* kernel, int bytes) {
+cudaError_t ensure_smem_limit_ptr(const void* kernel, int bytes, bool carveout_max) {
   // fixed table, no heap use on any launch path
   constexpr int kSlots = 256;
   static std::mutex mu;
@@ -35,6 +35,9 @@ cudaError_t ensure_smem_limit_ptr(const void* kernel, int bytes) {
     if (bytes > cap) bytes = cap;
   }
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && carveout_max)
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
   if (e == cudaSuccess && used < kSlots) {
     kern[used] = kernel;
     devs[used] = dev;

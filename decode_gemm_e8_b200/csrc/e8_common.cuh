@@ -458,10 +458,12 @@ __device__ __forceinline__ float bf16_hi_to_f32(uint32_t v) {
 // Raises a kernel's dynamic shared-memory limit once per (kernel, device) on
 // the host.  Done on first use rather than per launch so that launches can be
 // captured into CUDA graphs without any non-stream API call in between.
-cudaError_t ensure_smem_limit_ptr(const void* kernel, int bytes);
+// Raises the kernel's dynamic shared-memory limit (and, with carveout_max, asks
+// for the largest shared-memory carveout) once per kernel and device.
+cudaError_t ensure_smem_limit_ptr(const void* kernel, int bytes, bool carveout_max);
 template <class Kernel>
-inline cudaError_t ensure_smem_limit(Kernel* k, int bytes) {
-  return ensure_smem_limit_ptr(reinterpret_cast<const void*>(k), bytes);
+inline cudaError_t ensure_smem_limit(Kernel* k, int bytes, bool carveout_max = false) {
+  return ensure_smem_limit_ptr(reinterpret_cast<const void*>(k), bytes, carveout_max);
 }
 constexpr int kMaxDynSmem = 232448;   // 227 KB per block on sm_100
 

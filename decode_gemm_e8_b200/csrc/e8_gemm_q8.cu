@@ -618,10 +618,8 @@ static cudaError_t launch_gemm_q8(const DeviceCodebook& cb, const ActQ8Args& a, 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   auto kern = a.rows_b <= 32 ? k_gemm_q8<BPW, 32> : k_gemm_q8<BPW, 64>;
-  cudaError_t e = ensure_smem_limit(kern, kMaxDynSmem);
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
-                           cudaSharedmemCarveoutMaxShared);
+  // the largest carveout, as the transform kernel has: CTAs of the two can share an SM
+  cudaError_t e = ensure_smem_limit(kern, kMaxDynSmem, true);
   if (e != cudaSuccess) return e;
   e = cudaLaunchKernelEx(&cfg, kern, tb, ti1, ti2, ty, cb, (int)a.M, (int)a.N, (int)a.K,
                          a.rows_b, a.alpha, a.scales, a.colsum, a.Y, use_tma_y, a.early_codes);

@@ -31,9 +31,31 @@ inline EncodeTiledFn encode_tiled_fn() {
 
 // Row-major [rows][cols] tensor of `elem_bytes`-byte elements; box = [box_rows][box_cols].
 // Returns false if the driver rejects the description.
+// A map depends only on these arguments, so the last few encodings of each
+// host thread are kept and reused (the steady state of a layer loop encodes
+// nothing).
 inline bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
                          int elem_bytes, uint64_t rows, uint64_t cols, uint32_t box_rows,
                          uint32_t box_cols, CUtensorMapSwizzle swizzle) {
+  struct Entry {
+    const void* base;
+    uint64_t rows, cols;
+    uint32_t box_rows, box_cols;
+    int dtype, elem_bytes, swizzle;
+    CUtensorMap map;
+  };
+  constexpr int kEntries = 16;
+  thread_local Entry cache[kEntries];
+  thread_local int used = 0, next = 0;
+  for (int i = 0; i < used; ++i) {
+    const Entry& c = cache[i];
+    if (c.base == base && c.rows == rows && c.cols == cols && c.box_rows == box_rows &&
+        c.box_cols == box_cols && c.dtype == (int)dtype && c.elem_bytes == elem_bytes &&
+        c.swizzle == (int)swizzle) {
+      *map = c.map;
+      return true;
+    }
+  }
   EncodeTiledFn fn = encode_tiled_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
@@ -43,7 +65,20 @@ inline bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType
   CUresult r = fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  if (r != CUDA_SUCCESS) return false;
+  Entry& e = cache[next];
+  e.base = base;
+  e.rows = rows;
+  e.cols = cols;
+  e.box_rows = box_rows;
+  e.box_cols = box_cols;
+  e.dtype = (int)dtype;
+  e.elem_bytes = elem_bytes;
+  e.swizzle = (int)swizzle;
+  e.map = *map;
+  next = (next + 1) % kEntries;
+  if (used < kEntries) ++used;
+  return true;
 }
 
 }  // namespace e8
