@@ -280,26 +280,40 @@ def run_ours(args):
     r_ms = _time_graphs(rht_only, kern_steps, args.warmup, stream)
     rht_us = r_ms * 1e3 / kern_steps
 
-    # end to end through the public API with host buffers
-    Xpin = torch.from_numpy(Xh.view(np.int16)).view(torch.bfloat16).pin_memory()
-    Ypin = torch.empty((M, N), dtype=torch.float32).pin_memory()
-    Xe = torch.empty_like(X)
-    e2e_steps = min(args.steps, 2000)
-    with torch.cuda.stream(stream):
-        for i in range(max(3, min(args.warmup, 50))):
-            Xe.copy_(Xpin, non_blocking=True)
-            step(i)
-            Ypin.copy_(Y, non_blocking=True)
-        torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for i in range(e2e_steps):
-            Xe.copy_(Xpin, non_blocking=True)
+    # end to end through the public API with host buffers: every step copies its
+    # input in from pinned host memory and its result out to pinned host memory;
+    # two buffer slots on two streams let one step's copies overlap the other's
+    # kernels, as a serving loop would
+    streams = [stream, torch.cuda.Stream(device=dev)]
+    Xpin = [torch.from_numpy(Xh.view(np.int16)).view(torch.bfloat16).pin_memory() for _ in range(2)]
+    Ypin = [torch.empty((M, N), dtype=torch.float32).pin_memory() for _ in range(2)]
+    Xe = [torch.empty_like(X) for _ in range(2)]
+    Ye = [torch.empty_like(Y) for _ in range(2)]
+    wse = [wsb, torch.empty_like(wsb)]
+
+    def e2e_step(i):
+        k = i & 1
+        st = streams[k]
+        with torch.cuda.stream(st):
+            Xe[k].copy_(Xpin[k], non_blocking=True)
             c1, c2 = codes[i % ROTATE]
-            e8.e8_gemm(cb, Xe, c1, c2, N, K, bpw, rs, s, mode=mode, Y=Y, workspace=wsb,
-                       stream=stream)
-            Ypin.copy_(Y, non_blocking=True)
-        b.record(stream)
+            e8.e8_gemm(cb, Xe[k], c1, c2, N, K, bpw, rs, s, mode=mode, Y=Ye[k], workspace=wse[k],
+                       stream=st)
+            Ypin[k].copy_(Ye[k], non_blocking=True)
+
+    e2e_steps = min(args.steps, 2000)
+    for i in range(max(4, min(args.warmup, 50))):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(streams[0])
+    streams[1].wait_event(a)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    done1 = torch.cuda.Event()
+    done1.record(streams[1])
+    streams[0].wait_event(done1)
+    b.record(streams[0])
     torch.cuda.synchronize()
     e2e_ms = _max_over_ranks(a.elapsed_time(b), ws, dev)
     e2e_val = flop_step * e2e_steps * ws / (e2e_ms / 1e3) / 1e12
@@ -353,7 +367,9 @@ def run_ours(args):
             },
             "e2e": {"value": round(e2e_val, 3), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 4,
-                    "steps": e2e_steps, "path": "pinned host X -> e8_gemm -> pinned host Y"},
+                    "steps": e2e_steps,
+                    "path": "pinned host X -> e8_gemm -> pinned host Y, two buffer slots on two "
+                            "streams"},
             "gpu_launches": launches,
             "clocks": clocks,
             "rows": rows_out,
