@@ -505,7 +505,41 @@ def _decode_sweep_rows(e8, synth, cb, dev, stream, peaks):
             "ms_32_layers": round(32 * t * 1e3, 3), "GB_s": round(byt / t / 1e9, 1),
             "hbm_frac": round(byt / t / 1e9 / peaks["hbm_gbs"], 4)}
         del data
+        rows["encode_llama3_8b_layer_b%d" % bpw] = _encode_layer_row(e8, synth, cb, dev, stream,
+                                                                      mats, bpw)
     return rows
+
+
+def _encode_layer_row(e8, synth, cb, dev, stream, mats, bpw):
+    """Batched RHT + exact nearest-point encode of the 7 matrices of one
+    Llama-3-8B-shaped layer (weights N(0, 0.02^2) drawn on the device, one scale
+    per matrix from its rms); the 32-layer figure is 32 times the layer."""
+    import torch
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(200 + bpw)
+    total_s = 0.0
+    nw = 0
+    for lay in mats:
+        W = torch.randn((lay.N, lay.K), generator=gen, device=dev, dtype=torch.float32) * lay.std
+        rms = float(torch.sqrt(torch.mean(W.double() ** 2)))
+        s = float(np.float32(rms / synth.SIGMA_T[bpw]))
+        i1 = torch.empty((lay.N, lay.K // 8), dtype=torch.uint16, device=dev)
+        i2 = (torch.empty((lay.N, lay.K // 8), dtype=torch.uint8 if bpw == 3 else torch.uint16,
+                          device=dev) if bpw > 2 else None)
+        wsz = e8.e8_workspace_bytes(e8.E8_OP_ENCODE, 0, lay.N, lay.K, bpw)
+        ws = torch.empty(max(16, wsz), dtype=torch.uint8, device=dev)
+        e8.e8_encode(cb, W, bpw, lay.rht_seed, s, idx1=i1, idx2=i2, workspace=ws, stream=stream)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        e8.e8_encode(cb, W, bpw, lay.rht_seed, s, idx1=i1, idx2=i2, workspace=ws, stream=stream)
+        b.record(stream)
+        torch.cuda.synchronize()
+        total_s += a.elapsed_time(b) / 1e3
+        nw += lay.N * lay.K
+        del W, i1, i2, ws
+    return {"weights_per_s": nw / total_s, "ms_per_layer": round(total_s * 1e3, 2),
+            "s_32_layers": round(32 * total_s, 2)}
 
 
 def _other_rows(e8, synth, cb, Wd, W, codes, X, N, K, bpw, rs, s, dev, stream, args, peaks):
