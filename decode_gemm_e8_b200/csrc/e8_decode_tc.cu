@@ -34,7 +34,7 @@
 //   warps 10-17 readout: T -> scale, sign, bf16, TMA store
 // The product of slab i waits on one barrier: the decoder warps that wrote
 // its operand stage and the readout warps that emptied its accumulator
-// buffer (slab i - 3) arrive on the same one.
+// buffer (slab i - 4) arrive on the same one.
 #include <cuda_fp16.h>
 
 #include "e8_common.cuh"
@@ -48,17 +48,17 @@ namespace dtc {
 constexpr int SLAB = 8192;                  // weights per slab
 constexpr int GROUPS = SLAB / 8;
 constexpr int TABLE_BYTES = 131088;
-constexpr int STAGES = 3;                   // operand and accumulator rings
+constexpr int STAGES = 4;                   // operand and accumulator rings
 // Index-word ring: an even number of stages, so that each stage serves one
 // decoder group only.  Bulk copies may land out of order; were a stage shared
 // by both groups, a group could reach its next use of the stage while the
 // other group's copy into it was still in flight, and the parity wait would
 // take the barrier two phases behind for the phase it waits for.
-constexpr int CSTAGES = 4;
+constexpr int CSTAGES = 2;
 constexpr int CODE_BYTES = GROUPS * 4;      // idx1 (2 KB) + idx2 (up to 2 KB)
 constexpr int B_BYTES = 128 * 128;          // 128 rows x 64 fp16, 128-byte swizzled
 constexpr int YW_BYTES = 32 * 64;           // one readout warp's 32 x 32 bf16 tile
-constexpr int SIGN_CHUNKS = 512;            // sign words kept in shared memory (K <= 32768)
+constexpr int SIGN_CHUNKS = 256;            // sign words kept in shared memory (K <= 16384)
 constexpr int DEC_WARP0 = 2;
 constexpr int DEC_WARPS = 8;                // two groups of four
 constexpr int RD_WARP0 = DEC_WARP0 + DEC_WARPS;
@@ -66,13 +66,13 @@ constexpr int RD_WARPS = 8;
 constexpr int THREADS = 32 * (RD_WARP0 + RD_WARPS);
 // tensor memory columns
 constexpr uint32_t A_COL = 0;               // diag(H_R ...), f16: 64 columns
-constexpr uint32_t D_COL = 64;              // three buffers of 64
-constexpr uint32_t TMEM_COLS = 256;
+constexpr uint32_t D_COL = 64;              // four buffers of 64
+constexpr uint32_t TMEM_COLS = 512;
 // shared memory (after the table, from the next 1 KB boundary)
 constexpr int CODE_OFF = 0;
-constexpr int B_OFF = CODE_OFF + CSTAGES * CODE_BYTES;        // 16 KB
-constexpr int Y_OFF = B_OFF + STAGES * B_BYTES;               // 64 KB
-constexpr int SIGN_OFF = Y_OFF + RD_WARPS * YW_BYTES;         // 80 KB
+constexpr int B_OFF = CODE_OFF + CSTAGES * CODE_BYTES;        // 8 KB
+constexpr int Y_OFF = B_OFF + STAGES * B_BYTES;               // 72 KB
+constexpr int SIGN_OFF = Y_OFF + RD_WARPS * YW_BYTES;         // 88 KB
 constexpr int BAR_OFF = SIGN_OFF + SIGN_CHUNKS * 8;           // 96 KB
 constexpr int SMEM_TOTAL = TABLE_BYTES + 1024 + BAR_OFF + 256;
 static_assert(SMEM_TOTAL <= kMaxDynSmem, "shared memory budget");
@@ -180,11 +180,11 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
   uint8_t* ytile = smem + Y_OFF;
   uint32_t* sgn = reinterpret_cast<uint32_t*>(smem + SIGN_OFF);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
-  uint64_t* code_full = bars;                 // [4] index words landed
-  uint64_t* code_empty = bars + CSTAGES;      // [4] decoders hold them in registers
-  uint64_t* b_full = bars + 2 * CSTAGES;      // [3] operand written + accumulator buffer free
-  uint64_t* b_empty = b_full + STAGES;        // [3] product done with the operand
-  uint64_t* d_full = b_empty + STAGES;        // [3] product in tensor memory
+  uint64_t* code_full = bars;                 // [2] index words landed
+  uint64_t* code_empty = bars + CSTAGES;      // [2] decoders hold them in registers
+  uint64_t* b_full = bars + 2 * CSTAGES;      // [4] operand written + accumulator buffer free
+  uint64_t* b_empty = b_full + STAGES;        // [4] product done with the operand
+  uint64_t* d_full = b_empty + STAGES;        // [4] product in tensor memory
   uint64_t* table_full = d_full + STAGES;
   uint64_t* drain = table_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -406,7 +406,7 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
             x[g + h][e] = __hsub2(a, b);
           }
         }
-      // the product of slab i - 3 has read this operand stage
+      // the product of slab i - 4 has read this operand stage
       if (i >= STAGES && !warp_wait(&b_empty[s], ph ^ 1u, abort_flag, status, kDevTimeoutMma))
         break;
       // row r of the N-major operand: U[r][8 g' + k'] for g' = 0..7, one
@@ -453,7 +453,7 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&b_full[s]);   // accumulator buffer free for slab i + 3
+      if (lane == 0) mbar_arrive(&b_full[s]);   // accumulator buffer free for slab i + 4
       uint32_t pos = base + offm;
       if (pos >= K) pos -= K;
       uint32_t W;
