@@ -538,8 +538,49 @@ def _encode_layer_row(e8, synth, cb, dev, stream, mats, bpw):
         total_s += a.elapsed_time(b) / 1e3
         nw += lay.N * lay.K
         del W, i1, i2, ws
+    byt = nw * (4 + bpw / 8)
     return {"weights_per_s": nw / total_s, "ms_per_layer": round(total_s * 1e3, 2),
-            "s_32_layers": round(32 * total_s, 2)}
+            "s_32_layers": round(32 * total_s, 2), "GB_s": round(byt / total_s / 1e9, 2),
+            "hbm_frac": round(byt / total_s / 1e9 / _peaks()["hbm_gbs"], 5)}
+
+
+def _layer_chain_rows(e8, synth, cb, dev, stream, peaks, M=16):
+    """The seven projections of one Llama-3-8B-shaped decoder layer (q, k, v, o,
+    gate, up, down) through the fused small-batch decode GEMM, back to back in one
+    stream (programmatic dependent launch between the calls), M tokens, per rate;
+    two code sets alternate so more than L2 streams from HBM."""
+    import torch
+    rows = {}
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(300)
+    for bpw in (2, 3, 4):
+        mats = synth.workloads()["llama3_8b_x32_b%d" % bpw].layers[:7]
+        data = []
+        for lay in mats:
+            codes = [_random_codes(torch, dev, lay.N, lay.K, bpw, gen) for _ in range(2)]
+            X = (torch.randn((M, lay.K), generator=gen, device=dev)).to(torch.bfloat16)
+            Y = torch.empty((M, lay.N), dtype=torch.float32, device=dev)
+            wsz = e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT, M, lay.N, lay.K, bpw)
+            ws = torch.empty(max(16, wsz), dtype=torch.uint8, device=dev)
+            data.append((lay, codes, X, Y, ws))
+
+        def chain(i, data=data, bpw=bpw):
+            for lay, codes, X, Y, ws in data:
+                c1, c2 = codes[i % 2]
+                e8.e8_gemm(cb, X, c1, c2, lay.N, lay.K, bpw, lay.rht_seed, 0.02,
+                           mode=e8.E8_GEMM_ACT_RHT, Y=Y, workspace=ws, stream=stream)
+
+        n = 200
+        t = _time_graphs(chain, n, 4, stream) / 1e3 / n
+        nw = sum(lay.N * lay.K for lay in mats)
+        flop = sum(2.0 * M * lay.N * lay.K for lay in mats)
+        byt = sum(lay.N * lay.K * bpw / 8 + M * lay.K * 2 + M * lay.N * 4 for lay in mats)
+        rows["gemm_llama3_8b_layer_m%d_b%d" % (M, bpw)] = {
+            "us_per_layer": round(t * 1e6, 1), "TFLOP_s": round(flop / t / 1e12, 2),
+            "decoded_weights_per_s": nw / t, "GB_s": round(byt / t / 1e9, 1),
+            "hbm_frac": round(byt / t / 1e9 / peaks["hbm_gbs"], 4)}
+        del data
+    return rows
 
 
 def _other_rows(e8, synth, cb, Wd, W, codes, X, N, K, bpw, rs, s, dev, stream, args, peaks):
@@ -579,6 +620,7 @@ def _other_rows(e8, synth, cb, Wd, W, codes, X, N, K, bpw, rs, s, dev, stream, a
                               "bytes_per_weight": 2 + bpw / 8}
     rows.update(_prefill_rows(e8, synth, cb, dev, stream, peaks))
     rows.update(_decode_sweep_rows(e8, synth, cb, dev, stream, peaks))
+    rows.update(_layer_chain_rows(e8, synth, cb, dev, stream, peaks))
     for Mx in (1, 4):
         Xm = X[:Mx].contiguous()
         Ym = torch.empty((Mx, N), dtype=torch.float32, device=dev)
