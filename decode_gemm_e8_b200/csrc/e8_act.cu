@@ -249,169 +249,168 @@ cudaError_t launch_act_rht(const uint16_t* X, int64_t M, int64_t K, uint64_t see
 
 namespace e8 {
 
-// Activation transform for the int8 tensor-core path.  One CTA of 512
-// threads per token row, 8 values per thread, the row in chunks of up to
-// 4096 positions (several Hadamard blocks when n_h < 4096).  Position
-// p = 256 w + 8 l + e (warp w, lane l, register e): the stages of the
-// three low bits run in registers, the next five by warp shuffles, and the
-// stages across warps (n_h > 256) after one exchange through shared memory,
-// where thread t takes the 8 positions g + 256 (8 (t & 1) + j), g = t >> 1,
-// three stages in registers and the last by a shuffle with its neighbour.
-// The row's largest magnitude fixes the token's step s_m = max / 127, and the
+
+// Activation transform for the int8 tensor-core path.  A token row is cut
+// into chunks of up to 4096 positions, one CTA of 512 threads per chunk and
+// one thread-block cluster per row (at most 8 CTAs: K <= 32768).  A Hadamard
+// block (n_h a power of two, 256 <= n_h <= 4096, dividing K) never straddles
+// a chunk.  Inside a chunk, position p = 256 w + 8 l + e (warp w, lane l,
+// register e): the stages of the three low bits run in registers, the next
+// five by warp shuffles, and the stages across warps (n_h > 256) after one
+// exchange through shared memory, where thread t takes the 8 positions
+// g + 256 (8 (t & 1) + j), g = t >> 1, three stages in registers and the last
+// by a shuffle with its neighbour.
+// The row's largest magnitude (the chunks' maxima, exchanged through
+// distributed shared memory) fixes the token's step s_m = max / 127, and the
 // row is written as two int8 pieces
 //   q0 = rint(x / s_m),  q1 = rint((x - q0 s_m) * 128 / s_m),  |q1| <= 64,
 // so x = s_m (q0 + q1 / 128) + e with |e| <= s_m / 256.  Piece rows are
 // interleaved (row 2m = q0, row 2m + 1 = q1); colsum[row] = sum_k Xq[row][k]
-// lets the GEMM remove the +128 bias of its unsigned weight operand exactly.
-// Kept small (32 registers, K floats of shared memory) so that it can share an
-// SM with a CTA of the GEMM that follows it.
+// (the chunks' sums, added by the cluster's first CTA) lets the GEMM remove
+// the +128 bias of its unsigned weight operand exactly.
+// Kept small (32 registers, at most 16 KB of shared memory) so that a CTA can
+// share an SM with a CTA of the GEMM that follows it; the transform runs
+// before the wait for the preceding kernel, and only the stores wait for it.
 __global__ void __launch_bounds__(512, 4) k_act_q8(const uint16_t* __restrict__ X, int M, int K,
                                                    int nh, uint64_t seed,
                                                    int8_t* __restrict__ Xq,
                                                    float* __restrict__ scales,
                                                    int32_t* __restrict__ colsum, int rows,
                                                    float* __restrict__ Yz, int64_t yz_elems) {
-  extern __shared__ __align__(16) float s_row[];   // K floats
+  extern __shared__ __align__(16) float chunk[];   // the chunk's positions
   __shared__ float s_max[16];
   __shared__ int s_sum[2][16];
+  __shared__ float s_cmax;     // the chunk's largest magnitude, read by the cluster
+  __shared__ int s_csum[2];    // the chunk's piece sums, read by the cluster's CTA 0
+  __shared__ float s_amax;     // the row's largest magnitude
   // the GEMM that follows may start at once: it touches nothing that this
-  // kernel or its predecessor writes until its own wait for this grid
-  grid_dep_launch();
-  // With K <= 4096 each thread quantises at most 8 values: the row is read,
-  // transformed and quantised before the wait for the preceding kernel (a
+  // kernel or its predecessor writes until its own wait for this grid.  A
   // kernel that releases its dependents early writes nothing that this one
-  // reads: X comes from a finished kernel), and only the stores wait for it,
-  // so that this work overlaps the tail of the preceding GEMM.
-  const bool early = K <= 4096;
-  if (!early) grid_dep_wait();
+  // reads (X comes from a finished kernel), so everything up to the stores
+  // overlaps the tail of the preceding kernel.
+  grid_dep_launch();
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  const int m = blockIdx.x;
-  auto zero_outputs = [&]() {
-    // the output that the following GEMM accumulates into starts at zero
-    if (Yz) {
-      const int64_t per = ((yz_elems + gridDim.x - 1) / gridDim.x + 3) & ~int64_t(3);
-      const int64_t z0 = (int64_t)m * per, z1 = z0 + per < yz_elems ? z0 + per : yz_elems;
-      for (int64_t i = z0 + 4 * t; i < z1; i += 4 * blockDim.x) {
-        if (i + 4 <= z1) {
-          *reinterpret_cast<float4*>(Yz + i) = make_float4(0.f, 0.f, 0.f, 0.f);
-        } else {
-          for (int64_t j = i; j < z1; ++j) Yz[j] = 0.0f;
-        }
-      }
-    }
-    // padding rows 2M .. rows-1: zero bytes, zero sums
-    for (int pr = 2 * M + m; pr < rows; pr += M) {
-      for (int k = 16 * t; k < K; k += 16 * 512)
-        *reinterpret_cast<uint4*>(Xq + (size_t)pr * K + k) = make_uint4(0u, 0u, 0u, 0u);
-      if (t == 0) colsum[pr] = 0;
-    }
-  };
-  if (!early) zero_outputs();
+  const int nc = (K + 4095) >> 12;                          // chunks of the row
+  const int m = (int)blockIdx.x / nc, c = (int)blockIdx.x % nc;   // c: rank in the cluster
+  const int kb = c << 12;
+  const int C = K - kb < 4096 ? K - kb : 4096;              // a multiple of n_h
   const uint16_t* xrow = X + (size_t)m * K;
   float mx = 0.0f;
-  for (int kb = 0; kb < K; kb += 4096) {
-    const int C = K - kb < 4096 ? K - kb : 4096;   // a multiple of 256
-    float* chunk = s_row + kb;
-    if (8 * t < C) {
-      const int k0 = kb + 8 * t;
-      float y[8];
-      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(xrow + k0));
-      const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
+  if (8 * t < C) {
+    const int k0 = kb + 8 * t;
+    float y[8];
+    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(xrow + k0));
+    const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        y[2 * i] = bf16_lo_to_f32(rw[i]);
-        y[2 * i + 1] = bf16_hi_to_f32(rw[i]);
-      }
-      const uint32_t bits =
-          (uint32_t)(splitmix64_output(seed, (uint64_t)(k0 >> 6)) >> (k0 & 63));
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        y[i] = __uint_as_float(__float_as_uint(y[i]) ^ (((bits >> i) & 1u) << 31));
-      // butterflies (a, b) -> (a + b, a - b), a the lower position
-#pragma unroll
-      for (int h = 1; h < 8; h <<= 1) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          if ((i & h) == 0) {
-            const float a = y[i], c = y[i + h];
-            y[i] = a + c;
-            y[i + h] = a - c;
-          }
-        }
-      }
-#pragma unroll
-      for (int lm = 1; lm < 32; lm <<= 1) {
-        const bool upper = (lane & lm) != 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float o = __shfl_xor_sync(0xffffffffu, y[i], lm);
-          y[i] = upper ? o - y[i] : y[i] + o;
-        }
-      }
-      *reinterpret_cast<float4*>(chunk + 8 * t) = make_float4(y[0], y[1], y[2], y[3]);
-      *reinterpret_cast<float4*>(chunk + 8 * t + 4) = make_float4(y[4], y[5], y[6], y[7]);
+    for (int i = 0; i < 4; ++i) {
+      y[2 * i] = bf16_lo_to_f32(rw[i]);
+      y[2 * i + 1] = bf16_hi_to_f32(rw[i]);
     }
-    if (nh > 256) {
-      __syncthreads();
-      // stages across warps: h = 256 .. nh/2 on the positions g + 256 i
-      const int g = t >> 1, half = t & 1;
-      const int nw = C >> 8;                 // 256-position slices in the chunk
-      float y[8];
+    const uint32_t bits = (uint32_t)(splitmix64_output(seed, (uint64_t)(k0 >> 6)) >> (k0 & 63));
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int i = 8 * half + j;
-        y[j] = i < nw ? chunk[g + 256 * i] : 0.0f;
-      }
+    for (int i = 0; i < 8; ++i)
+      y[i] = __uint_as_float(__float_as_uint(y[i]) ^ (((bits >> i) & 1u) << 31));
+    // butterflies (a, b) -> (a + b, a - b), a the lower position
 #pragma unroll
-      for (int h = 1; h < 8; h <<= 1) {
-        if (256 * h < nh) {
+    for (int h = 1; h < 8; h <<= 1) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            if ((j & h) == 0) {
-              const float a = y[j], c = y[j + h];
-              y[j] = a + c;
-              y[j + h] = a - c;
-            }
-          }
+      for (int i = 0; i < 8; ++i) {
+        if ((i & h) == 0) {
+          const float a = y[i], d = y[i + h];
+          y[i] = a + d;
+          y[i + h] = a - d;
         }
       }
-      if (nh > 2048) {
+    }
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float o = __shfl_xor_sync(0xffffffffu, y[j], 1);
-          y[j] = half ? o - y[j] : y[j] + o;
-        }
+    for (int lm = 1; lm < 32; lm <<= 1) {
+      const bool upper = (lane & lm) != 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float o = __shfl_xor_sync(0xffffffffu, y[i], lm);
+        y[i] = upper ? o - y[i] : y[i] + o;
       }
+    }
+    *reinterpret_cast<float4*>(chunk + 8 * t) = make_float4(y[0], y[1], y[2], y[3]);
+    *reinterpret_cast<float4*>(chunk + 8 * t + 4) = make_float4(y[4], y[5], y[6], y[7]);
+    if (nh <= 256) {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int i = 8 * half + j;
-        if (i < nw) {
-          chunk[g + 256 * i] = y[j];
-          mx = fmaxf(mx, fabsf(y[j]));
-        }
-      }
-    } else if (8 * t < C) {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) mx = fmaxf(mx, fabsf(chunk[8 * t + j]));
+      for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(y[i]));
     }
   }
-  // largest magnitude of the row
+  if (nh > 256) {
+    __syncthreads();
+    // stages across warps: h = 256 .. nh/2 on the positions g + 256 i
+    const int g = t >> 1, half = t & 1;
+    const int nw = C >> 8;                 // 256-position slices in the chunk
+    float y[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int i = 8 * half + j;
+      y[j] = i < nw ? chunk[g + 256 * i] : 0.0f;
+    }
+#pragma unroll
+    for (int h = 1; h < 8; h <<= 1) {
+      if (256 * h < nh) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if ((j & h) == 0) {
+            const float a = y[j], d = y[j + h];
+            y[j] = a + d;
+            y[j + h] = a - d;
+          }
+        }
+      }
+    }
+    if (nh > 2048) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float o = __shfl_xor_sync(0xffffffffu, y[j], 1);
+        y[j] = half ? o - y[j] : y[j] + o;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int i = 8 * half + j;
+      if (i < nw) {
+        chunk[g + 256 * i] = y[j];
+        mx = fmaxf(mx, fabsf(y[j]));
+      }
+    }
+  }
+  // largest magnitude of the chunk, then of the row
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
   if (lane == 0) s_max[warp] = mx;
   __syncthreads();
-  float amax = 0.0f;
+  if (t == 0) {
+    float a = 0.0f;
 #pragma unroll
-  for (int w = 0; w < 16; ++w) amax = fmaxf(amax, s_max[w]);
+    for (int w = 0; w < 16; ++w) a = fmaxf(a, s_max[w]);
+    s_cmax = a;
+    if (nc == 1) s_amax = a;
+  }
+  if (nc > 1) {
+    // every CTA of the row publishes its maximum before any reads one
+    cluster_arrive();
+    cluster_wait();
+    if (warp == 0) {
+      float a = lane < nc ? ld_shared_cluster_f32(mapa_shared(smem_u32(&s_cmax), (uint32_t)lane))
+                          : 0.0f;
+#pragma unroll
+      for (int off = 4; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
+      if (lane == 0) s_amax = a;
+    }
+  }
+  __syncthreads();
+  const float amax = s_amax;
   const float step = amax > 0.0f ? amax / 127.0f : 1.0f;
   const float inv = 1.0f / step;
   int sum0 = 0, sum1 = 0;
-  int8_t* q0row = Xq + (size_t)(2 * m) * K;
-  int8_t* q1row = Xq + (size_t)(2 * m + 1) * K;
-  uint2 e0 = make_uint2(0u, 0u), e1 = make_uint2(0u, 0u);   // early: this thread's bytes
-  for (int k = 8 * t; k < K; k += 8 * 512) {
-    const float4 xa = *reinterpret_cast<const float4*>(s_row + k);
-    const float4 xb = *reinterpret_cast<const float4*>(s_row + k + 4);
+  uint2 e0 = make_uint2(0u, 0u), e1 = make_uint2(0u, 0u);   // this thread's bytes
+  if (8 * t < C) {
+    const float4 xa = *reinterpret_cast<const float4*>(chunk + 8 * t);
+    const float4 xb = *reinterpret_cast<const float4*>(chunk + 8 * t + 4);
     const float xs[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
     uint32_t p0[2] = {0u, 0u}, p1[2] = {0u, 0u};
 #pragma unroll
@@ -425,13 +424,8 @@ __global__ void __launch_bounds__(512, 4) k_act_q8(const uint16_t* __restrict__ 
       p0[i >> 2] |= (uint32_t)(ia & 0xFF) << (8 * (i & 3));
       p1[i >> 2] |= (uint32_t)(ib & 0xFF) << (8 * (i & 3));
     }
-    if (early) {
-      e0 = make_uint2(p0[0], p0[1]);
-      e1 = make_uint2(p1[0], p1[1]);
-    } else {
-      *reinterpret_cast<uint2*>(q0row + k) = make_uint2(p0[0], p0[1]);
-      *reinterpret_cast<uint2*>(q1row + k) = make_uint2(p1[0], p1[1]);
-    }
+    e0 = make_uint2(p0[0], p0[1]);
+    e1 = make_uint2(p1[0], p1[1]);
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) {
@@ -443,21 +437,69 @@ __global__ void __launch_bounds__(512, 4) k_act_q8(const uint16_t* __restrict__ 
     s_sum[1][warp] = sum1;
   }
   __syncthreads();
-  if (early) {
-    grid_dep_wait();
-    zero_outputs();
-    if (8 * t < K) {
-      *reinterpret_cast<uint2*>(q0row + 8 * t) = e0;
-      *reinterpret_cast<uint2*>(q1row + 8 * t) = e1;
-    }
-  }
-  if (t < 32) {
+  // piece sums of the chunk (lanes 0 / 16 of warp 0 hold q0's / q1's), then
+  // of the row, in thread 0 of the cluster's first CTA
+  int tot0 = 0, tot1 = 0;
+  if (warp == 0) {
     int a = lane < 16 ? s_sum[0][lane] : s_sum[1][lane - 16];
 #pragma unroll
     for (int off = 8; off > 0; off >>= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
-    if (lane == 0) colsum[2 * m] = a;
-    if (lane == 16) colsum[2 * m + 1] = a;
-    if (lane == 0) scales[m] = step;
+    tot0 = __shfl_sync(0xffffffffu, a, 0);
+    tot1 = __shfl_sync(0xffffffffu, a, 16);
+    if (lane == 0) {
+      s_csum[0] = tot0;
+      s_csum[1] = tot1;
+    }
+  }
+  if (nc > 1) {
+    cluster_arrive();
+    cluster_wait();
+    if (c == 0 && warp == 0) {
+      const uint32_t r = (uint32_t)(lane & 7);
+      int a = lane < nc ? (int)ld_shared_cluster_u32(mapa_shared(smem_u32(&s_csum[0]), r)) : 0;
+      int b = lane < nc ? (int)ld_shared_cluster_u32(mapa_shared(smem_u32(&s_csum[1]), r)) : 0;
+#pragma unroll
+      for (int off = 4; off > 0; off >>= 1) {
+        a += __shfl_xor_sync(0xffffffffu, a, off);
+        b += __shfl_xor_sync(0xffffffffu, b, off);
+      }
+      tot0 = a;
+      tot1 = b;
+    }
+    // no CTA of the row leaves while the first one may still read its sums
+    cluster_arrive();
+    cluster_wait();
+  }
+  // the stores wait for the preceding kernel, which may still read Xq, the
+  // steps, the sums and Y
+  grid_dep_wait();
+  if (Yz) {
+    // the output that the following GEMM accumulates into starts at zero
+    const int64_t nb = gridDim.x;
+    const int64_t per = ((yz_elems + nb - 1) / nb + 3) & ~int64_t(3);
+    const int64_t z0 = (int64_t)blockIdx.x * per, z1 = z0 + per < yz_elems ? z0 + per : yz_elems;
+    for (int64_t i = z0 + 4 * t; i < z1; i += 4 * blockDim.x) {
+      if (i + 4 <= z1) {
+        *reinterpret_cast<float4*>(Yz + i) = make_float4(0.f, 0.f, 0.f, 0.f);
+      } else {
+        for (int64_t j = i; j < z1; ++j) Yz[j] = 0.0f;
+      }
+    }
+  }
+  // padding rows 2M .. rows-1: zero bytes, zero sums
+  for (int pr = 2 * M + m; pr < rows; pr += M) {
+    for (int k = 16 * t; k < C; k += 16 * 512)
+      *reinterpret_cast<uint4*>(Xq + (size_t)pr * K + kb + k) = make_uint4(0u, 0u, 0u, 0u);
+    if (c == 0 && t == 0) colsum[pr] = 0;
+  }
+  if (8 * t < C) {
+    *reinterpret_cast<uint2*>(Xq + (size_t)(2 * m) * K + kb + 8 * t) = e0;
+    *reinterpret_cast<uint2*>(Xq + (size_t)(2 * m + 1) * K + kb + 8 * t) = e1;
+  }
+  if (c == 0 && t == 0) {
+    colsum[2 * m] = tot0;
+    colsum[2 * m + 1] = tot1;
+    scales[m] = step;
   }
 }
 
@@ -467,21 +509,26 @@ cudaError_t launch_act_q8(const uint16_t* X, int64_t M, int64_t K, uint64_t seed
   const int nh = (int)hadamard_block(K);
   if (nh < 256 || nh > 4096 || K > 32768 || M < 1 || M > 32 || rows < 2 * M || rows > 64)
     return cudaErrorInvalidValue;
-  const size_t smem = (size_t)K * sizeof(float);
+  const int nc = (int)((K + 4095) / 4096);
+  const size_t smem = (size_t)(K < 4096 ? K : 4096) * sizeof(float);
   // the same shared-memory carveout as the GEMM that follows, so that the two
   // can share an SM (an SM runs CTAs of one carveout at a time)
   cudaError_t e = ensure_smem_limit(k_act_q8, kMaxDynSmem, true);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)M);
+  cfg.gridDim = dim3((unsigned)(M * nc));
   cfg.blockDim = dim3(512);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = (unsigned)nc;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = nc > 1 ? 2 : 1;
   e = cudaLaunchKernelEx(&cfg, k_act_q8, X, (int)M, (int)K, nh, seed, Xq, scales, colsum,
                          (int)rows, Yz, yz_elems);
   if (e != cudaSuccess) return e;

@@ -137,7 +137,7 @@ int e8_act_rht(const uint16_t* X, int64_t M, int64_t K, uint64_t rht_seed, uint1
  * when N is not a multiple of 4): the last bits of Y can differ between runs.
  * workspace: at least e8_workspace_bytes(mode, M, N, K, bpw) bytes.
  * Ordering: the int8 path launches its kernels with programmatic dependent
- * launch; its kernels may read X (K <= 4096), idx1, idx2 and the codebook
+ * launch; its kernels may read X, idx1, idx2 and the codebook
  * before the kernel that precedes the call on the stream has finished, if
  * that kernel releases its dependents early (griddepcontrol.launch_dependents).
  * Kernels that do not release early (every kernel of this library that writes

@@ -155,6 +155,37 @@ def test_act_gemm_repeatable(gcb):
     assert e8.e8_sync_status(gcb) == e8.E8_OK
 
 
+def test_gemm_chain_mixed_depth_shared_workspace(gcb):
+    # products of different depths queued back to back on one stream with one
+    # workspace, three times over: the activation transform of each call runs
+    # before the GEMM of the previous call has finished and stores only after
+    import torch
+    M = 16
+    shapes = [(520, 14336, 4), (1024, 4096, 4), (264, 14336, 3), (512, 30720, 2),
+              (1024, 4096, 2), (136, 4352, 4)]
+    ws = torch.empty(max(e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT, M, N, K, b)
+                         for N, K, b in shapes), dtype=torch.uint8, device=gu.dev())
+    cases = []
+    for j, (N, K, bpw) in enumerate(shapes):
+        W = synth.gaussian_weights(N, K, 0.02, 3000 + j)
+        s = synth.suggest_scale(W, bpw)
+        i1, i2 = _layer_codes(gcb, W, bpw, 11 + j, s)
+        X = synth.activations_bf16(M, K, 4000 + j)
+        Y = torch.full((M, N), float("nan"), dtype=torch.float32, device=gu.dev())
+        cases.append((N, K, bpw, s, i1, i2, X, gu.bf16_dev(X), Y))
+    st = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    for _ in range(3):
+        for j, (N, K, bpw, s, i1, i2, X, Xd, Y) in enumerate(cases):
+            e8.e8_gemm(gcb, Xd, i1, i2, N, K, bpw, 11 + j, s, mode=e8.E8_GEMM_ACT_RHT, Y=Y,
+                       workspace=ws, stream=st)
+    torch.cuda.synchronize()
+    assert e8.e8_sync_status(gcb) == e8.E8_OK
+    for j, (N, K, bpw, s, i1, i2, X, Xd, Y) in enumerate(cases):
+        wd = orc.decode(gu.to_np(i1), None if i2 is None else gu.to_np(i2), N, K, bpw, 11 + j, s)
+        _check(gu.to_np(Y), orc.gemm(X, wd), e8.E8_GEMM_ACT_RHT)
+
+
 def test_gemm_xt_matches_gemm_and_graph_capture(gcb):
     import torch
     wl = synth.workloads()["llama_4096_b4"]
@@ -192,7 +223,8 @@ def test_gemm_xt_matches_gemm_and_graph_capture(gcb):
     assert e8.e8_sync_status(gcb) == e8.E8_OK
 
 
-@pytest.mark.parametrize("M,K", [(16, 4096), (3, 3072), (32, 256), (1, 12288)])
+@pytest.mark.parametrize("M,K", [(16, 4096), (3, 3072), (32, 256), (1, 12288), (5, 14336),
+                                 (7, 4352), (2, 20480), (3, 30720), (32, 14336)])
 def test_act_rht_q8_pieces(gcb, M, K):
     # xt = s_m (q0 + q1 / 128) within s_m / 256, s_m = max|xt| / 127, column sums
     X = synth.activations_bf16(M, K, 40 + M)
