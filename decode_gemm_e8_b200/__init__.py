@@ -28,7 +28,8 @@ E8_OP_ENCODE = 100
 EXPORTED = ("e8_codebook_build", "e8_codebook_free", "e8_codebook_export", "e8_rht_forward",
             "e8_encode", "e8_decode_to_bf16", "e8_act_rht", "e8_act_rht_q8", "e8_act_q8_bytes",
             "e8_gemm", "e8_gemm_xt",
-            "e8_gemm_xt_rows", "e8_gemm_act_noalloc", "e8_gemm_auto_mode",
+            "e8_gemm_xt_rows", "e8_gemm_act_noalloc", "e8_gemm_host",
+            "e8_gemm_host_workspace_bytes", "e8_gemm_auto_mode",
             "e8_workspace_bytes", "e8_sync_status", "e8_debug_wait_timeout", "e8_status_str",
             "e8_version")
 
@@ -67,6 +68,9 @@ def load_library(path: str = LIB_PATH):
         "e8_gemm_xt_rows": ([I64], c.c_int),
         "e8_gemm_act_noalloc": ([P, P, I64, P, P, I64, I64, c.c_int, U64, c.c_float, P, P],
                                 c.c_int),
+        "e8_gemm_host": ([P, P, I64, P, P, I64, I64, c.c_int, U64, c.c_float, P, c.c_int, P,
+                          c.c_size_t, P], c.c_int),
+        "e8_gemm_host_workspace_bytes": ([c.c_int, I64, I64, I64, c.c_int], c.c_size_t),
         "e8_gemm_auto_mode": ([I64, I64, I64, c.c_int], c.c_int),
         "e8_workspace_bytes": ([c.c_int, I64, I64, I64, c.c_int], c.c_size_t),
         "e8_sync_status": ([P, P], c.c_int),
@@ -233,6 +237,38 @@ def e8_gemm(cb: Codebook, X, idx1, idx2, N: int, K: int, bpw: int, rht_seed: int
                                   int(rht_seed) & (2**64 - 1), float(scale), _ptr(Y), int(mode),
                                   _ptr(ws), ws.numel(), _stream(stream)), "e8_gemm")
     return Y
+
+
+def e8_gemm_host_workspace_bytes(mode: int, M: int, N: int, K: int, bpw: int) -> int:
+    return int(load_library().e8_gemm_host_workspace_bytes(int(mode), int(M), int(N), int(K),
+                                                           int(bpw)))
+
+
+def _host_ptr(a):
+    # torch CPU tensor or numpy array
+    return a.data_ptr() if hasattr(a, "data_ptr") else a.ctypes.data
+
+
+def e8_gemm_host(cb: Codebook, X_host, idx1, idx2, N: int, K: int, bpw: int, rht_seed: int,
+                 scale: float, Y_host=None, mode: int = E8_GEMM_AUTO, workspace=None,
+                 stream=None):
+    """e8_gemm with X (bf16 [M, K]) and Y (fp32 [M, N]) in host memory.
+
+    One library call queues the copy of X in, the product and the copy of Y
+    out on the stream; Y_host holds the product once the stream has passed it.
+    X_host: a torch bf16/int16 CPU tensor or a numpy uint16/int16 array.
+    A new page-locked Y_host is made when None is given."""
+    import torch
+    M = X_host.shape[0]
+    if Y_host is None:
+        Y_host = torch.empty((M, N), dtype=torch.float32).pin_memory()
+    ws = workspace if workspace is not None else _workspace(
+        e8_gemm_host_workspace_bytes(mode, M, N, K, bpw), torch.device("cuda", cb.device))
+    _check(load_library().e8_gemm_host(cb.handle, _host_ptr(X_host), M, _ptr(idx1), _ptr(idx2),
+                                       N, K, int(bpw), int(rht_seed) & (2**64 - 1), float(scale),
+                                       _host_ptr(Y_host), int(mode), _ptr(ws), ws.numel(),
+                                       _stream(stream)), "e8_gemm_host")
+    return Y_host
 
 
 def e8_gemm_xt_rows(M: int) -> int:

@@ -199,6 +199,27 @@ int e8_gemm_act_noalloc(const e8_codebook* cb, const uint16_t* X, int64_t M,
                         const uint16_t* idx1, const void* idx2, int64_t N, int64_t K, int bpw,
                         uint64_t rht_seed, float scale, float* Y, void* stream);
 
+/* e8_gemm with X and Y in host memory: one call queues, on `stream`, the copy
+ * of X (bf16 [M][K], host) into the workspace, the product of e8_gemm in mode
+ * `mode` into a device copy of Y, and the copy of that Y (fp32 [M][N]) back
+ * to Y_host.  Nothing is waited for: Y_host holds the product once the stream
+ * has passed this call.  Page-locked host buffers (cudaHostAlloc /
+ * cudaHostRegister) make both copies asynchronous; with pageable memory the
+ * CUDA runtime stages them and the call may block until they are done.
+ * Arguments are those of e8_gemm; X_host and Y_host must be 16-byte aligned
+ * and may not overlap.  workspace: at least
+ * e8_gemm_host_workspace_bytes(mode, M, N, K, bpw) bytes of device memory,
+ * laid out as [X copy][Y copy][the workspace of e8_gemm], each part on a
+ * 256-byte boundary; it must not be used by other work until the stream
+ * passes this call.  Errors as e8_gemm (E8_ECUDA also for a failed copy). */
+int e8_gemm_host(const e8_codebook* cb, const uint16_t* X_host, int64_t M, const uint16_t* idx1,
+                 const void* idx2, int64_t N, int64_t K, int bpw, uint64_t rht_seed,
+                 float scale, float* Y_host, int mode, void* workspace, size_t ws_bytes,
+                 void* stream);
+
+/* Workspace bytes for e8_gemm_host; 0 if the arguments are invalid. */
+size_t e8_gemm_host_workspace_bytes(int mode, int64_t M, int64_t N, int64_t K, int bpw);
+
 /* Mode that E8_GEMM_AUTO selects for these sizes. */
 int e8_gemm_auto_mode(int64_t M, int64_t N, int64_t K, int bpw);
 

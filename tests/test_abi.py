@@ -63,6 +63,24 @@ def test_workspace_sizes(lib):
     assert e8.e8_workspace_bytes(e8.E8_OP_ENCODE, 0, N, 65536, 2) == 0
 
 
+def test_host_call_workspace_sizes(lib):
+    # [X copy][Y copy][the workspace of e8_gemm], each part on 256 bytes
+    M, N, K = 16, 4096, 4096
+    inner = e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT, M, N, K, 4)
+    assert e8.e8_gemm_host_workspace_bytes(e8.E8_GEMM_ACT_RHT, M, N, K, 4) == \
+        M * K * 2 + M * N * 4 + inner
+    assert e8.e8_gemm_host_workspace_bytes(e8.E8_GEMM_AUTO, M, N, K, 4) == \
+        M * K * 2 + M * N * 4 + inner
+    # ragged sizes round each part up to 256 bytes
+    assert e8.e8_gemm_host_workspace_bytes(e8.E8_GEMM_DECODED_W, 3, 100, 264, 2) == \
+        1792 + 1280 + e8.e8_workspace_bytes(e8.E8_GEMM_DECODED_W, 3, 100, 264, 2)
+    assert 3 * 264 * 2 <= 1792 < 3 * 264 * 2 + 256 and 3 * 100 * 4 <= 1280 < 3 * 100 * 4 + 256
+    # invalid arguments give 0
+    assert e8.e8_gemm_host_workspace_bytes(e8.E8_GEMM_ACT_RHT, 0, N, K, 4) == 0
+    assert e8.e8_gemm_host_workspace_bytes(7, M, N, K, 4) == 0
+    assert e8.e8_gemm_host_workspace_bytes(e8.E8_GEMM_ACT_RHT, M, N, 100, 4) == 0
+
+
 def test_auto_mode(lib):
     assert e8.e8_gemm_auto_mode(16, 4096, 4096, 4) == e8.E8_GEMM_ACT_RHT
     assert e8.e8_gemm_auto_mode(64, 4096, 4096, 4) == e8.E8_GEMM_ACT_RHT

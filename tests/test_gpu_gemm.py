@@ -186,6 +186,41 @@ def test_gemm_chain_mixed_depth_shared_workspace(gcb):
         _check(gu.to_np(Y), orc.gemm(X, wd), e8.E8_GEMM_ACT_RHT)
 
 
+@pytest.mark.parametrize("pinned", [True, False])
+@pytest.mark.parametrize("mode", [e8.E8_GEMM_ACT_RHT, e8.E8_GEMM_DECODED_W])
+def test_gemm_host_buffers(gcb, pinned, mode):
+    # one call copies X in, multiplies and copies Y out; the result is that of
+    # e8_gemm on device copies of the same inputs
+    import torch
+    M, N, K, bpw, rs = 16, 520, 3072, 3, 21
+    W = synth.gaussian_weights(N, K, 0.02, 77)
+    s = synth.suggest_scale(W, bpw)
+    i1, i2 = _layer_codes(gcb, W, bpw, rs, s)
+    X = synth.activations_bf16(M, K, 78)
+    Xh = torch.from_numpy(X.view(np.int16).copy())
+    Yh = torch.full((M, N), float("nan"), dtype=torch.float32)
+    if pinned:
+        Xh, Yh = Xh.pin_memory(), Yh.pin_memory()
+    ref = gu.to_np(e8.e8_gemm(gcb, gu.bf16_dev(X), i1, i2, N, K, bpw, rs, s, mode=mode))
+    st = torch.cuda.Stream()
+    out = e8.e8_gemm_host(gcb, Xh, i1, i2, N, K, bpw, rs, s, Y_host=Yh, mode=mode, stream=st)
+    st.synchronize()
+    assert out is Yh
+    assert e8.e8_sync_status(gcb) == e8.E8_OK
+    # N = 520 is not a multiple of 4: in the int8 path the 24 partial sums of
+    # an output (one per 128-wide K unit) are added by fp32 atomics in arrival
+    # order, so two runs differ by a few rounding steps of the partial sums
+    assert gu.rel_fro(Yh.numpy(), ref) < (2e-5 if mode == e8.E8_GEMM_ACT_RHT else REPEAT)
+    wd = orc.decode(gu.to_np(i1), gu.to_np(i2), N, K, bpw, rs, s)
+    _check(Yh.numpy().astype(np.float64), orc.gemm(X, wd), mode)
+    # a workspace one byte short is refused before anything is queued
+    need = e8.e8_gemm_host_workspace_bytes(mode, M, N, K, bpw)
+    small = torch.empty(need - 1, dtype=torch.uint8, device=gu.dev())
+    with pytest.raises(e8.E8Error) as ei:
+        e8.e8_gemm_host(gcb, Xh, i1, i2, N, K, bpw, rs, s, Y_host=Yh, mode=mode, workspace=small)
+    assert ei.value.code == e8.E8_EWORKSPACE
+
+
 def test_gemm_xt_matches_gemm_and_graph_capture(gcb):
     import torch
     wl = synth.workloads()["llama_4096_b4"]
