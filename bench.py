@@ -382,7 +382,7 @@ def run_ours(args):
 
 
 def _traffic_from_profile():
-    """DRAM bytes per launch of k_act_gemm from the committed ncu summary, or None
+    """DRAM bytes per launch of k_gemm_q8 from the committed ncu summary, or None
     when the kernel source changed since the counters were taken."""
     import hashlib
     prof = os.path.join(ROOT, "profiles", "k_gemm_q8_llama4096_m16.md")
