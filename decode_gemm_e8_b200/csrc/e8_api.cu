@@ -420,25 +420,39 @@ int e8_gemm_host(const e8_codebook* cb, const uint16_t* X_host, int64_t M, const
                  const void* idx2, int64_t N, int64_t K, int bpw, uint64_t rht_seed,
                  float scale, float* Y_host, int mode, void* workspace, size_t ws_bytes,
                  void* stream) {
-  (void)cudaGetLastError();  // a failed earlier launch must not be reported here
-  if (M < 0 || N < 0 || !valid_k(K) || !valid_bpw(bpw)) return E8_EINVAL;
+  // every argument is checked before anything is queued (no CUDA call before
+  // the device check)
+  if (!cb || M < 0 || N < 0 || !valid_k(K) || !valid_bpw(bpw) || !(scale > 0.0f) ||
+      !std::isfinite(scale))
+    return E8_EINVAL;
+  if ((bpw == 2) != (idx2 == nullptr)) return E8_EINVAL;
   if (M == 0 || N == 0) return E8_OK;
-  if (!X_host || !Y_host || !aligned16(X_host) || !aligned16(Y_host)) return E8_EINVAL;
+  const int m = mode == E8_GEMM_AUTO ? e8_gemm_auto_mode(M, N, K, bpw) : mode;
+  if (m < E8_GEMM_ACT_RHT || m > E8_GEMM_SIMT) return E8_EINVAL;
+  if ((m == E8_GEMM_ACT_RHT || m == E8_GEMM_ACT_RHT_SMEM) && (M > 64 || (K % 128) != 0))
+    return E8_EINVAL;
+  if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return E8_EINVAL;
+  if (!X_host || !Y_host || !idx1 || !aligned16(X_host) || !aligned16(Y_host) ||
+      !aligned16(idx1) || (idx2 && !aligned16(idx2)))
+    return E8_EINVAL;
   const size_t xb = (size_t)M * (size_t)K * 2, yb = (size_t)M * (size_t)N * 4;
   {
     const uintptr_t x0 = reinterpret_cast<uintptr_t>(X_host), y0 = reinterpret_cast<uintptr_t>(Y_host);
     if (x0 < y0 + yb && y0 < x0 + xb) return E8_EINVAL;
   }
-  const size_t need = e8_gemm_host_workspace_bytes(mode, M, N, K, bpw);
+  const size_t need = e8_gemm_host_workspace_bytes(m, M, N, K, bpw);
   if (need == 0) return E8_EINVAL;
   if (!workspace || !aligned16(workspace) || ws_bytes < need) return E8_EWORKSPACE;
+  (void)cudaGetLastError();  // a failed earlier launch must not be reported here
+  const int dc = check_device(cb);
+  if (dc != E8_OK) return dc;
   uint8_t* w = static_cast<uint8_t*>(workspace);
   uint16_t* Xd = reinterpret_cast<uint16_t*>(w);
   float* Yd = reinterpret_cast<float*>(w + round256(xb));
   uint8_t* inner = w + round256(xb) + round256(yb);
   cudaStream_t st = (cudaStream_t)stream;
   if (cudaMemcpyAsync(Xd, X_host, xb, cudaMemcpyHostToDevice, st) != cudaSuccess) return E8_ECUDA;
-  const int rc = e8_gemm(cb, Xd, M, idx1, idx2, N, K, bpw, rht_seed, scale, Yd, mode, inner,
+  const int rc = e8_gemm(cb, Xd, M, idx1, idx2, N, K, bpw, rht_seed, scale, Yd, m, inner,
                          ws_bytes - round256(xb) - round256(yb), stream);
   if (rc != E8_OK) return rc;
   if (cudaMemcpyAsync(Y_host, Yd, yb, cudaMemcpyDeviceToHost, st) != cudaSuccess) return E8_ECUDA;

@@ -211,7 +211,8 @@ int e8_gemm_act_noalloc(const e8_codebook* cb, const uint16_t* X, int64_t M,
  * e8_gemm_host_workspace_bytes(mode, M, N, K, bpw) bytes of device memory,
  * laid out as [X copy][Y copy][the workspace of e8_gemm], each part on a
  * 256-byte boundary; it must not be used by other work until the stream
- * passes this call.  Errors as e8_gemm (E8_ECUDA also for a failed copy). */
+ * passes this call.  Errors as e8_gemm (E8_ECUDA also for a failed copy);
+ * argument and workspace errors are returned before anything is queued. */
 int e8_gemm_host(const e8_codebook* cb, const uint16_t* X_host, int64_t M, const uint16_t* idx1,
                  const void* idx2, int64_t N, int64_t K, int bpw, uint64_t rht_seed,
                  float scale, float* Y_host, int mode, void* workspace, size_t ws_bytes,

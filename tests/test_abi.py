@@ -81,6 +81,46 @@ def test_host_call_workspace_sizes(lib):
     assert e8.e8_gemm_host_workspace_bytes(e8.E8_GEMM_ACT_RHT, M, N, 100, 4) == 0
 
 
+def test_host_call_refuses_bad_arguments_before_any_cuda_call(lib):
+    # e8_gemm_host checks every argument and the workspace size before its
+    # first CUDA call (this host has no GPU: a CUDA call would answer
+    # E8_ECUDA).  The codebook and device addresses below are stand-ins that
+    # these paths never dereference.
+    import numpy as np
+    X = np.zeros((16, 4096), np.uint16)
+    Y = np.zeros((16, 4096), np.float32)
+    cb, dev = 1 << 20, 1 << 24
+
+    def call(M=16, N=4096, K=4096, bpw=4, scale=0.02, x=None, y=None, i1=dev, i2=dev + 4096,
+             mode=e8.E8_GEMM_ACT_RHT, ws=dev + 8192, wsb=None, cbp=cb):
+        x = X.ctypes.data if x is None else x
+        y = Y.ctypes.data if y is None else y
+        if wsb is None:
+            wsb = e8.e8_gemm_host_workspace_bytes(mode, M, N, K, bpw)
+        return lib.e8_gemm_host(cbp, x, M, i1, i2, N, K, bpw, 5, scale, y, mode, ws, wsb, None)
+
+    assert call(cbp=None) == e8.E8_EINVAL
+    assert call(bpw=5) == e8.E8_EINVAL
+    assert call(K=100) == e8.E8_EINVAL
+    assert call(scale=0.0) == e8.E8_EINVAL
+    assert call(scale=float("nan")) == e8.E8_EINVAL
+    assert call(bpw=2) == e8.E8_EINVAL            # a residual index array at 2 bpw
+    assert call(bpw=3, i2=None) == e8.E8_EINVAL   # none at 3 bpw
+    assert call(mode=9) == e8.E8_EINVAL
+    assert call(M=65) == e8.E8_EINVAL             # the activation path takes M <= 64
+    assert call(x=X.ctypes.data + 2) == e8.E8_EINVAL
+    assert call(i1=dev + 2) == e8.E8_EINVAL
+    assert call(x=0) == e8.E8_EINVAL
+    assert call(y=X.ctypes.data + 64) == e8.E8_EINVAL   # Y overlaps X
+    need = e8.e8_gemm_host_workspace_bytes(e8.E8_GEMM_ACT_RHT, 16, 4096, 4096, 4)
+    assert call(wsb=need - 1) == e8.E8_EWORKSPACE
+    assert call(ws=None) == e8.E8_EWORKSPACE
+    assert call(ws=dev + 8) == e8.E8_EWORKSPACE
+    # nothing to do: no CUDA call either
+    assert call(M=0) == e8.E8_OK
+    assert call(N=0) == e8.E8_OK
+
+
 def test_auto_mode(lib):
     assert e8.e8_gemm_auto_mode(16, 4096, 4096, 4) == e8.E8_GEMM_ACT_RHT
     assert e8.e8_gemm_auto_mode(64, 4096, 4096, 4) == e8.E8_GEMM_ACT_RHT
