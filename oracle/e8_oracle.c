@@ -22,7 +22,7 @@
  *     of vectors whose coordinates are all integers or all half-integers and
  *     whose coordinate sum is even).
  *
- * Readings where the page is silent (each one is listed in the design doc):
+ * Readings where the page is silent:
  *   - the 7 shells are the squared norms 0,2,...,12 (the origin counts);
  *   - canonical order: origin first, then shells by increasing norm; inside a
  *     shell the vectors whose first nonzero coordinate is positive are sorted
@@ -32,7 +32,8 @@
  *     codebook at scale 1/4 (4 bpw), greedy second stage after the first;
  *   - exact Euclidean distances on the fp32 transformed weights, ties to the
  *     smallest index;
- *   - Hadamard block = largest power of two dividing K; sign vector from a
+ *   - Hadamard block = largest power of two dividing K (the *_nh entry points
+ *     take any power-of-two block dividing K instead); sign vector from a
  *     SplitMix64 stream; forward transform in fp32 with stages h = 1,2,4,...
  *     and butterfly (a+b, a-b); decoded weight = bf16_rne(d * fl32(t * alpha)).
  *
@@ -198,11 +199,21 @@ float orc_alpha(float scale, int64_t nh, int bpw) {
   return (float)((double)scale / ((double)m * sqrt((double)nh)));
 }
 
-/* Forward transform of every row: u = fl32(FWHT(D w) * gamma), per block. */
-int orc_rht_forward(const float* W, int64_t N, int64_t K, uint64_t rht_seed,
-                    float scale, float* U, int nthreads) {
-  int64_t nh = orc_hadamard_block(K);
-  if (nh == 0) return -1;
+/* The block size is left open by the pages (glq page, "How it works", item 2:
+ * a randomized Hadamard transform on the input dimension).  The default block
+ * is orc_hadamard_block(K); the *_nh entry points take any power of two n_h,
+ * 8 <= n_h <= ORC_MAX_NH, that divides K (the small-block storage variant uses
+ * n_h = 128 or 256).  Everything else -- signs, normalisation, rounding -- is
+ * the same for every block size. */
+int orc_valid_block(int64_t K, int64_t nh) {
+  if (K <= 0 || (K % 8) != 0 || nh < 8 || nh > ORC_MAX_NH || (nh & (nh - 1)) != 0) return 0;
+  return (K % nh) == 0;
+}
+
+/* Forward transform of every row: u = fl32(FWHT(D w) * gamma), per block of nh. */
+int orc_rht_forward_nh(const float* W, int64_t N, int64_t K, int64_t nh, uint64_t rht_seed,
+                       float scale, float* U, int nthreads) {
+  if (!orc_valid_block(K, nh)) return -1;
   int8_t* d = (int8_t*)malloc((size_t)K);
   if (!d) return -1;
   orc_signs(rht_seed, K, d);
@@ -220,6 +231,13 @@ int orc_rht_forward(const float* W, int64_t N, int64_t K, uint64_t rht_seed,
   (void)nthreads;
   free(d);
   return 0;
+}
+
+int orc_rht_forward(const float* W, int64_t N, int64_t K, uint64_t rht_seed,
+                    float scale, float* U, int nthreads) {
+  int64_t nh = orc_hadamard_block(K);
+  if (nh == 0) return -1;
+  return orc_rht_forward_nh(W, N, K, nh, rht_seed, scale, U, nthreads);
 }
 
 /* ------------------------------------------------------------------------- */
@@ -390,16 +408,24 @@ int orc_nearest_groups(const float* u, int64_t G, int bpw, const int8_t* cb,
   return fail ? -1 : 0;
 }
 
-/* Full encoder: forward RHT of W [N][K] then nearest-point quantisation. */
-int orc_encode(const float* W, int64_t N, int64_t K, int bpw, uint64_t rht_seed,
-               float scale, const int8_t* cb, uint16_t* idx1, void* idx2, int nthreads) {
-  if (orc_hadamard_block(K) == 0) return -1;
+/* Full encoder: forward RHT of W [N][K] (blocks of nh) then nearest-point
+ * quantisation. */
+int orc_encode_nh(const float* W, int64_t N, int64_t K, int64_t nh, int bpw, uint64_t rht_seed,
+                  float scale, const int8_t* cb, uint16_t* idx1, void* idx2, int nthreads) {
+  if (!orc_valid_block(K, nh)) return -1;
   float* U = (float*)malloc(sizeof(float) * (size_t)(N * K));
   if (!U) return -1;
-  int rc = orc_rht_forward(W, N, K, rht_seed, scale, U, nthreads);
+  int rc = orc_rht_forward_nh(W, N, K, nh, rht_seed, scale, U, nthreads);
   if (rc == 0) rc = orc_nearest_groups(U, N * K / 8, bpw, cb, idx1, idx2, nthreads);
   free(U);
   return rc;
+}
+
+int orc_encode(const float* W, int64_t N, int64_t K, int bpw, uint64_t rht_seed,
+               float scale, const int8_t* cb, uint16_t* idx1, void* idx2, int nthreads) {
+  int64_t nh = orc_hadamard_block(K);
+  if (nh == 0) return -1;
+  return orc_encode_nh(W, N, K, nh, bpw, rht_seed, scale, cb, idx1, idx2, nthreads);
 }
 
 /* ------------------------------------------------------------------------- */
@@ -426,12 +452,11 @@ static void orc_group_z(const int8_t* cb, int bpw, int i1, int i2, int64_t* z) {
   }
 }
 
-/* W_dec[n][k] = bf16_rne(d_k * fl32(t_k * alpha)), t = FWHT(z) per block. */
-int orc_decode(const uint16_t* idx1, const void* idx2, int64_t N, int64_t K, int bpw,
-               uint64_t rht_seed, float scale, const int8_t* cb, uint16_t* Wdec,
-               int nthreads) {
-  int64_t nh = orc_hadamard_block(K);
-  if (nh == 0 || bpw < 2 || bpw > 4) return -1;
+/* W_dec[n][k] = bf16_rne(d_k * fl32(t_k * alpha)), t = FWHT(z) per block of nh. */
+int orc_decode_nh(const uint16_t* idx1, const void* idx2, int64_t N, int64_t K, int64_t nh,
+                  int bpw, uint64_t rht_seed, float scale, const int8_t* cb, uint16_t* Wdec,
+                  int nthreads) {
+  if (!orc_valid_block(K, nh) || bpw < 2 || bpw > 4) return -1;
   int8_t* d = (int8_t*)malloc((size_t)K);
   if (!d) return -1;
   orc_signs(rht_seed, K, d);
@@ -472,6 +497,14 @@ int orc_decode(const uint16_t* idx1, const void* idx2, int64_t N, int64_t K, int
   (void)nthreads;
   free(d);
   return fail ? -1 : 0;
+}
+
+int orc_decode(const uint16_t* idx1, const void* idx2, int64_t N, int64_t K, int bpw,
+               uint64_t rht_seed, float scale, const int8_t* cb, uint16_t* Wdec,
+               int nthreads) {
+  int64_t nh = orc_hadamard_block(K);
+  if (nh == 0) return -1;
+  return orc_decode_nh(idx1, idx2, N, K, nh, bpw, rht_seed, scale, cb, Wdec, nthreads);
 }
 
 /* ------------------------------------------------------------------------- */

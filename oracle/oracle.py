@@ -72,6 +72,17 @@ def _load():
     lib.orc_decode.argtypes = [P, P, c.c_int64, c.c_int64, c.c_int, c.c_uint64, c.c_float, P, P,
                                c.c_int]
     lib.orc_decode.restype = c.c_int
+    lib.orc_valid_block.argtypes = [c.c_int64, c.c_int64]
+    lib.orc_valid_block.restype = c.c_int
+    lib.orc_rht_forward_nh.argtypes = [P, c.c_int64, c.c_int64, c.c_int64, c.c_uint64, c.c_float,
+                                       P, c.c_int]
+    lib.orc_rht_forward_nh.restype = c.c_int
+    lib.orc_encode_nh.argtypes = [P, c.c_int64, c.c_int64, c.c_int64, c.c_int, c.c_uint64,
+                                  c.c_float, P, P, P, c.c_int]
+    lib.orc_encode_nh.restype = c.c_int
+    lib.orc_decode_nh.argtypes = [P, P, c.c_int64, c.c_int64, c.c_int64, c.c_int, c.c_uint64,
+                                  c.c_float, P, P, c.c_int]
+    lib.orc_decode_nh.restype = c.c_int
     lib.orc_gemm.argtypes = [P, c.c_int64, P, c.c_int64, c.c_int64, P, c.c_int]
     lib.orc_gemm.restype = c.c_int
     lib.orc_max_threads.argtypes = []
@@ -106,6 +117,11 @@ def hadamard_block(K: int) -> int:
     return int(_load().orc_hadamard_block(K))
 
 
+def valid_block(K: int, nh: int) -> bool:
+    """n_h is a power of two, 8 <= n_h <= 32768, dividing K (K a multiple of 8)."""
+    return bool(_load().orc_valid_block(K, nh))
+
+
 def signs(rht_seed: int, K: int) -> np.ndarray:
     d = np.zeros(K, dtype=np.int8)
     _load().orc_signs(ctypes.c_uint64(rht_seed & (2**64 - 1)), K, _ptr(d))
@@ -120,12 +136,19 @@ def alpha(scale: float, nh: int, bpw: int) -> float:
     return float(_load().orc_alpha(scale, nh, bpw))
 
 
-def rht_forward(W: np.ndarray, rht_seed: int, scale: float, nthreads: int | None = None) -> np.ndarray:
+def rht_forward(W: np.ndarray, rht_seed: int, scale: float, nthreads: int | None = None,
+                nh: int | None = None) -> np.ndarray:
+    """u = fl32(FWHT(D w) * gamma) per row, in Hadamard blocks of the default size
+    (largest power of two dividing K) or of `nh`."""
     W = np.ascontiguousarray(W, dtype=np.float32)
     N, K = W.shape
     U = np.empty_like(W)
-    rc = _load().orc_rht_forward(_ptr(W), N, K, ctypes.c_uint64(rht_seed), scale, _ptr(U),
-                                 threads(nthreads))
+    if nh is None:
+        rc = _load().orc_rht_forward(_ptr(W), N, K, ctypes.c_uint64(rht_seed), scale, _ptr(U),
+                                     threads(nthreads))
+    else:
+        rc = _load().orc_rht_forward_nh(_ptr(W), N, K, nh, ctypes.c_uint64(rht_seed), scale,
+                                        _ptr(U), threads(nthreads))
     if rc != 0:
         raise ValueError("bad shape for the RHT (K=%d)" % K)
     return U
@@ -158,30 +181,41 @@ def nearest_groups(U: np.ndarray, bpw: int, nthreads: int | None = None):
     return i1, i2
 
 
-def encode(W: np.ndarray, bpw: int, rht_seed: int, scale: float, nthreads: int | None = None):
-    """idx1 [N, K/8] uint16 and idx2 [N, K/8] (uint8 for 3 bpw, uint16 for 4 bpw, None for 2)."""
+def encode(W: np.ndarray, bpw: int, rht_seed: int, scale: float, nthreads: int | None = None,
+           nh: int | None = None):
+    """idx1 [N, K/8] uint16 and idx2 [N, K/8] (uint8 for 3 bpw, uint16 for 4 bpw, None for 2).
+    `nh`: Hadamard block size (default: the largest power of two dividing K)."""
     W = np.ascontiguousarray(W, dtype=np.float32)
     N, K = W.shape
     i1 = np.zeros((N, K // 8), dtype=np.uint16)
     i2 = _idx2_alloc(bpw, (N, K // 8))
-    rc = _load().orc_encode(_ptr(W), N, K, bpw, ctypes.c_uint64(rht_seed), scale,
-                            _ptr(codebook()), _ptr(i1), _ptr(i2) if i2 is not None else None,
-                            threads(nthreads))
+    p2 = _ptr(i2) if i2 is not None else None
+    if nh is None:
+        rc = _load().orc_encode(_ptr(W), N, K, bpw, ctypes.c_uint64(rht_seed), scale,
+                                _ptr(codebook()), _ptr(i1), p2, threads(nthreads))
+    else:
+        rc = _load().orc_encode_nh(_ptr(W), N, K, nh, bpw, ctypes.c_uint64(rht_seed), scale,
+                                   _ptr(codebook()), _ptr(i1), p2, threads(nthreads))
     if rc != 0:
         raise ValueError("oracle encode rejected the arguments")
     return i1, i2
 
 
 def decode(idx1: np.ndarray, idx2, N: int, K: int, bpw: int, rht_seed: int, scale: float,
-           nthreads: int | None = None) -> np.ndarray:
-    """Decoded weights as raw bf16 bit patterns, uint16 [N, K]."""
+           nthreads: int | None = None, nh: int | None = None) -> np.ndarray:
+    """Decoded weights as raw bf16 bit patterns, uint16 [N, K].
+    `nh`: Hadamard block size (default: the largest power of two dividing K)."""
     idx1 = np.ascontiguousarray(idx1, dtype=np.uint16)
     if idx2 is not None:
         idx2 = np.ascontiguousarray(idx2, dtype=np.uint8 if bpw == 3 else np.uint16)
     out = np.zeros((N, K), dtype=np.uint16)
-    rc = _load().orc_decode(_ptr(idx1), _ptr(idx2) if idx2 is not None else None, N, K, bpw,
-                            ctypes.c_uint64(rht_seed), scale, _ptr(codebook()), _ptr(out),
-                            threads(nthreads))
+    p2 = _ptr(idx2) if idx2 is not None else None
+    if nh is None:
+        rc = _load().orc_decode(_ptr(idx1), p2, N, K, bpw, ctypes.c_uint64(rht_seed), scale,
+                                _ptr(codebook()), _ptr(out), threads(nthreads))
+    else:
+        rc = _load().orc_decode_nh(_ptr(idx1), p2, N, K, nh, bpw, ctypes.c_uint64(rht_seed),
+                                   scale, _ptr(codebook()), _ptr(out), threads(nthreads))
     if rc != 0:
         raise ValueError("oracle decode rejected the arguments")
     return out
