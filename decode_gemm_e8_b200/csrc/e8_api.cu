@@ -115,10 +115,11 @@ cudaError_t run_act_gemm(const e8_codebook* cb, const uint16_t* X, int64_t M,
 
 namespace {
 
-constexpr int64_t kMaxNh = 32768;
+using e8::aligned16;
+using e8::alpha_of;
+using e8::valid_bpw;
+using e8::valid_k;
 constexpr size_t kTableAlloc = 131088;  // 32769 u32 padded to a multiple of 16 bytes
-
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int check_device(const e8_codebook* cb) {
   if (!cb) return E8_EINVAL;
@@ -127,22 +128,8 @@ int check_device(const e8_codebook* cb) {
   return dev == cb->device ? E8_OK : E8_EDEVICE;
 }
 
-// K: positive multiple of 8 whose Hadamard block is at most 32768.
-bool valid_k(int64_t K) {
-  if (K < 8 || (K % 8) != 0) return false;
-  return e8::hadamard_block(K) <= kMaxNh;
-}
-
-bool valid_bpw(int bpw) { return bpw >= 2 && bpw <= 4; }
-
-int m_of(int bpw) { return bpw == 2 ? 2 : (bpw == 3 ? 4 : 8); }
-
 float gamma_of(float scale, int64_t nh) {
   return (float)(1.0 / ((double)scale * std::sqrt((double)nh)));
-}
-
-float alpha_of(float scale, int64_t nh, int bpw) {
-  return (float)((double)scale / ((double)m_of(bpw) * std::sqrt((double)nh)));
 }
 
 e8::DeviceCodebook dev_view(const e8_codebook* cb) {
@@ -380,7 +367,7 @@ int e8_gemm(const e8_codebook* cb, const uint16_t* X, int64_t M, const uint16_t*
   if (mode == E8_GEMM_AUTO) mode = e8_gemm_auto_mode(M, N, K, bpw);
   if (mode < E8_GEMM_ACT_RHT || mode > E8_GEMM_SIMT) return E8_EINVAL;
   const bool act = mode == E8_GEMM_ACT_RHT || mode == E8_GEMM_ACT_RHT_SMEM;
-  if (act && (M > 64 || (K % 128) != 0)) return E8_EINVAL;
+  if (act && !e8::act_shape_ok(M, K)) return E8_EINVAL;
   if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return E8_EINVAL;
   if (M == 0 || N == 0) return E8_OK;
   if (!X || !idx1 || !Y || !aligned16(X) || !aligned16(idx1) || !aligned16(Y) ||

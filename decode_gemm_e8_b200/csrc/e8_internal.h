@@ -1,10 +1,12 @@
 // Declarations shared between the kernel translation units and the C ABI layer.
 #pragma once
 
+#include <cmath>
 #include <cstdint>
 #include <cuda_runtime.h>
 
 #include "e8_codebook.cuh"
+#include "e8_common.cuh"
 
 // The opaque handle of include/e8.h: device tables of one codebook.
 struct e8_codebook {
@@ -22,6 +24,24 @@ struct e8_codebook {
 };
 
 namespace e8 {
+
+// Argument rules shared by every C entry point (one definition, so that the
+// entry points that must agree -- e8_gemm in E8_GEMM_ACT_RHT and
+// e8_gemm_act_noalloc, for instance -- cannot drift apart).
+constexpr int64_t kMaxNh = 32768;
+// K: positive multiple of 8 whose Hadamard block is at most 32768.
+inline bool valid_k(int64_t K) { return K >= 8 && (K % 8) == 0 && hadamard_block(K) <= kMaxNh; }
+inline bool valid_bpw(int bpw) { return bpw >= 2 && bpw <= 4; }
+inline bool valid_scale(float s) { return s > 0.0f && std::isfinite(s); }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+// Shapes of the activation-side GEMM (E8_GEMM_ACT_RHT and _SMEM).
+inline bool act_shape_ok(int64_t M, int64_t K) { return M <= 64 && (K % 128) == 0; }
+// Integer multiplier of the group vectors: z = m (c1 + beta c2).
+inline int m_of(int bpw) { return bpw == 2 ? 2 : (bpw == 3 ? 4 : 8); }
+// Decode constant alpha = fl32(scale / (m sqrt(n_h))), computed in binary64.
+inline float alpha_of(float scale, int64_t nh, int bpw) {
+  return (float)((double)scale / ((double)m_of(bpw) * std::sqrt((double)nh)));
+}
 
 // One group that the encoder's fast path could not decide exactly.
 struct WorkItem {

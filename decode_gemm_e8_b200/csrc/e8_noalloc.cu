@@ -1,18 +1,18 @@
 // e8_gemm_act_noalloc: the small-batch fused GEMM (E8_GEMM_ACT_RHT) for callers
 // that cannot hand the library a workspace.
 //
-// Some callers are not allowed to allocate device memory at the point where
-// they run the layer: code being captured into a CUDA graph (cudaMalloc is not a
-// capturable call), plugins whose host framework owns every byte of device
-// memory and gives them none at enqueue time, and latency-critical loops where
-// an allocation could synchronise the device.  This entry point keeps its only
-// scratch buffer -- the transformed activations, hi and lo rows -- in a
-// fixed-size array that lives in the library's own device image, so it needs
-// neither a workspace argument nor any allocation.
+// Some callers may not allocate device memory at the point where they run a
+// layer: plugins whose host framework owns every byte of device memory and
+// hands them none when they are enqueued, services that run under a fixed
+// device-memory budget decided at start-up, and latency-critical loops where
+// an allocation could synchronise the device or fail half-way through a
+// request.  This entry point keeps its only scratch buffer -- the transformed
+// activations -- in a fixed-size array that lives in the library's own device
+// image, so it needs neither a workspace argument nor any allocation.
 //
 // Limits and rules (also stated in include/e8.h):
-//   - the scratch is 2 MiB: requests whose activation buffer (the workspace
-//     e8_gemm would need for E8_GEMM_ACT_RHT) is larger return E8_EWORKSPACE
+//   - the scratch is 2 MiB: requests for which e8_workspace_bytes(
+//     E8_GEMM_ACT_RHT, M, N, K, bpw) exceeds 2 MiB return E8_EWORKSPACE
 //     without launching anything;
 //   - every GPU that loads the library keeps this 2 MiB until the process exits;
 //   - all calls share the one array and it keeps the last call's contents; the
@@ -56,8 +56,6 @@ int scratch_address(int dev, uint16_t** out) {
   return E8_OK;
 }
 
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
 }  // namespace
 
 extern "C" int e8_gemm_act_noalloc(const e8_codebook* cb, const uint16_t* X, int64_t M,
@@ -69,24 +67,21 @@ extern "C" int e8_gemm_act_noalloc(const e8_codebook* cb, const uint16_t* X, int
   if (cudaGetDevice(&dev) != cudaSuccess) return E8_ECUDA;
   if (dev != cb->device) return E8_EDEVICE;
   (void)cudaGetLastError();  // an earlier failed launch must not be reported here
-  if (M < 0 || N < 0 || K < 8 || (K % 8) != 0 || bpw < 2 || bpw > 4 || !(scale > 0.0f) ||
-      !std::isfinite(scale))
+  // the argument rules of e8_gemm in mode E8_GEMM_ACT_RHT (shared helpers)
+  if (M < 0 || N < 0 || !e8::valid_k(K) || !e8::valid_bpw(bpw) || !e8::valid_scale(scale))
     return E8_EINVAL;
-  const int64_t nh = e8::hadamard_block(K);
-  if (nh > 32768) return E8_EINVAL;
   if ((bpw == 2) != (idx2 == nullptr)) return E8_EINVAL;
-  if (M > 64 || (K % 128) != 0 || N > INT32_MAX || K > INT32_MAX) return E8_EINVAL;
+  if (!e8::act_shape_ok(M, K) || N > INT32_MAX || K > INT32_MAX) return E8_EINVAL;
   if (M == 0 || N == 0) return E8_OK;
   const size_t need = e8::act_scratch_bytes(M, K, 0);
   if (need > (size_t)kNoallocBytes) return E8_EWORKSPACE;
-  if (!X || !idx1 || !Y || !aligned16(X) || !aligned16(idx1) || !aligned16(Y) ||
-      (idx2 && !aligned16(idx2)))
+  if (!X || !idx1 || !Y || !e8::aligned16(X) || !e8::aligned16(idx1) || !e8::aligned16(Y) ||
+      (idx2 && !e8::aligned16(idx2)))
     return E8_EINVAL;
   uint16_t* xt = nullptr;
   int rc = scratch_address(dev, &xt);
   if (rc != E8_OK) return rc;
-  const int m = bpw == 2 ? 2 : (bpw == 3 ? 4 : 8);
-  const float alpha = (float)((double)scale / ((double)m * std::sqrt((double)nh)));
+  const float alpha = e8::alpha_of(scale, e8::hadamard_block(K), bpw);
   const cudaError_t e = e8::run_act_gemm(cb, X, M, idx1, idx2, N, K, bpw, rht_seed, alpha, Y, 0,
                                          xt, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? E8_OK : E8_ECUDA;

@@ -14,9 +14,11 @@ from dataclasses import dataclass, field
 import numpy as np
 
 # Per-bpw target RMS of the transformed, scaled weights (scale = rms(W) / SIGMA_T).
-# Frozen from a sweep of the oracle's reconstruction MSE on Gaussian rows
-# (oracle/sigma_sweep.py prints the sweep); the scale is an input of the
-# quantiser, so these numbers affect quality only, never parity.
+# Frozen once from the oracle's relative reconstruction MSE (encode -> decode)
+# on 64 x 1024 Gaussian rows, swept over sigma_t = 0.70, 0.75, ..., 1.10 and
+# rounded to the sweep's grid: the minimisers are 1.00, 1.00 and 0.90 for 2, 3
+# and 4 bpw.  The scale is an input of the quantiser, so these numbers affect
+# quality only, never parity.
 SIGMA_T = {2: 1.00, 3: 1.00, 4: 0.90}
 
 

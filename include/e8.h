@@ -112,9 +112,12 @@ int e8_encode(const e8_codebook* cb, const float* W, int64_t N, int64_t K, int b
               uint64_t rht_seed, float scale, uint16_t* idx1, void* idx2, void* workspace,
               size_t ws_bytes, void* stream);
 
-/* Decoder: indices -> bf16 weights W_dec [N][K] (raw bf16 bits), the exact
- * inverse transform followed by the two roundings given at the top of this
- * file, bit-exact.  Needs no workspace. */
+/* Decoder ("How it works", items 1-2; "Bit widths" table): indices -> bf16
+ * weights W_dec [N][K] (raw bf16 bits).  Each group's vector is rebuilt from
+ * the codebook (z = m (c1 + beta c2)), the sign flips and the Walsh-Hadamard
+ * transform are undone exactly, then the two roundings given at the top of
+ * this file are applied; bit-exact.  idx1 / idx2 as e8_encode writes them
+ * (idx2 NULL for bpw 2).  Needs no workspace. */
 int e8_decode_to_bf16(const e8_codebook* cb, const uint16_t* idx1, const void* idx2, int64_t N,
                       int64_t K, int bpw, uint64_t rht_seed, float scale, uint16_t* W_dec,
                       void* stream);
@@ -126,7 +129,9 @@ int e8_decode_to_bf16(const e8_codebook* cb, const uint16_t* idx1, const void* i
 int e8_act_rht(const uint16_t* X, int64_t M, int64_t K, uint64_t rht_seed, uint16_t* Xt,
                int64_t rows, void* stream);
 
-/* GEMM with compressed weights: Y fp32 [M][N] = X bf16 [M][K] * W_dec^T, where
+/* GEMM with compressed weights ("How it works", items 1-2: the weights are
+ * rebuilt from their codebook indices and the inverse transform at run time):
+ * Y fp32 [M][N] = X bf16 [M][K] * W_dec^T, where
  * W_dec is what e8_decode_to_bf16 returns for (idx1, idx2, scale, rht_seed).
  * In the DECODED_W and SIMT modes the product uses W_dec itself; in the
  * ACT_RHT modes it uses the unrounded decoded weights (relative Frobenius
@@ -182,10 +187,12 @@ int e8_gemm_xt(const e8_codebook* cb, const void* xq, int64_t M, const uint16_t*
 int e8_gemm_xt_rows(int64_t M);
 
 /* E8_GEMM_ACT_RHT without a workspace, for callers that may not allocate device
- * memory where they run the layer: code being captured into a CUDA graph,
- * plugins whose host framework owns all device memory, latency-critical loops
- * that cannot risk an allocation synchronising the device.  The paper has no
- * counterpart; this is a deployment convenience of this library.
+ * memory where they run the layer: plugins whose host framework owns all
+ * device memory and hands them none when they are enqueued, services held to
+ * a device-memory budget fixed at start-up, and latency-critical loops that
+ * cannot risk an allocation synchronising the device or failing mid-request.
+ * The paper has no counterpart; this is a deployment convenience of this
+ * library.
  * Same arguments and result as e8_gemm with mode E8_GEMM_ACT_RHT, minus the
  * workspace.  The transformed activations go to a fixed 2 MiB array compiled
  * into the library (every GPU that loads the library holds it until the process
