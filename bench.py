@@ -554,7 +554,9 @@ def _layer_chain_rows(e8, synth, cb, dev, stream, peaks, M=16):
     """The seven projections of one Llama-3-8B-shaped decoder layer (q, k, v, o,
     gate, up, down) through the fused small-batch decode GEMM, back to back in one
     stream (programmatic dependent launch between the calls), M tokens, per rate;
-    two code sets alternate so more than L2 streams from HBM."""
+    two code sets alternate so more than L2 streams from HBM.  Timed twice: seven
+    single-matrix calls, and four calls with q, k, v and gate, up grouped
+    (e8_gemm_grouped: the matrices of a group read the same tokens)."""
     import torch
     rows = {}
     gen = torch.Generator(device=dev)
@@ -576,16 +578,35 @@ def _layer_chain_rows(e8, synth, cb, dev, stream, peaks, M=16):
                 e8.e8_gemm(cb, X, c1, c2, lay.N, lay.K, bpw, lay.rht_seed, 0.02,
                            mode=e8.E8_GEMM_ACT_RHT, Y=Y, workspace=ws, stream=stream)
 
+        # the same layer with the matrices that read the same tokens grouped:
+        # (q, k, v), o, (gate, up), down -- four calls instead of seven
+        groups = [[0, 1, 2], [3], [4, 5], [6]]
+        gws = [torch.empty(max(16, e8.e8_gemm_grouped_workspace_bytes(M, mats[g[0]].K, bpw,
+                                                                      len(g))),
+                           dtype=torch.uint8, device=dev) for g in groups]
+
+        def chain_grouped(i, data=data, bpw=bpw, groups=groups, gws=gws):
+            for g, ws in zip(groups, gws):
+                X = data[g[0]][2]
+                items = []
+                for j in g:
+                    lay, codes, _, Y, _ = data[j]
+                    c1, c2 = codes[i % 2]
+                    items.append((c1, c2, lay.N, lay.rht_seed, 0.02, Y))
+                e8.e8_gemm_grouped(cb, X, items, mats[g[0]].K, bpw, workspace=ws, stream=stream)
+
         n = 200
-        t = _time_graphs(chain, n, 4, stream) / 1e3 / n
         nw = sum(lay.N * lay.K for lay in mats)
         flop = sum(2.0 * M * lay.N * lay.K for lay in mats)
         byt = sum(lay.N * lay.K * bpw / 8 + M * lay.K * 2 + M * lay.N * 4 for lay in mats)
-        rows["gemm_llama3_8b_layer_m%d_b%d" % (M, bpw)] = {
-            "us_per_layer": round(t * 1e6, 1), "TFLOP_s": round(flop / t / 1e12, 2),
-            "decoded_weights_per_s": nw / t, "GB_s": round(byt / t / 1e9, 1),
-            "hbm_frac": round(byt / t / 1e9 / peaks["hbm_gbs"], 4)}
-        del data
+        for name, fn in (("gemm_llama3_8b_layer_m%d_b%d" % (M, bpw), chain),
+                         ("gemm_llama3_8b_layer_m%d_b%d_grouped" % (M, bpw), chain_grouped)):
+            t = _time_graphs(fn, n, 4, stream) / 1e3 / n
+            rows[name] = {
+                "us_per_layer": round(t * 1e6, 1), "TFLOP_s": round(flop / t / 1e12, 2),
+                "decoded_weights_per_s": nw / t, "GB_s": round(byt / t / 1e9, 1),
+                "hbm_frac": round(byt / t / 1e9 / peaks["hbm_gbs"], 4)}
+        del data, gws
     return rows
 
 

@@ -29,6 +29,7 @@ EXPORTED = ("e8_codebook_build", "e8_codebook_free", "e8_codebook_export", "e8_r
             "e8_encode", "e8_decode_to_bf16", "e8_act_rht", "e8_act_rht_q8", "e8_act_q8_bytes",
             "e8_gemm", "e8_gemm_xt",
             "e8_gemm_xt_rows", "e8_gemm_act_noalloc", "e8_gemm_host",
+            "e8_gemm_grouped", "e8_gemm_grouped_workspace_bytes",
             "e8_gemm_host_workspace_bytes", "e8_gemm_auto_mode",
             "e8_workspace_bytes", "e8_sync_status", "e8_debug_wait_timeout", "e8_status_str",
             "e8_version")
@@ -72,6 +73,8 @@ def load_library(path: str = LIB_PATH):
                           c.c_size_t, P], c.c_int),
         "e8_gemm_host_workspace_bytes": ([c.c_int, I64, I64, I64, c.c_int], c.c_size_t),
         "e8_gemm_auto_mode": ([I64, I64, I64, c.c_int], c.c_int),
+        "e8_gemm_grouped": ([P, P, I64, I64, c.c_int, P, c.c_int, P, c.c_size_t, P], c.c_int),
+        "e8_gemm_grouped_workspace_bytes": ([I64, I64, c.c_int, c.c_int], c.c_size_t),
         "e8_workspace_bytes": ([c.c_int, I64, I64, I64, c.c_int], c.c_size_t),
         "e8_sync_status": ([P, P], c.c_int),
         "e8_debug_wait_timeout": ([P, c.c_int, P], c.c_int),
@@ -84,6 +87,16 @@ def load_library(path: str = LIB_PATH):
         f.restype = res
     _lib = lib
     return lib
+
+
+E8_GROUP_MAX = 4
+
+
+class GemmItem(ctypes.Structure):
+    """struct e8_gemm_item of include/e8.h."""
+    _fields_ = [("idx1", ctypes.c_void_p), ("idx2", ctypes.c_void_p), ("N", ctypes.c_int64),
+                ("rht_seed", ctypes.c_uint64), ("scale", ctypes.c_float),
+                ("Y", ctypes.c_void_p)]
 
 
 def status_str(code: int) -> str:
@@ -329,3 +342,34 @@ def e8_debug_wait_timeout(cb: Codebook, wait_ms: int, stream=None) -> None:
 
 def e8_version() -> int:
     return int(load_library().e8_version())
+
+
+def e8_gemm_grouped_workspace_bytes(M: int, K: int, bpw: int, count: int) -> int:
+    return int(load_library().e8_gemm_grouped_workspace_bytes(int(M), int(K), int(bpw),
+                                                              int(count)))
+
+
+def e8_gemm_grouped(cb: Codebook, X, items, K: int, bpw: int, workspace=None, stream=None):
+    """Y_i = X W_dec_i^T for several weight matrices that read the same X.
+
+    items: sequence of (idx1, idx2, N, rht_seed, scale) or
+    (idx1, idx2, N, rht_seed, scale, Y); a missing Y is allocated (fp32 [M, N]).
+    Returns the list of Y tensors."""
+    import torch
+    M = int(X.shape[0])
+    arr = (GemmItem * max(1, len(items)))()
+    outs = []
+    for i, it in enumerate(items):
+        idx1, idx2, N, rs, scale = it[:5]
+        Y = it[5] if len(it) > 5 and it[5] is not None else torch.empty(
+            (M, int(N)), dtype=torch.float32, device=X.device)
+        outs.append(Y)
+        arr[i] = GemmItem(_ptr(idx1), _ptr(idx2), int(N), int(rs), float(scale), _ptr(Y))
+    if workspace is None:
+        workspace = torch.empty(max(16, e8_gemm_grouped_workspace_bytes(M, K, bpw, len(items))),
+                                dtype=torch.uint8, device=X.device)
+    _check(load_library().e8_gemm_grouped(cb.handle, _ptr(X), M, int(K), int(bpw),
+                                          ctypes.cast(arr, ctypes.c_void_p), len(items),
+                                          _ptr(workspace), workspace.numel(), _stream(stream)),
+           "e8_gemm_grouped")
+    return outs

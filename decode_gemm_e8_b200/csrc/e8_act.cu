@@ -265,23 +265,40 @@ namespace e8 {
 // row is written as two int8 pieces
 //   q0 = rint(x / s_m),  q1 = rint((x - q0 s_m) * 128 / s_m),  |q1| <= 64,
 // so x = s_m (q0 + q1 / 128) + e with |e| <= s_m / 256.  Piece rows are
-// interleaved (row 2m = q0, row 2m + 1 = q1); colsum[row] = sum_k Xq[row][k]
-// (the chunks' sums, added by the cluster's first CTA) lets the GEMM remove
-// the +128 bias of its unsigned weight operand exactly.
+// interleaved (row 2m = q0, row 2m + 1 = q1); colsum[u][row] = the sum of
+// Xq[row][k] over the 128 positions k of unit u lets every partial product of
+// the GEMM remove the +128 bias of its unsigned weight operand over its own
+// K range, exactly.
 // Kept small (32 registers, at most 16 KB of shared memory) so that a CTA can
 // share an SM with a CTA of the GEMM that follows it; the transform runs
 // before the wait for the preceding kernel, and only the stores wait for it.
+// Several seeds (a grouped call: one set of outputs per weight matrix) run in
+// one launch: CTA b serves output set b / (M nc), token row (b mod M nc) / nc.
+struct ActQ8Group {
+  int count;
+  uint64_t seed[kMaxGroup];
+  int8_t* Xq[kMaxGroup];
+  float* scales[kMaxGroup];
+  int32_t* colsum[kMaxGroup];
+  float* Yz[kMaxGroup];
+  int64_t yz_elems[kMaxGroup];
+};
+
+// a[g] for a runtime g without dynamic indexing of the parameter array
+template <typename T>
+__device__ __forceinline__ T pick_group(const T (&a)[kMaxGroup], int g) {
+  T r = a[0];
+#pragma unroll
+  for (int j = 1; j < kMaxGroup; ++j)
+    if (g == j) r = a[j];
+  return r;
+}
+
 __global__ void __launch_bounds__(512, 4) k_act_q8(const uint16_t* __restrict__ X, int M, int K,
-                                                   int nh, uint64_t seed,
-                                                   int8_t* __restrict__ Xq,
-                                                   float* __restrict__ scales,
-                                                   int32_t* __restrict__ colsum, int rows,
-                                                   float* __restrict__ Yz, int64_t yz_elems) {
+                                                   int nh, const ActQ8Group grp, int rows) {
   extern __shared__ __align__(16) float chunk[];   // the chunk's positions
   __shared__ float s_max[16];
-  __shared__ int s_sum[2][16];
   __shared__ float s_cmax;     // the chunk's largest magnitude, read by the cluster
-  __shared__ int s_csum[2];    // the chunk's piece sums, read by the cluster's CTA 0
   __shared__ float s_amax;     // the row's largest magnitude
   // the GEMM that follows may start at once: it touches nothing that this
   // kernel or its predecessor writes until its own wait for this grid.  A
@@ -291,7 +308,16 @@ __global__ void __launch_bounds__(512, 4) k_act_q8(const uint16_t* __restrict__ 
   grid_dep_launch();
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int nc = (K + 4095) >> 12;                          // chunks of the row
-  const int m = (int)blockIdx.x / nc, c = (int)blockIdx.x % nc;   // c: rank in the cluster
+  const int per_set = M * nc;                              // CTAs of one output set
+  const int g = (int)blockIdx.x / per_set;
+  const int rem = (int)blockIdx.x - g * per_set;
+  const int m = rem / nc, c = rem % nc;                     // c: rank in the cluster
+  const uint64_t seed = pick_group(grp.seed, g);
+  int8_t* __restrict__ Xq = pick_group(grp.Xq, g);
+  float* __restrict__ scales = pick_group(grp.scales, g);
+  int32_t* __restrict__ colsum = pick_group(grp.colsum, g);
+  float* __restrict__ Yz = pick_group(grp.Yz, g);
+  const int64_t yz_elems = pick_group(grp.yz_elems, g);
   const int kb = c << 12;
   const int C = K - kb < 4096 ? K - kb : 4096;              // a multiple of n_h
   const uint16_t* xrow = X + (size_t)m * K;
@@ -401,6 +427,9 @@ __global__ void __launch_bounds__(512, 4) k_act_q8(const uint16_t* __restrict__ 
       for (int off = 4; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
       if (lane == 0) s_amax = a;
     }
+    // no CTA of the row leaves while another may still read its maximum
+    cluster_arrive();
+    cluster_wait();
   }
   __syncthreads();
   const float amax = s_amax;
@@ -427,57 +456,22 @@ __global__ void __launch_bounds__(512, 4) k_act_q8(const uint16_t* __restrict__ 
     e0 = make_uint2(p0[0], p0[1]);
     e1 = make_uint2(p1[0], p1[1]);
   }
+  // piece sums of every 128-position unit: the 16 threads of a half-warp hold
+  // one unit (positions 128 (t / 16) .. + 127 of the chunk); lanes 0 and 16
+  // end with the sums
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
+  for (int off = 8; off > 0; off >>= 1) {
     sum0 += __shfl_xor_sync(0xffffffffu, sum0, off);
     sum1 += __shfl_xor_sync(0xffffffffu, sum1, off);
-  }
-  if (lane == 0) {
-    s_sum[0][warp] = sum0;
-    s_sum[1][warp] = sum1;
-  }
-  __syncthreads();
-  // piece sums of the chunk (lanes 0 / 16 of warp 0 hold q0's / q1's), then
-  // of the row, in thread 0 of the cluster's first CTA
-  int tot0 = 0, tot1 = 0;
-  if (warp == 0) {
-    int a = lane < 16 ? s_sum[0][lane] : s_sum[1][lane - 16];
-#pragma unroll
-    for (int off = 8; off > 0; off >>= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
-    tot0 = __shfl_sync(0xffffffffu, a, 0);
-    tot1 = __shfl_sync(0xffffffffu, a, 16);
-    if (lane == 0) {
-      s_csum[0] = tot0;
-      s_csum[1] = tot1;
-    }
-  }
-  if (nc > 1) {
-    cluster_arrive();
-    cluster_wait();
-    if (c == 0 && warp == 0) {
-      const uint32_t r = (uint32_t)(lane & 7);
-      int a = lane < nc ? (int)ld_shared_cluster_u32(mapa_shared(smem_u32(&s_csum[0]), r)) : 0;
-      int b = lane < nc ? (int)ld_shared_cluster_u32(mapa_shared(smem_u32(&s_csum[1]), r)) : 0;
-#pragma unroll
-      for (int off = 4; off > 0; off >>= 1) {
-        a += __shfl_xor_sync(0xffffffffu, a, off);
-        b += __shfl_xor_sync(0xffffffffu, b, off);
-      }
-      tot0 = a;
-      tot1 = b;
-    }
-    // no CTA of the row leaves while the first one may still read its sums
-    cluster_arrive();
-    cluster_wait();
   }
   // the stores wait for the preceding kernel, which may still read Xq, the
   // steps, the sums and Y
   grid_dep_wait();
   if (Yz) {
     // the output that the following GEMM accumulates into starts at zero
-    const int64_t nb = gridDim.x;
+    const int64_t nb = per_set;
     const int64_t per = ((yz_elems + nb - 1) / nb + 3) & ~int64_t(3);
-    const int64_t z0 = (int64_t)blockIdx.x * per, z1 = z0 + per < yz_elems ? z0 + per : yz_elems;
+    const int64_t z0 = (int64_t)rem * per, z1 = z0 + per < yz_elems ? z0 + per : yz_elems;
     for (int64_t i = z0 + 4 * t; i < z1; i += 4 * blockDim.x) {
       if (i + 4 <= z1) {
         *reinterpret_cast<float4*>(Yz + i) = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -487,28 +481,40 @@ __global__ void __launch_bounds__(512, 4) k_act_q8(const uint16_t* __restrict__ 
     }
   }
   // padding rows 2M .. rows-1: zero bytes, zero sums
+  const bool unit_lead = (t & 15) == 0 && 8 * t < C;
+  const size_t unit = (size_t)((kb >> 7) + (t >> 4));     // this half-warp's unit of the row
   for (int pr = 2 * M + m; pr < rows; pr += M) {
     for (int k = 16 * t; k < C; k += 16 * 512)
       *reinterpret_cast<uint4*>(Xq + (size_t)pr * K + kb + k) = make_uint4(0u, 0u, 0u, 0u);
-    if (c == 0 && t == 0) colsum[pr] = 0;
+    if (unit_lead) colsum[unit * rows + pr] = 0;
   }
   if (8 * t < C) {
     *reinterpret_cast<uint2*>(Xq + (size_t)(2 * m) * K + kb + 8 * t) = e0;
     *reinterpret_cast<uint2*>(Xq + (size_t)(2 * m + 1) * K + kb + 8 * t) = e1;
   }
-  if (c == 0 && t == 0) {
-    colsum[2 * m] = tot0;
-    colsum[2 * m + 1] = tot1;
-    scales[m] = step;
+  if (unit_lead) {
+    colsum[unit * rows + 2 * m] = sum0;
+    colsum[unit * rows + 2 * m + 1] = sum1;
   }
+  if (c == 0 && t == 0) scales[m] = step;
 }
 
-cudaError_t launch_act_q8(const uint16_t* X, int64_t M, int64_t K, uint64_t seed, int8_t* Xq,
-                          float* scales, int32_t* colsum, int64_t rows, cudaStream_t st,
-                          int pdl, float* Yz, int64_t yz_elems) {
+cudaError_t launch_act_q8_group(const uint16_t* X, int64_t M, int64_t K, const ActQ8Out* outs,
+                                int count, int64_t rows, cudaStream_t st, int pdl) {
   const int nh = (int)hadamard_block(K);
-  if (nh < 256 || nh > 4096 || K > 32768 || M < 1 || M > 32 || rows < 2 * M || rows > 64)
+  if (nh < 256 || nh > 4096 || K > 32768 || M < 1 || M > 32 || rows < 2 * M || rows > 64 ||
+      count < 1 || count > kMaxGroup)
     return cudaErrorInvalidValue;
+  ActQ8Group grp = {};
+  grp.count = count;
+  for (int g = 0; g < count; ++g) {
+    grp.seed[g] = outs[g].seed;
+    grp.Xq[g] = outs[g].Xq;
+    grp.scales[g] = outs[g].scales;
+    grp.colsum[g] = outs[g].colsum;
+    grp.Yz[g] = outs[g].Yz;
+    grp.yz_elems[g] = outs[g].Yz ? outs[g].yz_elems : 0;
+  }
   const int nc = (int)((K + 4095) / 4096);
   const size_t smem = (size_t)(K < 4096 ? K : 4096) * sizeof(float);
   // the same shared-memory carveout as the GEMM that follows, so that the two
@@ -516,7 +522,7 @@ cudaError_t launch_act_q8(const uint16_t* X, int64_t M, int64_t K, uint64_t seed
   cudaError_t e = ensure_smem_limit(k_act_q8, kMaxDynSmem, true);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(M * nc));
+  cfg.gridDim = dim3((unsigned)(M * nc * count));
   cfg.blockDim = dim3(512);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
@@ -529,10 +535,22 @@ cudaError_t launch_act_q8(const uint16_t* X, int64_t M, int64_t K, uint64_t seed
   attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = nc > 1 ? 2 : 1;
-  e = cudaLaunchKernelEx(&cfg, k_act_q8, X, (int)M, (int)K, nh, seed, Xq, scales, colsum,
-                         (int)rows, Yz, yz_elems);
+  e = cudaLaunchKernelEx(&cfg, k_act_q8, X, (int)M, (int)K, nh, grp, (int)rows);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+cudaError_t launch_act_q8(const uint16_t* X, int64_t M, int64_t K, uint64_t seed, int8_t* Xq,
+                          float* scales, int32_t* colsum, int64_t rows, cudaStream_t st,
+                          int pdl, float* Yz, int64_t yz_elems) {
+  ActQ8Out o;
+  o.seed = seed;
+  o.Xq = Xq;
+  o.scales = scales;
+  o.colsum = colsum;
+  o.Yz = Yz;
+  o.yz_elems = yz_elems;
+  return launch_act_q8_group(X, M, K, &o, 1, rows, st, pdl);
 }
 
 }  // namespace e8

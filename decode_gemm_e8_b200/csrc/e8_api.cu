@@ -506,6 +506,76 @@ int e8_gemm_xt(const e8_codebook* cb, const void* xq, int64_t M, const uint16_t*
 
 int e8_gemm_xt_rows(int64_t M) { return M < 0 ? 0 : rows_b_for(M); }
 
+size_t e8_gemm_grouped_workspace_bytes(int64_t M, int64_t K, int bpw, int count) {
+  if (M < 1 || !valid_k(K) || !valid_bpw(bpw) || count < 1 || count > E8_GROUP_MAX ||
+      !e8::q8_eligible(M, K))
+    return 0;
+  return (size_t)count * e8::q8_layout(M, K, rows_b_for(M)).total;
+}
+
+int e8_gemm_grouped(const e8_codebook* cb, const uint16_t* X, int64_t M, int64_t K, int bpw,
+                    const e8_gemm_item* items, int count, void* workspace, size_t ws_bytes,
+                    void* stream) {
+  // every argument and the workspace are checked before the first CUDA call
+  if (!cb || !items || count < 1 || count > E8_GROUP_MAX || M < 0 || !valid_k(K) ||
+      !valid_bpw(bpw))
+    return E8_EINVAL;
+  for (int g = 0; g < count; ++g) {
+    const e8_gemm_item& it = items[g];
+    if (it.N < 0 || it.N > INT32_MAX || !e8::valid_scale(it.scale) ||
+        (it.N > 0 && (bpw == 2) != (it.idx2 == nullptr)))
+      return E8_EINVAL;
+    if (it.N > 0 && M > 0 &&
+        (!it.idx1 || !it.Y || !aligned16(it.idx1) || !aligned16(it.Y) ||
+         (it.idx2 && !aligned16(it.idx2))))
+      return E8_EINVAL;
+  }
+  if (M == 0) return E8_OK;
+  if (!e8::q8_eligible(M, K) || !X || !aligned16(X)) return E8_EINVAL;
+  const size_t need = e8_gemm_grouped_workspace_bytes(M, K, bpw, count);
+  if (!workspace || !aligned16(workspace) || ws_bytes < need) return E8_EWORKSPACE;
+  int nonempty = 0;
+  for (int g = 0; g < count; ++g) nonempty += items[g].N > 0 ? 1 : 0;
+  if (nonempty == 0) return E8_OK;
+  (void)cudaGetLastError();  // a failed earlier launch must not be reported here
+  int rc = check_device(cb);
+  if (rc != E8_OK) return rc;
+  const int64_t rows = rows_b_for(M);
+  const e8::Q8Layout l = e8::q8_layout(M, K, rows);
+  const int64_t nh = e8::hadamard_block(K);
+  e8::ActQ8Out outs[e8::kMaxGroup];
+  e8::Q8Item its[e8::kMaxGroup];
+  int n = 0;
+  for (int g = 0; g < count; ++g) {
+    const e8_gemm_item& it = items[g];
+    if (it.N == 0) continue;   // nothing to compute for an empty matrix
+    uint8_t* buf = static_cast<uint8_t*>(workspace) + (size_t)g * l.total;
+    outs[n].seed = it.rht_seed;
+    outs[n].Xq = reinterpret_cast<int8_t*>(buf);
+    outs[n].scales = reinterpret_cast<float*>(buf + l.scales_off);
+    outs[n].colsum = reinterpret_cast<int32_t*>(buf + l.colsum_off);
+    outs[n].Yz = it.Y;   // zeroed by the transform, accumulated into by the GEMM
+    outs[n].yz_elems = M * it.N;
+    its[n].idx1 = it.idx1;
+    its[n].idx2 = it.idx2;
+    its[n].N = it.N;
+    its[n].alpha = alpha_of(it.scale, nh, bpw);
+    its[n].Xq = outs[n].Xq;
+    its[n].scales = outs[n].scales;
+    its[n].colsum = outs[n].colsum;
+    its[n].Y = it.Y;
+    ++n;
+  }
+  cudaStream_t st = (cudaStream_t)stream;
+  // programmatic launches, as the single-matrix int8 path: the GEMM's prologue
+  // and index loads overlap the transform, which writes only the workspace and Y
+  cudaError_t e = e8::launch_act_q8_group(X, M, K, outs, n, rows, st, 1);
+  if (e != cudaSuccess) return E8_ECUDA;
+  e = e8::launch_gemm_q8_group(dev_view(cb), its, n, M, K, (int)rows, bpw, 1, 1, cb->sm_count,
+                               st);
+  return cuda_status(e);
+}
+
 int e8_sync_status(const e8_codebook* cb, void* stream) {
   int rc = check_device(cb);
   if (rc != E8_OK) return rc;

@@ -9,15 +9,21 @@
 //   xt_m = s_m (q0_m + q1_m / 128).
 // The weight operand is z + 128 as unsigned bytes, decoded on chip straight
 // into tensor memory; tcgen05.mma kind::i8 accumulates exactly in int32 and
-// the epilogue removes the +128 bias with the row sums of Xq:
+// the epilogue removes the +128 bias with the sums of the Xq rows over the
+// K units that the partial product covers (cs, from the transform's per-unit
+// sums), exactly in int32, before anything is rounded:
 //   y[m][n] = alpha s_m ((D[n][2m] - 128 cs[2m]) + (D[n][2m+1] - 128 cs[2m+1]) / 128).
 //
 // Work split (stream-K): the (128-row tile, 128-wide K unit) pairs are laid out
 // tile by tile and every CTA of a one-per-SM grid takes a contiguous run of
-// them, so all SMs get the same number of units within one.  A run covers at
-// most a few tiles; the partial tile of each is added into Y (zeroed by the
-// transform kernel that precedes this one) by a TMA bulk reduce-add, so the
-// order of the few partial sums of an output is not fixed.
+// them, so all SMs get the same number of units within one.  A launch may
+// serve a group of up to four weight matrices with the same K and rate (for
+// instance q, k and v, which read the same tokens): their tiles are
+// concatenated, each with its own activation pieces, alpha and output, so the
+// pair table, the grid boundaries and the tail are paid once per group.  A
+// run covers at most a few tiles; the partial tile of each is added into Y
+// (zeroed by the transform kernel that precedes this one) by a TMA bulk
+// reduce-add, so the order of the few partial sums of an output is not fixed.
 //
 // Roles (one CTA per SM):
 //   warp 0      TMA producer: the codebook pair table (once) and the index
@@ -61,7 +67,8 @@ constexpr uint32_t ACC_TOTAL = 4 * ACC_COLS;
 constexpr uint32_t A_COLS = KU / 4;       // 4 int8 weights per TMEM column
 constexpr int MAX_STAGES = 8;
 static_assert(MAX_STAGES % 2 == 0, "each operand stage serves one decoder group and one issuer");
-constexpr int AUX_BYTES = 512;            // per-token steps [32] and row sums [64]
+// per matrix: alpha times the per-token steps [32]; then the segment's piece sums [2][64]
+constexpr int AUX_BYTES = 128 * kMaxGroup + 512;
 constexpr int BAR_BYTES = 512;
 // shared memory left free on the SM for a CTA of the activation transform
 // (K = 4096: 16 KB), so that it can run next to this kernel's CTA
@@ -121,6 +128,35 @@ __device__ __forceinline__ uint32_t sk_entry(const uint8_t* table, uint32_t off)
   return *reinterpret_cast<const uint32_t*>(table + off);
 }
 
+// Tensor maps of a group (kernel parameter space): per matrix the Xq pieces
+// (box rows_b x 128), the index arrays (box 128 rows x 16 groups) and Y.
+struct SkMaps {
+  CUtensorMap B[kMaxGroup], I1[kMaxGroup], I2[kMaxGroup], Y[kMaxGroup];
+};
+struct SkMat {
+  int tile0;             // first tile of the matrix in the concatenation
+  int N;
+  float alpha;
+  int use_tma_y;         // Y by bulk reduce-add (else fp32 atomics)
+  const float* tok_scale;
+  const int32_t* colsum;
+  float* Y;
+};
+struct SkGroup {
+  int count;
+  int tiles;             // tiles of all matrices
+  SkMat mat[kMaxGroup];
+};
+
+// Matrix of a tile of the concatenation.
+__device__ __forceinline__ int sk_mat_of(const SkGroup& g, int tile) {
+  int j = 0;
+#pragma unroll
+  for (int q = 1; q < kMaxGroup; ++q)
+    if (q < g.count && tile >= g.mat[q].tile0) j = q;
+  return j;
+}
+
 // Offset of the 16-byte half `h` of row r in a 32-byte-swizzled index tile.
 __device__ __forceinline__ uint32_t sw32_off(int r, int h) {
   return (uint32_t)(r * 32 + ((h ^ ((r >> 2) & 1)) << 4));
@@ -151,6 +187,14 @@ __device__ __forceinline__ void sk_tmem_st16(uint32_t taddr, const uint32_t (&v)
       : "memory");
 }
 
+// 32 lanes x 32 bit, 8 consecutive columns per thread.
+__device__ __forceinline__ void sk_tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+
 // No memory clobber: nothing later in the thread depends on the sum, and the
 // shared-memory loads feeding the next adds may then be hoisted past it.
 __device__ __forceinline__ void red_add_f32(float* p, float v) {
@@ -174,16 +218,14 @@ __device__ __forceinline__ int sk_unit_begin(int c, int U, int G) {
 }
 
 // CW: accumulator columns read by the epilogue (32 for up to 16 tokens, else 64).
-// tmY: Y [M][N] fp32, box 128 x M (valid when use_tma_y; else fp32 atomics).
+// maps.Y[j]: Y [M][N] fp32 of matrix j, box 128 x M (valid when its
+// use_tma_y; else fp32 atomics).
 // At most 64 registers, so that a CTA of the activation transform (512
 // threads x 32 registers) fits on the SM next to it.
 template <int BPW, int CW>
 __global__ void __maxnreg__(64)
-    k_gemm_q8(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmI1,
-              const __grid_constant__ CUtensorMap tmI2, const __grid_constant__ CUtensorMap tmY,
-              DeviceCodebook cb, int M, int N, int K, int rows_b, float alpha,
-              const float* __restrict__ tok_scale, const int32_t* __restrict__ colsum,
-              float* __restrict__ Y, int use_tma_y, int early_codes) {
+    k_gemm_q8(const __grid_constant__ SkMaps maps, const SkGroup grp, DeviceCodebook cb, int M,
+              int K, int rows_b, int early_codes) {
   using namespace sk;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const uint8_t* table = smem_raw;
@@ -202,16 +244,15 @@ __global__ void __maxnreg__(64)
   uint64_t* drain = acc_full + 5;                 // [2] one per issuer
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 7);
   volatile uint32_t* abort_flag = tmem_slot + 1;
-  float* s_sc = reinterpret_cast<float*>(smem + plan.aux_off);             // [32]
-  int32_t* s_cs = reinterpret_cast<int32_t*>(smem + plan.aux_off + 128);   // [64]
+  float* s_sc = reinterpret_cast<float*>(smem + plan.aux_off);                          // [G][32]
+  int32_t* s_cs = reinterpret_cast<int32_t*>(smem + plan.aux_off + 128 * kMaxGroup);    // [2][64]
   float* s_y = reinterpret_cast<float*>(smem + plan.y_off);                // [M][128]
   uint8_t* xq_ring = smem;
   uint8_t* code_ring = smem + plan.code_off;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kunits = K / KU;
-  const int tiles = (N + ROWS - 1) / ROWS;
-  const int U = tiles * kunits;
+  const int U = grp.tiles * kunits;
   const int u_begin = sk_unit_begin((int)blockIdx.x, U, (int)gridDim.x);
   const int nu = sk_unit_begin((int)blockIdx.x + 1, U, (int)gridDim.x) - u_begin;
   const int first_tile = u_begin / kunits;
@@ -253,10 +294,12 @@ __global__ void __maxnreg__(64)
 
   if (warp == 0) {
     if (lane == 0) {
-      tma_prefetch_desc(&tmB);
-      tma_prefetch_desc(&tmI1);
-      if (BPW > 2) tma_prefetch_desc(&tmI2);
-      if (use_tma_y) tma_prefetch_desc(&tmY);
+      for (int j = 0; j < grp.count; ++j) {
+        tma_prefetch_desc(&maps.B[j]);
+        tma_prefetch_desc(&maps.I1[j]);
+        if (BPW > 2) tma_prefetch_desc(&maps.I2[j]);
+        if (grp.mat[j].use_tma_y) tma_prefetch_desc(&maps.Y[j]);
+      }
       // the pair table in eight 16 KB pieces plus the last entry, starting at a
       // CTA-dependent piece so that the SMs do not all read the same L2 lines
       mbar_arrive_expect_tx(table_full, TABLE_BYTES);
@@ -269,12 +312,15 @@ __global__ void __maxnreg__(64)
                 table_full);
       auto load_codes = [&](int i, int s) {
         const int u = u_begin + i;
+        const int tile = u / kunits;
+        const int j = sk_mat_of(grp, tile);
+        const int lt = tile - grp.mat[j].tile0;
         uint8_t* dst = code_ring + s * plan.code_bytes;
         mbar_arrive_expect_tx(&full_code[s], code_tx);
-        tma_load_2d(dst, &tmI1, &full_code[s], (u % kunits) * GROUPS, (u / kunits) * ROWS);
+        tma_load_2d(dst, &maps.I1[0] + j, &full_code[s], (u % kunits) * GROUPS, lt * ROWS);
         if (BPW > 2)
-          tma_load_2d(dst + I1_BYTES, &tmI2, &full_code[s], (u % kunits) * GROUPS,
-                      (u / kunits) * ROWS);
+          tma_load_2d(dst + I1_BYTES, &maps.I2[0] + j, &full_code[s], (u % kunits) * GROUPS,
+                      lt * ROWS);
       };
       // Index tiles do not depend on the preceding kernel: before waiting for
       // it, load those of the first SC + SA units (the decoders of units
@@ -401,8 +447,10 @@ __global__ void __maxnreg__(64)
                                         abort_flag, status, kDevTimeoutEmpty))
           break;
         const int u = u_begin + i;
+        const int j = sk_mat_of(grp, u / kunits);
         mbar_arrive_expect_tx(&full_a[sa], (uint32_t)plan.b_bytes);
-        tma_load_2d(xq_ring + (i % SX) * plan.b_bytes, &tmB, &full_a[sa], (u % kunits) * KU, 0);
+        tma_load_2d(xq_ring + (i % SX) * plan.b_bytes, &maps.B[0] + j, &full_a[sa],
+                    (u % kunits) * KU, 0);
         if (++sa == SA) sa = 0;
       }
       if (ld_shared_volatile(abort_flag)) {
@@ -478,13 +526,13 @@ __global__ void __maxnreg__(64)
     const int q = warp & 3;
     const int r = q * 32 + lane;
     const bool issuer = warp == EPI_WARP0 && lane == 0;
-    grid_dep_wait();   // steps, row sums and the zeroed Y come from the transform
+    grid_dep_wait();   // steps, unit sums and the zeroed Y come from the transform
     if (warp == EPI_WARP0) {
-      s_sc[lane] = lane < M ? alpha * __ldg(tok_scale + lane) : 0.0f;
-      s_cs[lane] = lane < rows_b ? __ldg(colsum + lane) : 0;
-      s_cs[32 + lane] = 32 + lane < rows_b ? __ldg(colsum + 32 + lane) : 0;
+      for (int j = 0; j < grp.count; ++j) {
+        const SkMat& mt = grp.mat[j];
+        s_sc[32 * j + lane] = lane < M ? mt.alpha * __ldg(mt.tok_scale + lane) : 0.0f;
+      }
     }
-    asm volatile("bar.sync 1, 128;" ::: "memory");
     // every epilogue thread runs the same sequence of named barriers, also
     // after a failed wait (it then only skips the work)
     bool ok = true;
@@ -496,52 +544,72 @@ __global__ void __maxnreg__(64)
       // which issuers accumulated into the segment (units of parity 0 / 1)
       const bool has0 = hi - lo >= 2 || (lo & 1) == 0;
       const bool has1 = hi - lo >= 2 || (lo & 1) == 1;
+      const int tile = first_tile + seg;
+      const int mj = sk_mat_of(grp, tile);
+      // sums of the Xq rows over the segment's K units [ku_lo, ku_hi): the
+      // bias this partial product carries (double-buffered by segment parity:
+      // the other buffer may still be read for the previous segment)
+      int32_t* cs = s_cs + 64 * b;
+      if (warp == EPI_WARP0) {
+        const int ku_lo = u_begin + lo - tile * kunits, ku_hi = u_begin + hi - tile * kunits;
+        const int32_t* src = grp.mat[mj].colsum;
+        int a0 = 0, a1 = 0;
+        for (int ku = ku_lo; ku < ku_hi; ++ku) {
+          if (lane < rows_b) a0 += __ldg(src + (size_t)ku * rows_b + lane);
+          if (32 + lane < rows_b) a1 += __ldg(src + (size_t)ku * rows_b + 32 + lane);
+        }
+        cs[lane] = a0;
+        cs[32 + lane] = a1;
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
       lo = hi;
       ok = ok && mbar_wait_sleep(&acc_full[b], (uint32_t)(seg >> 1) & 1u, abort_flag, status,
                                  kDevTimeoutMma);
       tc_fence_after();
-      const int tile = first_tile + seg;
-      const int n = tile * ROWS + r;
-      // the segment holding K unit 0 of its tile removes the bias of the whole row
-      const int corr = tile * kunits >= u_begin ? 128 : 0;
+      const int N = grp.mat[mj].N;
+      float* __restrict__ Y = grp.mat[mj].Y;
+      const int use_tma_y = grp.mat[mj].use_tma_y;
+      const float* sc = s_sc + 32 * mj;
+      const int n = (tile - grp.mat[mj].tile0) * ROWS + r;
+      constexpr int corr = 128;
       const uint32_t lane_off = (uint32_t)(q * 32) << 16;
       const uint32_t t0a = tmem_base + (uint32_t)b * ACC_COLS + lane_off;         // parity 0
       const uint32_t t1a = tmem_base + (uint32_t)(2 + b) * ACC_COLS + lane_off;   // parity 1
-      // 16 accumulator columns (8 tokens) per pass
+      // 8 accumulator columns (4 tokens) per pass
 #pragma unroll
-      for (int c0 = 0; c0 < CW; c0 += 16) {
+      for (int c0 = 0; c0 < CW; c0 += 8) {
         if (!ok) break;
-        uint32_t dv[16], dw[16];
+        uint32_t dv[8], dw[8];
         if (c0 < rows_b) {
-          if (has0) tmem_ld16(t0a + (uint32_t)c0, dv);
-          if (has1) tmem_ld16(t1a + (uint32_t)c0, dw);
+          if (has0) sk_tmem_ld8(t0a + (uint32_t)c0, dv);
+          if (has1) sk_tmem_ld8(t1a + (uint32_t)c0, dw);
           tmem_ld_wait();
         }
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
+        for (int j = 0; j < 8; ++j) {
           const uint32_t x0 = (c0 < rows_b && has0) ? dv[j] : 0u;
           const uint32_t x1 = (c0 < rows_b && has1) ? dw[j] : 0u;
           dv[j] = x0 + x1;
         }
         if (use_tma_y) {
-          // tokens past M have zero steps and row sums: staged as zeros (the
+          // tokens past M have zero steps and unit sums: staged as zeros (the
           // bulk reduce covers only M rows), no branch in the loop
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
+          for (int j = 0; j < 4; ++j) {
             const int m = (c0 >> 1) + j;
-            const int d0 = (int)dv[2 * j] - corr * s_cs[2 * m];
-            const int d1 = (int)dv[2 * j + 1] - corr * s_cs[2 * m + 1];
-            s_y[m * ROWS + r] = s_sc[m] * ((float)d0 + (float)d1 * (1.0f / 128.0f));
+            const int d0 = (int)dv[2 * j] - corr * cs[2 * m];
+            const int d1 = (int)dv[2 * j + 1] - corr * cs[2 * m + 1];
+            s_y[m * ROWS + r] = sc[m] * ((float)d0 + (float)d1 * (1.0f / 128.0f));
           }
         } else if (n < N) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
+          for (int j = 0; j < 4; ++j) {
             const int m = (c0 >> 1) + j;
-            const int d0 = (int)dv[2 * j] - corr * s_cs[2 * m];
-            const int d1 = (int)dv[2 * j + 1] - corr * s_cs[2 * m + 1];
+            const int d0 = (int)dv[2 * j] - corr * cs[2 * m];
+            const int d1 = (int)dv[2 * j + 1] - corr * cs[2 * m + 1];
             if (m < M)
               red_add_f32(Y + (size_t)m * N + n,
-                          s_sc[m] * ((float)d0 + (float)d1 * (1.0f / 128.0f)));
+                          sc[m] * ((float)d0 + (float)d1 * (1.0f / 128.0f)));
           }
         }
       }
@@ -554,13 +622,13 @@ __global__ void __maxnreg__(64)
         fence_proxy_async_smem();
         asm volatile("bar.sync 1, 128;" ::: "memory");
         if (issuer && ok) {
-          tma_reduce_add_2d(&tmY, smem_u32(s_y), tile * ROWS, 0);
+          tma_reduce_add_2d(&maps.Y[0] + mj, smem_u32(s_y), (tile - grp.mat[mj].tile0) * ROWS, 0);
           bulk_wait_read_all();
         }
         asm volatile("bar.sync 1, 128;" ::: "memory");
       }
     }
-    if (issuer && use_tma_y) bulk_wait_all();
+    if (issuer) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -573,39 +641,63 @@ __global__ void __maxnreg__(64)
 }
 
 template <int BPW>
-static cudaError_t launch_gemm_q8(const DeviceCodebook& cb, const ActQ8Args& a, int sm_count,
-                                  cudaStream_t st) {
+static cudaError_t launch_gemm_q8(const DeviceCodebook& cb, const Q8Item* items, int count,
+                                  int64_t M, int64_t K, int rows_b, int pdl, int early_codes,
+                                  int sm_count, cudaStream_t st) {
   using namespace sk;
-  if (a.rows_b < 16 || a.rows_b > 64 || (a.rows_b % 16) != 0 || a.M < 1 || a.M > 32 ||
-      2 * a.M > a.rows_b || (a.K % KU) != 0)
+  if (rows_b < 16 || rows_b > 64 || (rows_b % 16) != 0 || M < 1 || M > 32 || 2 * M > rows_b ||
+      (K % KU) != 0 || K > INT32_MAX || count < 1 || count > kMaxGroup)
     return cudaErrorInvalidValue;
-  CUtensorMap tb, ti1, ti2, ty;
-  if (!make_tmap_2d(&tb, a.Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.rows_b,
-                    (uint64_t)a.K, (uint32_t)a.rows_b, KU, CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorInvalidValue;
-  if (!make_tmap_2d(&ti1, a.idx1, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)a.N,
-                    (uint64_t)(a.K / 8), ROWS, GROUPS, CU_TENSOR_MAP_SWIZZLE_32B))
-    return cudaErrorInvalidValue;
-  if (BPW == 4) {
-    if (!make_tmap_2d(&ti2, a.idx2, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)a.N,
-                      (uint64_t)(a.K / 8), ROWS, GROUPS, CU_TENSOR_MAP_SWIZZLE_32B))
+  SkMaps maps;
+  SkGroup grp = {};
+  grp.count = count;
+  int64_t tiles = 0;
+  for (int g = 0; g < count; ++g) {
+    const Q8Item& a = items[g];
+    if (a.N < 1 || a.N > INT32_MAX) return cudaErrorInvalidValue;
+    if (!make_tmap_2d(&maps.B[g], a.Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)rows_b,
+                      (uint64_t)K, (uint32_t)rows_b, KU, CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
-  } else if (BPW == 3) {
-    if (!make_tmap_2d(&ti2, a.idx2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.N,
-                      (uint64_t)(a.K / 8), ROWS, GROUPS, CU_TENSOR_MAP_SWIZZLE_NONE))
+    if (!make_tmap_2d(&maps.I1[g], a.idx1, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)a.N,
+                      (uint64_t)(K / 8), ROWS, GROUPS, CU_TENSOR_MAP_SWIZZLE_32B))
       return cudaErrorInvalidValue;
-  } else {
-    ti2 = ti1;
+    if (BPW == 4) {
+      if (!make_tmap_2d(&maps.I2[g], a.idx2, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)a.N,
+                        (uint64_t)(K / 8), ROWS, GROUPS, CU_TENSOR_MAP_SWIZZLE_32B))
+        return cudaErrorInvalidValue;
+    } else if (BPW == 3) {
+      if (!make_tmap_2d(&maps.I2[g], a.idx2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.N,
+                        (uint64_t)(K / 8), ROWS, GROUPS, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    } else {
+      maps.I2[g] = maps.I1[g];
+    }
+    // Y by bulk reduce-add when its rows are 16-byte multiples (else fp32 atomics)
+    int use_tma_y = (a.N % 4) == 0 &&
+                    make_tmap_2d(&maps.Y[g], a.Y, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)M,
+                                 (uint64_t)a.N, (uint32_t)M, ROWS, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (!use_tma_y) maps.Y[g] = maps.B[g];
+    SkMat& mt = grp.mat[g];
+    mt.tile0 = (int)tiles;
+    mt.N = (int)a.N;
+    mt.alpha = a.alpha;
+    mt.use_tma_y = use_tma_y;
+    mt.tok_scale = a.scales;
+    mt.colsum = a.colsum;
+    mt.Y = a.Y;
+    tiles += (a.N + ROWS - 1) / ROWS;
   }
-  // Y by bulk reduce-add when its rows are 16-byte multiples (else fp32 atomics)
-  int use_tma_y = (a.N % 4) == 0 &&
-                  make_tmap_2d(&ty, a.Y, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)a.M,
-                               (uint64_t)a.N, (uint32_t)a.M, ROWS, CU_TENSOR_MAP_SWIZZLE_NONE);
-  if (!use_tma_y) ty = tb;
-  const SkPlan plan = sk_plan(a.rows_b, BPW);
+  for (int g = count; g < kMaxGroup; ++g) {
+    maps.B[g] = maps.B[0];
+    maps.I1[g] = maps.I1[0];
+    maps.I2[g] = maps.I2[0];
+    maps.Y[g] = maps.Y[0];
+  }
+  const SkPlan plan = sk_plan(rows_b, BPW);
   if (plan.sa < 2 || plan.sc < 2 || plan.total > kMaxDynSmem) return cudaErrorInvalidValue;
-  const int64_t units = ((a.N + ROWS - 1) / ROWS) * (a.K / KU);
+  const int64_t units = tiles * (K / KU);
   if (units > INT32_MAX) return cudaErrorInvalidValue;
+  grp.tiles = (int)tiles;
   const int grid = (int)(units < sm_count ? units : sm_count);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
@@ -614,24 +706,41 @@ static cudaError_t launch_gemm_q8(const DeviceCodebook& cb, const ActQ8Args& a, 
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = a.pdl ? 1 : 0;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  auto kern = a.rows_b <= 32 ? k_gemm_q8<BPW, 32> : k_gemm_q8<BPW, 64>;
+  auto kern = rows_b <= 32 ? k_gemm_q8<BPW, 32> : k_gemm_q8<BPW, 64>;
   // the largest carveout, as the transform kernel has: CTAs of the two can share an SM
   cudaError_t e = ensure_smem_limit(kern, kMaxDynSmem, true);
   if (e != cudaSuccess) return e;
-  e = cudaLaunchKernelEx(&cfg, kern, tb, ti1, ti2, ty, cb, (int)a.M, (int)a.N, (int)a.K,
-                         a.rows_b, a.alpha, a.scales, a.colsum, a.Y, use_tma_y, a.early_codes);
+  e = cudaLaunchKernelEx(&cfg, kern, maps, grp, cb, (int)M, (int)K, rows_b, early_codes);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
+cudaError_t launch_gemm_q8_group(const DeviceCodebook& cb, const Q8Item* items, int count,
+                                 int64_t M, int64_t K, int rows_b, int bpw, int pdl,
+                                 int early_codes, int sm_count, cudaStream_t st) {
+  if (bpw == 2) return launch_gemm_q8<2>(cb, items, count, M, K, rows_b, pdl, early_codes,
+                                         sm_count, st);
+  if (bpw == 3) return launch_gemm_q8<3>(cb, items, count, M, K, rows_b, pdl, early_codes,
+                                         sm_count, st);
+  return launch_gemm_q8<4>(cb, items, count, M, K, rows_b, pdl, early_codes, sm_count, st);
+}
+
 cudaError_t launch_act_gemm_q8(const DeviceCodebook& cb, const ActQ8Args& a, int sm_count,
                                cudaStream_t st) {
-  if (a.bpw == 2) return launch_gemm_q8<2>(cb, a, sm_count, st);
-  if (a.bpw == 3) return launch_gemm_q8<3>(cb, a, sm_count, st);
-  return launch_gemm_q8<4>(cb, a, sm_count, st);
+  Q8Item it;
+  it.idx1 = a.idx1;
+  it.idx2 = a.idx2;
+  it.N = a.N;
+  it.alpha = a.alpha;
+  it.Xq = a.Xq;
+  it.scales = a.scales;
+  it.colsum = a.colsum;
+  it.Y = a.Y;
+  return launch_gemm_q8_group(cb, &it, 1, a.M, a.K, a.rows_b, a.bpw, a.pdl, a.early_codes,
+                              sm_count, st);
 }
 
 }  // namespace e8

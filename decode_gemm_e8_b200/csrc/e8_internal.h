@@ -120,7 +120,7 @@ cudaError_t launch_act_gemm(const DeviceCodebook& cb, const ActGemmArgs& a, int 
 struct ActQ8Args {
   const int8_t* Xq;
   const float* scales;   // [M]
-  const int32_t* colsum; // [rows_b]
+  const int32_t* colsum; // [K / 128][rows_b]
   int64_t M, N, K;
   int rows_b;
   const uint16_t* idx1;
@@ -133,15 +133,47 @@ struct ActQ8Args {
 };
 cudaError_t launch_act_gemm_q8(const DeviceCodebook& cb, const ActQ8Args& a, int sm_count,
                                cudaStream_t st);
+
+// Grouped int8 path: up to kMaxGroup weight matrices that share K, bpw and the
+// token count, each with its own transformed activations (its own RHT seed),
+// alpha and output, in one launch whose stream-K units run over the
+// concatenated 128-row tiles of all of them.
+constexpr int kMaxGroup = 4;
+struct Q8Item {
+  const uint16_t* idx1;
+  const void* idx2;
+  int64_t N;
+  float alpha;
+  const int8_t* Xq;       // [rows_b][K], token m: rows 2m, 2m + 1
+  const float* scales;    // [M]
+  const int32_t* colsum;  // [K / 128][rows_b]
+  float* Y;               // [M][N], zero when the kernel starts
+};
+cudaError_t launch_gemm_q8_group(const DeviceCodebook& cb, const Q8Item* items, int count,
+                                 int64_t M, int64_t K, int rows_b, int bpw, int pdl,
+                                 int early_codes, int sm_count, cudaStream_t st);
 // When Yz is not null the kernel also zeroes Yz[0, yz_elems) (the fp32 output
 // that launch_act_gemm_q8 accumulates into), after the preceding kernel ends.
 cudaError_t launch_act_q8(const uint16_t* X, int64_t M, int64_t K, uint64_t seed, int8_t* Xq,
                           float* scales, int32_t* colsum, int64_t rows, cudaStream_t st,
                           int pdl, float* Yz = nullptr, int64_t yz_elems = 0);
+// One output set of the grouped transform: X transformed with `seed` into
+// Xq / scales / colsum, and Yz[0, yz_elems) zeroed (Yz may be null).
+struct ActQ8Out {
+  uint64_t seed;
+  int8_t* Xq;
+  float* scales;
+  int32_t* colsum;
+  float* Yz;
+  int64_t yz_elems;
+};
+// The same transform for up to kMaxGroup seeds in one launch.
+cudaError_t launch_act_q8_group(const uint16_t* X, int64_t M, int64_t K, const ActQ8Out* outs,
+                                int count, int64_t rows, cudaStream_t st, int pdl);
 
 // Layout of the int8 activation buffer: Xq [rows][K] int8, then the per-token
-// steps (fp32 [M]) and the per-row column sums (int32 [rows]), each part
-// starting on a 256-byte boundary.
+// steps (fp32 [M]) and the sums of every row over every 128-column unit
+// (int32 [K / 128][rows]), each part starting on a 256-byte boundary.
 struct Q8Layout {
   size_t scales_off, colsum_off, total;
 };
@@ -150,7 +182,7 @@ inline Q8Layout q8_layout(int64_t M, int64_t K, int64_t rows) {
   Q8Layout l;
   l.scales_off = r256((size_t)rows * (size_t)K);
   l.colsum_off = l.scales_off + r256((size_t)M * 4);
-  l.total = l.colsum_off + r256((size_t)rows * 4);
+  l.total = l.colsum_off + r256((size_t)rows * (size_t)(K / 128) * 4);
   return l;
 }
 // Shapes served by the int8 path: up to 32 tokens, K a multiple of 256 whose

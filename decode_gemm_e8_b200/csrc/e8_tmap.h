@@ -44,7 +44,7 @@ inline bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType
     int dtype, elem_bytes, swizzle;
     CUtensorMap map;
   };
-  constexpr int kEntries = 16;
+  constexpr int kEntries = 64;
   thread_local Entry cache[kEntries];
   thread_local int used = 0, next = 0;
   for (int i = 0; i < used; ++i) {

@@ -159,8 +159,9 @@ int e8_gemm(const e8_codebook* cb, const uint16_t* X, int64_t M, const uint16_t*
  *     q1 of token m, where xt = FWHT(D x_m) per Hadamard block,
  *     s_m = max|xt| / 127, q0 = rint(xt / s_m), q1 = rint((xt - q0 s_m) 128 / s_m),
  *     so xt = s_m (q0 + q1 / 128) within s_m / 256; padding rows are zero;
- *   then s_m (fp32 [M]) and the row sums of Xq (int32 [rows]), each part
- *     starting on a 256-byte boundary after the previous one.
+ *   then s_m (fp32 [M]) and the sums of every Xq row over every unit of 128
+ *     columns (int32 [K / 128][rows], unit-major), each part starting on a
+ *     256-byte boundary after the previous one.
  * Shapes: 1 <= M <= 32, K a multiple of 256 whose Hadamard block is 256..4096,
  * K <= 32768 (else E8_EINVAL). */
 int e8_act_rht_q8(const uint16_t* X, int64_t M, int64_t K, uint64_t rht_seed, void* buf,
@@ -185,6 +186,44 @@ int e8_gemm_xt(const e8_codebook* cb, const void* xq, int64_t M, const uint16_t*
 /* Row count of the transformed-activation buffers for M tokens: 2M rounded up to
  * a multiple of 16. */
 int e8_gemm_xt_rows(int64_t M);
+
+/* One weight matrix of e8_gemm_grouped: its codes (as e8_encode writes them;
+ * idx2 NULL for bpw 2), row count N, transform seed, global scale and output
+ * Y fp32 [M][N] (device). */
+typedef struct e8_gemm_item {
+  const uint16_t* idx1;
+  const void* idx2;
+  int64_t N;
+  uint64_t rht_seed;
+  float scale;
+  float* Y;
+} e8_gemm_item;
+
+#define E8_GROUP_MAX 4
+
+/* Small-batch GEMM of several weight matrices that read the same activations
+ * ("How it works", items 1-2: weights rebuilt from their indices and the
+ * inverse transform at run time), for instance the q, k and v or the gate and
+ * up projections of a decoder layer: for every item,
+ *   Y_i = X * W_dec_i^T,
+ * as e8_gemm in mode E8_GEMM_ACT_RHT computes it on the int8 path (same
+ * accuracy, same arrival-order partial sums), in two launches for the whole
+ * group: one activation transform per item seed and one fused decode + GEMM
+ * whose work runs over the concatenated row tiles of all items, so the
+ * per-launch costs (codebook table load, grid boundaries, tail) are paid once.
+ * X bf16 [M][K]; 1 <= M <= 32; K as for e8_act_rht_q8; all items share K and
+ * bpw; 1 <= count <= E8_GROUP_MAX; an item with N == 0 is skipped; the Y
+ * buffers may not overlap one another, X or the workspace.  workspace: at least
+ * e8_gemm_grouped_workspace_bytes(M, K, bpw, count) bytes (the int8
+ * activations of every item).  Ordering as e8_gemm's int8 path.  Errors:
+ * E8_EINVAL (arguments, shapes, alignment), E8_EWORKSPACE, E8_EDEVICE,
+ * E8_ECUDA; all are reported before anything is launched except E8_ECUDA. */
+int e8_gemm_grouped(const e8_codebook* cb, const uint16_t* X, int64_t M, int64_t K, int bpw,
+                    const e8_gemm_item* items, int count, void* workspace, size_t ws_bytes,
+                    void* stream);
+
+/* Workspace bytes for e8_gemm_grouped; 0 if the arguments are invalid. */
+size_t e8_gemm_grouped_workspace_bytes(int64_t M, int64_t K, int bpw, int count);
 
 /* E8_GEMM_ACT_RHT without a workspace, for callers that may not allocate device
  * memory where they run the layer: plugins whose host framework owns all

@@ -48,11 +48,13 @@ def test_workspace_sizes(lib):
     # fast path, then what the class search leaves open)
     assert e8.e8_workspace_bytes(e8.E8_OP_ENCODE, 0, N, K, 4) == 256 + 2 * 48 * N * K // 8
     assert e8.e8_workspace_bytes(e8.E8_GEMM_DECODED_W, 4096, N, K, 3) == N * K * 2
-    # int8 pieces for 16 tokens: 32 rows of K bytes, 16 steps, 32 row sums
-    assert e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT, 16, N, K, 4) == 32 * K + 256 + 256
-    assert e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT, 1, N, K, 4) == 16 * K + 256 + 256
-    assert e8.e8_workspace_bytes(e8.E8_GEMM_AUTO, 16, N, K, 4) == 32 * K + 256 + 256
-    assert e8.e8_act_q8_bytes(16, K) == 32 * K + 512
+    # int8 pieces for 16 tokens: 32 rows of K bytes, 16 steps, then the sums of
+    # the 32 rows over each of the K / 128 units
+    units = K // 128
+    assert e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT, 16, N, K, 4) == 32 * K + 256 + 32 * units * 4
+    assert e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT, 1, N, K, 4) == 16 * K + 256 + 16 * units * 4
+    assert e8.e8_workspace_bytes(e8.E8_GEMM_AUTO, 16, N, K, 4) == 32 * K + 256 + 32 * units * 4
+    assert e8.e8_act_q8_bytes(16, K) == 32 * K + 256 + 32 * units * 4
     # bf16 hi and lo rows where the int8 path does not apply (more than 32 tokens)
     assert e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT, 40, N, K, 4) == 80 * K * 2
     assert e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT_SMEM, 16, N, K, 4) == 32 * K * 2
@@ -136,3 +138,62 @@ def test_missing_library_fails_loudly(tmp_path):
             e8.load_library(str(tmp_path / "absent.so"))
     finally:
         e8._lib = saved
+
+
+def test_grouped_workspace_sizes(lib):
+    # one int8 activation buffer per item: 2M rows (padded to 16) of K bytes,
+    # the per-token steps and the row sums, each on 256 bytes
+    one = e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT, 16, 4096, 4096, 4)
+    assert e8.e8_gemm_grouped_workspace_bytes(16, 4096, 4, 3) == 3 * one
+    assert e8.e8_gemm_grouped_workspace_bytes(5, 14336, 2, 4) == \
+        4 * (16 * 14336 + 256 + 16 * (14336 // 128) * 4)
+    # invalid: no items, too many, more than 32 tokens, K outside the int8 path
+    assert e8.e8_gemm_grouped_workspace_bytes(16, 4096, 4, 0) == 0
+    assert e8.e8_gemm_grouped_workspace_bytes(16, 4096, 4, e8.E8_GROUP_MAX + 1) == 0
+    assert e8.e8_gemm_grouped_workspace_bytes(33, 4096, 4, 2) == 0
+    assert e8.e8_gemm_grouped_workspace_bytes(16, 4104, 4, 2) == 0
+
+
+def test_grouped_call_refuses_bad_arguments_before_any_cuda_call(lib):
+    # like e8_gemm_host: argument and workspace errors come before the first
+    # CUDA call (a CUDA call on this GPU-less host would answer E8_ECUDA); the
+    # codebook and device addresses are stand-ins that are never dereferenced
+    import ctypes
+    cb, dev = 1 << 20, 1 << 24
+    M, K, bpw = 16, 4096, 4
+
+    def items(n=3, change=None):
+        arr = (e8.GemmItem * max(1, n))()
+        for i in range(n):
+            d = dict(idx1=dev + 0x100000 * i, idx2=dev + 0x100000 * i + 0x80000, N=1024,
+                     rht_seed=i, scale=0.02, Y=dev + 0x4000000 + 0x100000 * i)
+            d.update((change or {}).get(i, {}))
+            arr[i] = e8.GemmItem(d["idx1"], d["idx2"], d["N"], d["rht_seed"], d["scale"], d["Y"])
+        return arr
+
+    def call(arr=None, n=3, M=M, K=K, bpw=bpw, x=dev + 0x8000000, ws=dev + 0x9000000, wsb=None,
+             cbp=cb):
+        arr = items(n) if arr is None else arr
+        if wsb is None:
+            wsb = e8.e8_gemm_grouped_workspace_bytes(M, K, bpw, n)
+        return lib.e8_gemm_grouped(cbp, x, M, K, bpw, ctypes.cast(arr, ctypes.c_void_p), n, ws,
+                                   wsb, None)
+
+    assert call(cbp=None) == e8.E8_EINVAL
+    assert call(n=0, arr=items(1)) == e8.E8_EINVAL
+    assert call(n=e8.E8_GROUP_MAX + 1, arr=items(e8.E8_GROUP_MAX + 1)) == e8.E8_EINVAL
+    assert call(bpw=5) == e8.E8_EINVAL
+    assert call(K=100) == e8.E8_EINVAL
+    assert call(M=33) == e8.E8_EINVAL                      # int8 path: at most 32 tokens
+    assert call(arr=items(3, {1: dict(scale=0.0)})) == e8.E8_EINVAL
+    assert call(arr=items(3, {2: dict(idx2=None)})) == e8.E8_EINVAL   # 4 bpw needs idx2
+    assert call(arr=items(3, {0: dict(idx1=dev + 2)})) == e8.E8_EINVAL
+    assert call(arr=items(3, {1: dict(Y=None)})) == e8.E8_EINVAL
+    assert call(arr=items(3, {1: dict(N=-1)})) == e8.E8_EINVAL
+    assert call(x=dev + 8) == e8.E8_EINVAL
+    need = e8.e8_gemm_grouped_workspace_bytes(M, K, bpw, 3)
+    assert call(wsb=need - 1) == e8.E8_EWORKSPACE
+    assert call(ws=None) == e8.E8_EWORKSPACE
+    # nothing to do: no CUDA call either
+    assert call(M=0) == e8.E8_OK
+    assert call(arr=items(3, {0: dict(N=0), 1: dict(N=0), 2: dict(N=0)})) == e8.E8_OK
