@@ -35,10 +35,11 @@
 //   warps 1, 22 tensor-memory allocation (warp 1); one elected lane of each
 //               issues tcgen05.mma (M = 128 weight rows, N = rows_b, K = 32)
 //               and the commits for the even / odd units
-//   warps 2-17  decoders, two groups of eight taking alternate units: each
-//               thread owns one weight row (its TMEM lane) and 8 of the 16
-//               groups of a unit: index loads, pair-table gathers, combine,
-//               tcgen05.st of 16 columns into the unit's operand stage
+//   warps 2-17  decoders, four groups of four (one warp per TMEM lane
+//               quarter) taking units in turn: each thread owns one weight
+//               row (its TMEM lane) and the 16 groups of the unit: index
+//               loads, pair-table gathers, combine, two tcgen05.st of 16
+//               columns into the unit's operand stage
 //   warps 18-21 epilogue, one per TMEM lane quarter: accumulator -> shared
 //               memory -> bulk reduce-add into Y
 // The tensor cores are used only for the X W^T contraction.
@@ -53,8 +54,8 @@ namespace sk {
 constexpr int ROWS = 128;                 // weight rows per tile (MMA M)
 constexpr int KU = 128;                   // K of one work unit
 constexpr int GROUPS = KU / 8;            // groups of a row in one unit
-constexpr int DEC_GROUPS = 2;
-constexpr int DEC_WARPS = 8 * DEC_GROUPS;
+constexpr int DEC_GROUPS = 4;
+constexpr int DEC_WARPS = 4 * DEC_GROUPS;
 constexpr int EPI_WARP0 = 2 + DEC_WARPS;
 constexpr int MMA2_WARP = EPI_WARP0 + 4;  // issuer of the odd units
 constexpr int XQ_WARP = MMA2_WARP + 1;    // producer of the Xq tiles
@@ -66,9 +67,10 @@ constexpr uint32_t ACC_COLS = 64;         // int32 accumulator columns per buffe
 constexpr uint32_t ACC_TOTAL = 4 * ACC_COLS;
 constexpr uint32_t A_COLS = KU / 4;       // 4 int8 weights per TMEM column
 constexpr int MAX_STAGES = 8;
-static_assert(MAX_STAGES % 2 == 0, "each operand stage serves one decoder group and one issuer");
-// per matrix: alpha times the per-token steps [32]; then the segment's piece sums [2][64]
-constexpr int AUX_BYTES = 128 * kMaxGroup + 512;
+static_assert(MAX_STAGES % DEC_GROUPS == 0 && MAX_STAGES % 2 == 0,
+              "each operand stage serves one decoder group and one issuer");
+// per matrix: alpha times the per-token steps [32]; then the segments' piece sums [3][64]
+constexpr int AUX_BYTES = 128 * kMaxGroup + 768;
 constexpr int BAR_BYTES = 512;
 // shared memory left free on the SM for a CTA of the activation transform
 // (K = 4096: 16 KB), so that it can run next to this kernel's CTA
@@ -103,12 +105,12 @@ __host__ __device__ inline SkPlan sk_plan(int rows_b, int bpw) {
     if (budget - p.sx * p.b_bytes >= 4 * p.code_bytes) break;
   p.sc = (budget - p.sx * p.b_bytes) / p.code_bytes;
   if (p.sc > MAX_STAGES) p.sc = MAX_STAGES;
-  // An even number of index stages keeps each stage with one decoder group
-  // (groups take alternate units).  Bulk copies may land out of order: were a
+  // A multiple of four index stages keeps each stage with one decoder group
+  // (the four groups take units in turn).  Bulk copies may land out of order: were a
   // stage shared, a group could reach its next use of it while the other
   // group's copy into it was still in flight, and the parity wait would take
   // the barrier two phases behind for the phase it waits for.
-  p.sc &= ~1;
+  p.sc &= ~3;
   p.code_off = p.sx * p.b_bytes;
   p.y_off = p.code_off + p.sc * p.code_bytes;
   p.aux_off = p.y_off + y_bytes;
@@ -245,7 +247,7 @@ __global__ void __maxnreg__(64)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 7);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   float* s_sc = reinterpret_cast<float*>(smem + plan.aux_off);                          // [G][32]
-  int32_t* s_cs = reinterpret_cast<int32_t*>(smem + plan.aux_off + 128 * kMaxGroup);    // [2][64]
+  int32_t* s_cs = reinterpret_cast<int32_t*>(smem + plan.aux_off + 128 * kMaxGroup);    // [3][64]
   float* s_y = reinterpret_cast<float*>(smem + plan.y_off);                // [M][128]
   uint8_t* xq_ring = smem;
   uint8_t* code_ring = smem + plan.code_off;
@@ -262,10 +264,10 @@ __global__ void __maxnreg__(64)
   if (threadIdx.x == 0) {
     for (int s = 0; s < SC; ++s) {
       mbar_init(&full_code[s], 1);
-      mbar_init(&code_empty[s], 8);
+      mbar_init(&code_empty[s], 4);
     }
     for (int s = 0; s < SA; ++s) {
-      mbar_init(&full_a[s], 9);   // eight decoder warps + the Xq tile
+      mbar_init(&full_a[s], 5);   // four decoder warps + the Xq tile
       mbar_init(&a_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -310,17 +312,16 @@ __global__ void __maxnreg__(64)
       }
       bulk_load(smem_raw + 8 * 16384, reinterpret_cast<const uint8_t*>(cb.table) + 8 * 16384, 16,
                 table_full);
-      auto load_codes = [&](int i, int s) {
+      // m1 / m2: the index maps of the unit's matrix, tile0 its first tile
+      auto load_codes = [&](int i, int s, const CUtensorMap* m1, const CUtensorMap* m2,
+                            int tile0) {
         const int u = u_begin + i;
-        const int tile = u / kunits;
-        const int j = sk_mat_of(grp, tile);
-        const int lt = tile - grp.mat[j].tile0;
+        const int lt = u / kunits - tile0;
         uint8_t* dst = code_ring + s * plan.code_bytes;
         mbar_arrive_expect_tx(&full_code[s], code_tx);
-        tma_load_2d(dst, &maps.I1[0] + j, &full_code[s], (u % kunits) * GROUPS, lt * ROWS);
+        tma_load_2d(dst, m1, &full_code[s], (u % kunits) * GROUPS, lt * ROWS);
         if (BPW > 2)
-          tma_load_2d(dst + I1_BYTES, &maps.I2[0] + j, &full_code[s], (u % kunits) * GROUPS,
-                      lt * ROWS);
+          tma_load_2d(dst + I1_BYTES, m2, &full_code[s], (u % kunits) * GROUPS, lt * ROWS);
       };
       // Index tiles do not depend on the preceding kernel: before waiting for
       // it, load those of the first SC + SA units (the decoders of units
@@ -330,14 +331,15 @@ __global__ void __maxnreg__(64)
       int cs = 0;
       uint32_t cph = 0;
       bool ok = true;
-      auto next_codes = [&](int limit) {
+      auto next_codes = [&](int limit, const CUtensorMap* m1, const CUtensorMap* m2,
+                            int tile0) {
         while (ok && cn < limit) {
           if (cn >= SC &&
               !mbar_wait_sleep(&code_empty[cs], cph ^ 1u, abort_flag, status, kDevTimeoutEmpty)) {
             ok = false;
             break;
           }
-          load_codes(cn, cs);
+          load_codes(cn, cs, m1, m2, tile0);
           ++cn;
           if (++cs == SC) {
             cs = 0;
@@ -346,9 +348,20 @@ __global__ void __maxnreg__(64)
         }
       };
       // every index tile, as the decoders free stages; the Xq tiles, which
-      // come from the preceding kernel, have a producer of their own
+      // come from the preceding kernel, have a producer of their own.  The
+      // run is walked matrix by matrix with constant indices into the maps:
+      // a TMA given a tensor map at a run-time offset into the parameters is
+      // markedly slower per copy.
       if (!early_codes) grid_dep_wait();
-      next_codes(nu);
+#pragma unroll
+      for (int jj = 0; jj < kMaxGroup; ++jj) {
+        if (jj < grp.count) {
+          const int end_tile = jj + 1 < grp.count ? grp.mat[jj + 1 < kMaxGroup ? jj + 1 : jj].tile0
+                                                  : grp.tiles;
+          const int64_t lim = (int64_t)end_tile * kunits - u_begin;
+          next_codes(lim < nu ? (int)lim : nu, &maps.I1[jj], &maps.I2[jj], grp.mat[jj].tile0);
+        }
+      }
       if (ld_shared_volatile(abort_flag)) {
         // let the copies in flight land before the CTA exits (bounded waits:
         // a stage's barrier may never complete once the other roles stopped)
@@ -435,23 +448,34 @@ __global__ void __maxnreg__(64)
     if (lane == 0) {
       grid_dep_wait();
       int sa = 0;                    // operand stage of unit i
-      for (int i = 0; i < nu; ++i) {
-        // the Xq stage of unit i was last read by the MMAs of unit i - SX, and
-        // the operand stage's barrier must have completed the phase of unit
-        // i - SA before this unit's arrival (the two issuers' MMAs, of
-        // alternate units, complete in no fixed order)
-        if (i >= SX && !mbar_wait_sleep(&a_empty[(i - SX) % SA], (uint32_t)((i - SX) / SA) & 1u,
-                                        abort_flag, status, kDevTimeoutEmpty))
-          break;
-        if (i >= SA && !mbar_wait_sleep(&a_empty[(i - SA) % SA], (uint32_t)((i - SA) / SA) & 1u,
-                                        abort_flag, status, kDevTimeoutEmpty))
-          break;
-        const int u = u_begin + i;
-        const int j = sk_mat_of(grp, u / kunits);
-        mbar_arrive_expect_tx(&full_a[sa], (uint32_t)plan.b_bytes);
-        tma_load_2d(xq_ring + (i % SX) * plan.b_bytes, &maps.B[0] + j, &full_a[sa],
-                    (u % kunits) * KU, 0);
-        if (++sa == SA) sa = 0;
+      int i = 0;
+#pragma unroll
+      for (int jj = 0; jj < kMaxGroup; ++jj) {
+        if (jj >= grp.count) break;
+        // the units of matrix jj, with its map at a constant index (see the
+        // index producer)
+        const int end_tile = jj + 1 < grp.count ? grp.mat[jj + 1 < kMaxGroup ? jj + 1 : jj].tile0
+                                                : grp.tiles;
+        const int64_t lim64 = (int64_t)end_tile * kunits - u_begin;
+        const int lim = lim64 < nu ? (int)lim64 : nu;
+        const CUtensorMap* mb = &maps.B[jj];
+        for (; i < lim; ++i) {
+          // the Xq stage of unit i was last read by the MMAs of unit i - SX, and
+          // the operand stage's barrier must have completed the phase of unit
+          // i - SA before this unit's arrival (the two issuers' MMAs, of
+          // alternate units, complete in no fixed order)
+          if (i >= SX && !mbar_wait_sleep(&a_empty[(i - SX) % SA], (uint32_t)((i - SX) / SA) & 1u,
+                                          abort_flag, status, kDevTimeoutEmpty))
+            break;
+          if (i >= SA && !mbar_wait_sleep(&a_empty[(i - SA) % SA], (uint32_t)((i - SA) / SA) & 1u,
+                                          abort_flag, status, kDevTimeoutEmpty))
+            break;
+          const int u = u_begin + i;
+          mbar_arrive_expect_tx(&full_a[sa], (uint32_t)plan.b_bytes);
+          tma_load_2d(xq_ring + (i % SX) * plan.b_bytes, mb, &full_a[sa], (u % kunits) * KU, 0);
+          if (++sa == SA) sa = 0;
+        }
+        if (i < lim) break;   // a wait gave up
       }
       if (ld_shared_volatile(abort_flag)) {
         // let the copies in flight land before the CTA exits
@@ -464,8 +488,7 @@ __global__ void __maxnreg__(64)
     // ------------------------------------------------------------ decoders
     const int dw = warp - 2;
     const int q = warp & 3;
-    const int p = dw >> 2;
-    const int dg = p >> 1, h = p & 1;
+    const int dg = dw >> 2;
     const int r = q * 32 + lane;
     const uint32_t lane_bits = (uint32_t)(q * 32) << 16;
     bool ok = mbar_wait_sleep(table_full, 0, abort_flag, status, kDevTimeoutFull);
@@ -474,14 +497,18 @@ __global__ void __maxnreg__(64)
     for (int i = dg; i < nu && ok; i += DEC_GROUPS) {
       if (!mbar_wait_sleep(&full_code[cs], cph, abort_flag, status, kDevTimeoutFull)) break;
       const uint8_t* si1 = code_ring + cs * plan.code_bytes;
-      const uint4 c1 = *reinterpret_cast<const uint4*>(si1 + sw32_off(r, h));
-      uint4 c2 = make_uint4(0u, 0u, 0u, 0u);
-      if (BPW == 4) {
-        c2 = *reinterpret_cast<const uint4*>(si1 + I1_BYTES + sw32_off(r, h));
-      } else if (BPW == 3) {
-        const uint2 c = *reinterpret_cast<const uint2*>(si1 + I1_BYTES + r * 16 + h * 8);
-        c2 = make_uint4(__byte_perm(c.x, 0u, 0x4140), __byte_perm(c.x, 0u, 0x4342),
-                        __byte_perm(c.y, 0u, 0x4140), __byte_perm(c.y, 0u, 0x4342));
+      uint4 c1h[2], c2h[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        c1h[h] = *reinterpret_cast<const uint4*>(si1 + sw32_off(r, h));
+        c2h[h] = make_uint4(0u, 0u, 0u, 0u);
+        if (BPW == 4) {
+          c2h[h] = *reinterpret_cast<const uint4*>(si1 + I1_BYTES + sw32_off(r, h));
+        } else if (BPW == 3) {
+          const uint2 c = *reinterpret_cast<const uint2*>(si1 + I1_BYTES + r * 16 + h * 8);
+          c2h[h] = make_uint4(__byte_perm(c.x, 0u, 0x4140), __byte_perm(c.x, 0u, 0x4342),
+                              __byte_perm(c.y, 0u, 0x4140), __byte_perm(c.y, 0u, 0x4342));
+        }
       }
       // the indices are in registers: the index-tile stage can be refilled
       // once these shared-memory reads are ordered before the next bulk copy
@@ -493,19 +520,24 @@ __global__ void __maxnreg__(64)
           !mbar_wait_sleep(&a_empty[as], aph ^ 1u, abort_flag, status, kDevTimeoutMma))
         break;
       tc_fence_after();
-      const uint32_t w1[4] = {c1.x, c1.y, c1.z, c1.w};
-      const uint32_t w2[4] = {c2.x, c2.y, c2.z, c2.w};
-      uint32_t v[16];
+      // the two halves of the row's 16 groups, 16 TMEM columns each
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const uint32_t ea0 = sk_entry(table, sk_off_lo(w1[k]));
-        const uint32_t ea1 = sk_entry(table, sk_off_hi(w1[k]));
-        const uint32_t eb0 = BPW > 2 ? sk_entry(table, sk_off_lo(w2[k])) : 0u;
-        const uint32_t eb1 = BPW > 2 ? sk_entry(table, sk_off_hi(w2[k])) : 0u;
-        decode_group_q8<BPW>(w1[k] & 0xFFFFu, w2[k] & 0xFFFFu, ea0, eb0, v[4 * k], v[4 * k + 1]);
-        decode_group_q8<BPW>(w1[k] >> 16, w2[k] >> 16, ea1, eb1, v[4 * k + 2], v[4 * k + 3]);
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t w1[4] = {c1h[h].x, c1h[h].y, c1h[h].z, c1h[h].w};
+        const uint32_t w2[4] = {c2h[h].x, c2h[h].y, c2h[h].z, c2h[h].w};
+        uint32_t v[16];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t ea0 = sk_entry(table, sk_off_lo(w1[k]));
+          const uint32_t ea1 = sk_entry(table, sk_off_hi(w1[k]));
+          const uint32_t eb0 = BPW > 2 ? sk_entry(table, sk_off_lo(w2[k])) : 0u;
+          const uint32_t eb1 = BPW > 2 ? sk_entry(table, sk_off_hi(w2[k])) : 0u;
+          decode_group_q8<BPW>(w1[k] & 0xFFFFu, w2[k] & 0xFFFFu, ea0, eb0, v[4 * k],
+                               v[4 * k + 1]);
+          decode_group_q8<BPW>(w1[k] >> 16, w2[k] >> 16, ea1, eb1, v[4 * k + 2], v[4 * k + 3]);
+        }
+        sk_tmem_st16(tmem_a + lane_bits + (uint32_t)as * A_COLS + (uint32_t)(h * 16), v);
       }
-      sk_tmem_st16(tmem_a + lane_bits + (uint32_t)as * A_COLS + (uint32_t)(h * 16), v);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -533,6 +565,39 @@ __global__ void __maxnreg__(64)
         s_sc[32 * j + lane] = lane < M ? mt.alpha * __ldg(mt.tok_scale + lane) : 0.0f;
       }
     }
+    // Sums of the Xq rows over the K units [ku_lo, ku_hi) of segment sg: the
+    // bias its partial product carries.  Warp EPI_WARP0 computes those of the
+    // next segment while the current one is still being decoded, into a ring
+    // of three buffers (one being read, one being written, one that slow
+    // warps may still read for the previous segment until the barrier).
+    auto seg_sums = [&](int sg) {
+      const int slo = sg == 0 ? 0 : kunits - ku_first + (sg - 1) * kunits;
+      const int slen = kunits - (sg == 0 ? ku_first : 0);
+      const int shi = slo + slen < nu ? slo + slen : nu;
+      const int tl = first_tile + sg;
+      const int32_t* src = grp.mat[sk_mat_of(grp, tl)].colsum;
+      const int ku_lo = u_begin + slo - tl * kunits, ku_hi = u_begin + shi - tl * kunits;
+      int a0 = 0, a1 = 0;
+      for (int ku = ku_lo; ku < ku_hi; ku += 8) {
+        int v0[8], v1[8];   // eight independent loads in flight
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const bool in = ku + j < ku_hi;
+          const int32_t* p = src + (size_t)(ku + j) * rows_b;
+          v0[j] = in && lane < rows_b ? __ldg(p + lane) : 0;
+          v1[j] = in && 32 + lane < rows_b ? __ldg(p + 32 + lane) : 0;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          a0 += v0[j];
+          a1 += v1[j];
+        }
+      }
+      int32_t* dst = s_cs + 64 * (sg % 3);
+      dst[lane] = a0;
+      dst[32 + lane] = a1;
+    };
+    if (warp == EPI_WARP0 && nseg > 0) seg_sums(0);
     // every epilogue thread runs the same sequence of named barriers, also
     // after a failed wait (it then only skips the work)
     bool ok = true;
@@ -546,22 +611,11 @@ __global__ void __maxnreg__(64)
       const bool has1 = hi - lo >= 2 || (lo & 1) == 1;
       const int tile = first_tile + seg;
       const int mj = sk_mat_of(grp, tile);
-      // sums of the Xq rows over the segment's K units [ku_lo, ku_hi): the
-      // bias this partial product carries (double-buffered by segment parity:
-      // the other buffer may still be read for the previous segment)
-      int32_t* cs = s_cs + 64 * b;
-      if (warp == EPI_WARP0) {
-        const int ku_lo = u_begin + lo - tile * kunits, ku_hi = u_begin + hi - tile * kunits;
-        const int32_t* src = grp.mat[mj].colsum;
-        int a0 = 0, a1 = 0;
-        for (int ku = ku_lo; ku < ku_hi; ++ku) {
-          if (lane < rows_b) a0 += __ldg(src + (size_t)ku * rows_b + lane);
-          if (32 + lane < rows_b) a1 += __ldg(src + (size_t)ku * rows_b + 32 + lane);
-        }
-        cs[lane] = a0;
-        cs[32 + lane] = a1;
-      }
+      if (warp == EPI_WARP0 && seg + 1 < nseg) seg_sums(seg + 1);
+      // the barrier publishes the sums of this segment (written one segment
+      // earlier) and the steps
       asm volatile("bar.sync 1, 128;" ::: "memory");
+      const int32_t* cs = s_cs + 64 * (seg % 3);
       lo = hi;
       ok = ok && mbar_wait_sleep(&acc_full[b], (uint32_t)(seg >> 1) & 1u, abort_flag, status,
                                  kDevTimeoutMma);
@@ -622,7 +676,12 @@ __global__ void __maxnreg__(64)
         fence_proxy_async_smem();
         asm volatile("bar.sync 1, 128;" ::: "memory");
         if (issuer && ok) {
-          tma_reduce_add_2d(&maps.Y[0] + mj, smem_u32(s_y), (tile - grp.mat[mj].tile0) * ROWS, 0);
+          const int ty = (tile - grp.mat[mj].tile0) * ROWS;
+          // constant map indices (see the index producer)
+          if (mj == 0) tma_reduce_add_2d(&maps.Y[0], smem_u32(s_y), ty, 0);
+          else if (mj == 1) tma_reduce_add_2d(&maps.Y[1], smem_u32(s_y), ty, 0);
+          else if (mj == 2) tma_reduce_add_2d(&maps.Y[2], smem_u32(s_y), ty, 0);
+          else tma_reduce_add_2d(&maps.Y[3], smem_u32(s_y), ty, 0);
           bulk_wait_read_all();
         }
         asm volatile("bar.sync 1, 128;" ::: "memory");
