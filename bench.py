@@ -210,6 +210,9 @@ def run_ours(args):
     if args.profile == "decode":
         _profile_decode(e8, dev)
         return
+    if args.profile in ("dense_up", "dense_out", "encode", "gemm_mlp"):
+        _profile_other(e8, synth, dev, args.profile)
+        return
     peaks = _peaks()
     lay = synth.workloads()[WORKLOAD].layers[0]
     N, K, bpw = lay.N, lay.K, lay.bpw
@@ -424,6 +427,49 @@ def _profile_decode(e8, dev):
     if e8.e8_sync_status(cb) != 0:
         raise RuntimeError("decoder reported a device error")
     print("profile decodes done", flush=True)
+    cb.free()
+
+
+def _profile_other(e8, synth, dev, mode):
+    """Small workloads for ncu captures of one kernel each (a few hundred MB on
+    the device at most):
+      dense_up   prefill GEMM of the MLP up-projection (14336 x 4096, 3 bpw,
+                 4096 tokens): decode to bf16, then k_dense_gemm, twice
+      dense_out  the same for the DiT out projection (3072 x 3072, 4 bpw)
+      encode     two encodes of the 4096 x 4096 Llama layer at 4 bpw
+      gemm_mlp   three small-batch products (16 tokens) of a 14336 x 4096
+                 matrix at 4 bpw on pre-transformed activations (k_gemm_q8)"""
+    import torch
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(7)
+    cb = e8.Codebook(dev.index)
+    if mode.startswith("dense"):
+        M, N, K, bpw = (4096, 14336, 4096, 3) if mode == "dense_up" else (4096, 3072, 3072, 4)
+        c1, c2 = _random_codes(torch, dev, N, K, bpw, gen)
+        X = torch.randn((M, K), generator=gen, device=dev).to(torch.bfloat16)
+        ws = torch.empty(e8.e8_workspace_bytes(e8.E8_GEMM_DECODED_W, M, N, K, bpw),
+                         dtype=torch.uint8, device=dev)
+        for _ in range(2):
+            e8.e8_gemm(cb, X, c1, c2, N, K, bpw, 1, 0.02, mode=e8.E8_GEMM_DECODED_W, workspace=ws)
+    elif mode == "encode":
+        lay = synth.workloads()[WORKLOAD].layers[0]
+        W = synth.gaussian_weights(lay.N, lay.K, lay.std, lay.w_seed)
+        s = synth.suggest_scale(W, lay.bpw)
+        Wd = torch.from_numpy(W).to(dev)
+        for _ in range(2):
+            e8.e8_encode(cb, Wd, lay.bpw, lay.rht_seed, s)
+    else:
+        M, N, K, bpw = 16, 14336, 4096, 4
+        codes = [_random_codes(torch, dev, N, K, bpw, gen) for _ in range(3)]
+        X = torch.randn((M, K), generator=gen, device=dev).to(torch.bfloat16)
+        xq = e8.e8_act_rht_q8(X, 2)
+        Y = torch.zeros((M, N), device=dev)
+        for c1, c2 in codes:
+            e8.e8_gemm_xt(cb, xq, M, c1, c2, N, K, bpw, 0.02, Y=Y)
+    torch.cuda.synchronize()
+    if e8.e8_sync_status(cb) != 0:
+        raise RuntimeError("a kernel reported a device error")
+    print("profile %s done" % mode, flush=True)
     cb.free()
 
 
@@ -745,10 +791,12 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-load", action="store_true",
                     help="skip the load phase that precedes the timed region (clock record)")
-    ap.add_argument("--profile", nargs="?", const="gemm", choices=["gemm", "decode"],
-                    help="run 8 eager steps of the headline call (gemm) or 3 bf16 decodes "
-                         "of the 14336 x 4096 MLP up-projection at 4 bpw (decode), then exit "
-                         "(ncu captures)")
+    ap.add_argument("--profile", nargs="?", const="gemm",
+                    choices=["gemm", "decode", "dense_up", "dense_out", "encode", "gemm_mlp"],
+                    help="small runs for ncu captures, then exit: 8 eager steps of the "
+                         "headline call (gemm), 3 bf16 decodes of a 14336 x 4096 matrix "
+                         "(decode), prefill GEMMs (dense_up, dense_out), two encodes "
+                         "(encode), small-batch products of a 14336 x 4096 matrix (gemm_mlp)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
