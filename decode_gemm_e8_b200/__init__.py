@@ -30,6 +30,8 @@ EXPORTED = ("e8_codebook_build", "e8_codebook_free", "e8_codebook_export", "e8_r
             "e8_gemm", "e8_gemm_xt",
             "e8_gemm_xt_rows", "e8_gemm_act_noalloc", "e8_gemm_host",
             "e8_gemm_grouped", "e8_gemm_grouped_workspace_bytes",
+            "e8_rht_forward_nh", "e8_encode_nh", "e8_decode_to_bf16_nh", "e8_gemm_nh",
+            "e8_workspace_bytes_nh",
             "e8_gemm_host_workspace_bytes", "e8_gemm_auto_mode",
             "e8_workspace_bytes", "e8_sync_status", "e8_debug_wait_timeout", "e8_status_str",
             "e8_version")
@@ -74,6 +76,14 @@ def load_library(path: str = LIB_PATH):
         "e8_gemm_host_workspace_bytes": ([c.c_int, I64, I64, I64, c.c_int], c.c_size_t),
         "e8_gemm_auto_mode": ([I64, I64, I64, c.c_int], c.c_int),
         "e8_gemm_grouped": ([P, P, I64, I64, c.c_int, P, c.c_int, P, c.c_size_t, P], c.c_int),
+        "e8_rht_forward_nh": ([P, P, I64, I64, I64, U64, c.c_float, P, P], c.c_int),
+        "e8_encode_nh": ([P, P, I64, I64, I64, c.c_int, U64, c.c_float, P, P, P, c.c_size_t, P],
+                         c.c_int),
+        "e8_decode_to_bf16_nh": ([P, P, P, I64, I64, I64, c.c_int, U64, c.c_float, P, P],
+                                 c.c_int),
+        "e8_gemm_nh": ([P, P, I64, P, P, I64, I64, I64, c.c_int, U64, c.c_float, P, c.c_int, P,
+                        c.c_size_t, P], c.c_int),
+        "e8_workspace_bytes_nh": ([c.c_int, I64, I64, I64, I64, c.c_int], c.c_size_t),
         "e8_gemm_grouped_workspace_bytes": ([I64, I64, c.c_int, c.c_int], c.c_size_t),
         "e8_workspace_bytes": ([c.c_int, I64, I64, I64, c.c_int], c.c_size_t),
         "e8_sync_status": ([P, P], c.c_int),
@@ -167,18 +177,27 @@ def e8_codebook_export(cb: Codebook):
     return out
 
 
-def e8_rht_forward(cb: Codebook, W, rht_seed: int, scale: float, U=None, stream=None):
+def e8_rht_forward(cb: Codebook, W, rht_seed: int, scale: float, U=None, stream=None, nh=None):
+    """nh: explicit Hadamard block (e8_rht_forward_nh); None for the default."""
     import torch
     N, K = W.shape
     if U is None:
         U = torch.empty_like(W)
-    _check(load_library().e8_rht_forward(cb.handle, _ptr(W), N, K, int(rht_seed) & (2**64 - 1),
-                                         float(scale), _ptr(U), _stream(stream)),
-           "e8_rht_forward")
+    lib = load_library()
+    if nh is None:
+        rc = lib.e8_rht_forward(cb.handle, _ptr(W), N, K, int(rht_seed) & (2**64 - 1),
+                                float(scale), _ptr(U), _stream(stream))
+    else:
+        rc = lib.e8_rht_forward_nh(cb.handle, _ptr(W), N, K, int(nh), int(rht_seed) & (2**64 - 1),
+                                   float(scale), _ptr(U), _stream(stream))
+    _check(rc, "e8_rht_forward")
     return U
 
 
-def e8_workspace_bytes(op: int, M: int, N: int, K: int, bpw: int) -> int:
+def e8_workspace_bytes(op: int, M: int, N: int, K: int, bpw: int, nh=None) -> int:
+    if nh is not None:
+        return int(load_library().e8_workspace_bytes_nh(int(op), int(M), int(N), int(K), int(nh),
+                                                        int(bpw)))
     return int(load_library().e8_workspace_bytes(int(op), int(M), int(N), int(K), int(bpw)))
 
 
@@ -194,8 +213,9 @@ def _workspace(nbytes: int, device, workspace=None):
 
 
 def e8_encode(cb: Codebook, W, bpw: int, rht_seed: int, scale: float, idx1=None, idx2=None,
-              workspace=None, stream=None):
-    """W fp32 [N, K] (CUDA) -> (idx1 uint16 [N, K/8], idx2 uint8/uint16 [N, K/8] or None)."""
+              workspace=None, stream=None, nh=None):
+    """W fp32 [N, K] (CUDA) -> (idx1 uint16 [N, K/8], idx2 uint8/uint16 [N, K/8] or None).
+    nh: explicit Hadamard block (e8_encode_nh); None for the default."""
     import torch
     N, K = W.shape
     dev = W.device
@@ -205,21 +225,36 @@ def e8_encode(cb: Codebook, W, bpw: int, rht_seed: int, scale: float, idx1=None,
         idx2 = torch.empty((N, K // 8), dtype=torch.uint8 if bpw == 3 else torch.uint16, device=dev)
     need = e8_workspace_bytes(E8_OP_ENCODE, 0, N, K, bpw)
     ws = _workspace(need, dev, workspace)
-    _check(load_library().e8_encode(cb.handle, _ptr(W), N, K, int(bpw), int(rht_seed) & (2**64 - 1),
-                                    float(scale), _ptr(idx1), _ptr(idx2), _ptr(ws), ws.numel(),
-                                    _stream(stream)), "e8_encode")
+    lib = load_library()
+    if nh is None:
+        rc = lib.e8_encode(cb.handle, _ptr(W), N, K, int(bpw), int(rht_seed) & (2**64 - 1),
+                           float(scale), _ptr(idx1), _ptr(idx2), _ptr(ws), ws.numel(),
+                           _stream(stream))
+    else:
+        rc = lib.e8_encode_nh(cb.handle, _ptr(W), N, K, int(nh), int(bpw),
+                              int(rht_seed) & (2**64 - 1), float(scale), _ptr(idx1), _ptr(idx2),
+                              _ptr(ws), ws.numel(), _stream(stream))
+    _check(rc, "e8_encode")
     return idx1, idx2
 
 
 def e8_decode_to_bf16(cb: Codebook, idx1, idx2, N: int, K: int, bpw: int, rht_seed: int,
-                      scale: float, out=None, stream=None):
-    """Decoded weights, torch.bfloat16 [N, K] on the device of idx1."""
+                      scale: float, out=None, stream=None, nh=None):
+    """Decoded weights, torch.bfloat16 [N, K] on the device of idx1.
+    nh: explicit Hadamard block (e8_decode_to_bf16_nh); None for the default."""
     import torch
     if out is None:
         out = torch.empty((N, K), dtype=torch.bfloat16, device=idx1.device)
-    _check(load_library().e8_decode_to_bf16(cb.handle, _ptr(idx1), _ptr(idx2), N, K, int(bpw),
-                                            int(rht_seed) & (2**64 - 1), float(scale), _ptr(out),
-                                            _stream(stream)), "e8_decode_to_bf16")
+    lib = load_library()
+    if nh is None:
+        rc = lib.e8_decode_to_bf16(cb.handle, _ptr(idx1), _ptr(idx2), N, K, int(bpw),
+                                   int(rht_seed) & (2**64 - 1), float(scale), _ptr(out),
+                                   _stream(stream))
+    else:
+        rc = lib.e8_decode_to_bf16_nh(cb.handle, _ptr(idx1), _ptr(idx2), N, K, int(nh), int(bpw),
+                                      int(rht_seed) & (2**64 - 1), float(scale), _ptr(out),
+                                      _stream(stream))
+    _check(rc, "e8_decode_to_bf16")
     return out
 
 
@@ -236,8 +271,9 @@ def e8_act_rht(X, rht_seed: int, rows: int | None = None, out=None, stream=None)
 
 
 def e8_gemm(cb: Codebook, X, idx1, idx2, N: int, K: int, bpw: int, rht_seed: int, scale: float,
-            mode: int = E8_GEMM_AUTO, Y=None, workspace=None, stream=None):
-    """Y fp32 [M, N] = X bf16 [M, K] times the decoded weights transposed."""
+            mode: int = E8_GEMM_AUTO, Y=None, workspace=None, stream=None, nh=None):
+    """Y fp32 [M, N] = X bf16 [M, K] times the decoded weights transposed.
+    nh: explicit Hadamard block (e8_gemm_nh); None for the default."""
     import torch
     M = X.shape[0]
     dev = X.device
@@ -245,10 +281,17 @@ def e8_gemm(cb: Codebook, X, idx1, idx2, N: int, K: int, bpw: int, rht_seed: int
         Y = torch.empty((M, N), dtype=torch.float32, device=dev)
     # a caller's workspace is checked by the library (E8_EWORKSPACE if too small)
     ws = workspace if workspace is not None else _workspace(
-        e8_workspace_bytes(mode, M, N, K, bpw), dev)
-    _check(load_library().e8_gemm(cb.handle, _ptr(X), M, _ptr(idx1), _ptr(idx2), N, K, int(bpw),
-                                  int(rht_seed) & (2**64 - 1), float(scale), _ptr(Y), int(mode),
-                                  _ptr(ws), ws.numel(), _stream(stream)), "e8_gemm")
+        e8_workspace_bytes(mode, M, N, K, bpw, nh), dev)
+    lib = load_library()
+    if nh is None:
+        rc = lib.e8_gemm(cb.handle, _ptr(X), M, _ptr(idx1), _ptr(idx2), N, K, int(bpw),
+                         int(rht_seed) & (2**64 - 1), float(scale), _ptr(Y), int(mode),
+                         _ptr(ws), ws.numel(), _stream(stream))
+    else:
+        rc = lib.e8_gemm_nh(cb.handle, _ptr(X), M, _ptr(idx1), _ptr(idx2), N, K, int(nh),
+                            int(bpw), int(rht_seed) & (2**64 - 1), float(scale), _ptr(Y),
+                            int(mode), _ptr(ws), ws.numel(), _stream(stream))
+    _check(rc, "e8_gemm")
     return Y
 
 

@@ -208,9 +208,9 @@ __global__ void __launch_bounds__(512) k_act_rht_fast(const uint16_t* __restrict
 }
 
 cudaError_t launch_act_rht(const uint16_t* X, int64_t M, int64_t K, uint64_t seed, uint16_t* Xt,
-                           int64_t rows, cudaStream_t st, int pdl) {
+                           int64_t rows, cudaStream_t st, int pdl, int64_t nh_arg) {
   {
-    const int nh = (int)hadamard_block(K);
+    const int nh = (int)resolve_nh(K, nh_arg);
     if (nh >= 256 && nh <= 4096) {
       const int64_t data = M * K / nh;
       const int64_t pad_elems = (rows - 2 * M) * K;
@@ -231,7 +231,7 @@ cudaError_t launch_act_rht(const uint16_t* X, int64_t M, int64_t K, uint64_t see
       return cudaGetLastError();
     }
   }
-  const int nh = (int)hadamard_block(K);
+  const int nh = (int)resolve_nh(K, nh_arg);
   const int epc = nh < 2048 ? 2048 : nh;
   const int64_t total = M * K;
   const int64_t ctas = (total + epc - 1) / epc;
@@ -500,8 +500,9 @@ __global__ void __launch_bounds__(512, 4) k_act_q8(const uint16_t* __restrict__ 
 }
 
 cudaError_t launch_act_q8_group(const uint16_t* X, int64_t M, int64_t K, const ActQ8Out* outs,
-                                int count, int64_t rows, cudaStream_t st, int pdl) {
-  const int nh = (int)hadamard_block(K);
+                                int count, int64_t rows, cudaStream_t st, int pdl,
+                                int64_t nh_arg) {
+  const int nh = (int)resolve_nh(K, nh_arg);
   if (nh < 256 || nh > 4096 || K > 32768 || M < 1 || M > 32 || rows < 2 * M || rows > 64 ||
       count < 1 || count > kMaxGroup)
     return cudaErrorInvalidValue;
@@ -542,7 +543,7 @@ cudaError_t launch_act_q8_group(const uint16_t* X, int64_t M, int64_t K, const A
 
 cudaError_t launch_act_q8(const uint16_t* X, int64_t M, int64_t K, uint64_t seed, int8_t* Xq,
                           float* scales, int32_t* colsum, int64_t rows, cudaStream_t st,
-                          int pdl, float* Yz, int64_t yz_elems) {
+                          int pdl, float* Yz, int64_t yz_elems, int64_t nh) {
   ActQ8Out o;
   o.seed = seed;
   o.Xq = Xq;
@@ -550,7 +551,7 @@ cudaError_t launch_act_q8(const uint16_t* X, int64_t M, int64_t K, uint64_t seed
   o.colsum = colsum;
   o.Yz = Yz;
   o.yz_elems = yz_elems;
-  return launch_act_q8_group(X, M, K, &o, 1, rows, st, pdl);
+  return launch_act_q8_group(X, M, K, &o, 1, rows, st, pdl, nh);
 }
 
 }  // namespace e8

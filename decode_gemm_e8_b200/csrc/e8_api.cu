@@ -46,16 +46,16 @@ cudaError_t ensure_smem_limit_ptr(const void* kernel, int bytes, bool carveout_m
   return e;
 }
 
-size_t act_scratch_bytes(int64_t M, int64_t K, int smem_variant) {
+size_t act_scratch_bytes(int64_t M, int64_t K, int smem_variant, int64_t nh) {
   const int64_t rows = (2 * M + 15) / 16 * 16;
-  if (!smem_variant && q8_eligible(M, K)) return q8_layout(M, K, rows).total;
+  if (!smem_variant && q8_eligible(M, K, nh)) return q8_layout(M, K, rows).total;
   return (((size_t)rows * (size_t)K * 2) + 255) & ~size_t(255);
 }
 
 cudaError_t run_act_gemm(const e8_codebook* cb, const uint16_t* X, int64_t M,
                          const uint16_t* idx1, const void* idx2, int64_t N, int64_t K, int bpw,
                          uint64_t seed, float alpha, float* Y, int smem_variant, void* scratch,
-                         cudaStream_t st) {
+                         cudaStream_t st, int64_t nh) {
   DeviceCodebook d;
   d.vecs = cb->vecs;
   d.table = cb->table;
@@ -66,7 +66,7 @@ cudaError_t run_act_gemm(const e8_codebook* cb, const uint16_t* X, int64_t M,
   d.clist_len = cb->clist_len;
   d.status = cb->status;
   const int rows = (int)((2 * M + 15) / 16 * 16);
-  if (!smem_variant && q8_eligible(M, K)) {
+  if (!smem_variant && q8_eligible(M, K, nh)) {
     const Q8Layout l = q8_layout(M, K, rows);
     uint8_t* buf = static_cast<uint8_t*>(scratch);
     ActQ8Args a;
@@ -87,12 +87,12 @@ cudaError_t run_act_gemm(const e8_codebook* cb, const uint16_t* X, int64_t M,
     cudaError_t e = launch_act_q8(X, M, K, seed, reinterpret_cast<int8_t*>(buf),
                                   reinterpret_cast<float*>(buf + l.scales_off),
                                   reinterpret_cast<int32_t*>(buf + l.colsum_off), rows, st, 1, Y,
-                                  M * N);
+                                  M * N, nh);
     if (e != cudaSuccess) return e;
     return launch_act_gemm_q8(d, a, cb->sm_count, st);
   }
   uint16_t* Xt = static_cast<uint16_t*>(scratch);
-  cudaError_t e = launch_act_rht(X, M, K, seed, Xt, rows, st, 0);
+  cudaError_t e = launch_act_rht(X, M, K, seed, Xt, rows, st, 0, nh);
   if (e != cudaSuccess) return e;
   ActGemmArgs a;
   a.Xt = Xt;
@@ -259,39 +259,48 @@ int e8_codebook_export(const e8_codebook* cb, int8_t* host_vecs) {
   return cuda_status(e);
 }
 
-int e8_rht_forward(const e8_codebook* cb, const float* W, int64_t N, int64_t K,
-                   uint64_t rht_seed, float scale, float* U, void* stream) {
+int e8_rht_forward_nh(const e8_codebook* cb, const float* W, int64_t N, int64_t K, int64_t nh,
+                      uint64_t rht_seed, float scale, float* U, void* stream) {
   (void)cudaGetLastError();  // a failed earlier launch must not be reported here
   int rc = check_device(cb);
   if (rc != E8_OK) return rc;
-  if (N < 0 || !valid_k(K) || !(scale > 0.0f) || !std::isfinite(scale)) return E8_EINVAL;
+  if (N < 0 || !valid_k(K) || !e8::valid_nh(K, nh) || !e8::valid_scale(scale)) return E8_EINVAL;
   if (N == 0) return E8_OK;
   if (!W || !U || !aligned16(W) || !aligned16(U) || W == U) return E8_EINVAL;
-  const int64_t nh = e8::hadamard_block(K);
-  cudaError_t e = e8::launch_encode(dev_view(cb), W, N, K, 2, rht_seed, gamma_of(scale, nh),
+  const int64_t nb = e8::resolve_nh(K, nh);
+  cudaError_t e = e8::launch_encode(dev_view(cb), W, N, K, 2, rht_seed, gamma_of(scale, nb),
                                     nullptr, nullptr, nullptr, nullptr, 0, U, 0, cb->sm_count,
-                                    (cudaStream_t)stream);
+                                    (cudaStream_t)stream, nb);
   return cuda_status(e);
 }
 
-size_t e8_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int bpw) {
-  if (!valid_bpw(bpw) || N < 0 || M < 0 || !valid_k(K)) return 0;
+int e8_rht_forward(const e8_codebook* cb, const float* W, int64_t N, int64_t K,
+                   uint64_t rht_seed, float scale, float* U, void* stream) {
+  return e8_rht_forward_nh(cb, W, N, K, 0, rht_seed, scale, U, stream);
+}
+
+size_t e8_workspace_bytes_nh(int op, int64_t M, int64_t N, int64_t K, int64_t nh, int bpw) {
+  if (!valid_bpw(bpw) || N < 0 || M < 0 || !valid_k(K) || !e8::valid_nh(K, nh)) return 0;
   const size_t G = (size_t)N * (size_t)(K / 8);
   switch (op) {
     case E8_OP_ENCODE:
       return 256 + 2 * G * sizeof(e8::WorkItem);
     case E8_GEMM_AUTO:
-      return e8_workspace_bytes(e8_gemm_auto_mode(M, N, K, bpw), M, N, K, bpw);
+      return e8_workspace_bytes_nh(e8_gemm_auto_mode(M, N, K, bpw), M, N, K, nh, bpw);
     case E8_GEMM_ACT_RHT:
-      return e8::act_scratch_bytes(M, K, 0);
+      return e8::act_scratch_bytes(M, K, 0, nh);
     case E8_GEMM_ACT_RHT_SMEM:
-      return e8::act_scratch_bytes(M, K, 1);
+      return e8::act_scratch_bytes(M, K, 1, nh);
     case E8_GEMM_DECODED_W:
     case E8_GEMM_SIMT:
       return round256((size_t)N * (size_t)K * 2);
     default:
       return 0;
   }
+}
+
+size_t e8_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int bpw) {
+  return e8_workspace_bytes_nh(op, M, N, K, 0, bpw);
 }
 
 int e8_gemm_auto_mode(int64_t M, int64_t N, int64_t K, int bpw) {
@@ -301,13 +310,14 @@ int e8_gemm_auto_mode(int64_t M, int64_t N, int64_t K, int bpw) {
   return E8_GEMM_DECODED_W;
 }
 
-int e8_encode(const e8_codebook* cb, const float* W, int64_t N, int64_t K, int bpw,
-              uint64_t rht_seed, float scale, uint16_t* idx1, void* idx2, void* workspace,
-              size_t ws_bytes, void* stream) {
+int e8_encode_nh(const e8_codebook* cb, const float* W, int64_t N, int64_t K, int64_t nh,
+                 int bpw, uint64_t rht_seed, float scale, uint16_t* idx1, void* idx2,
+                 void* workspace, size_t ws_bytes, void* stream) {
   (void)cudaGetLastError();  // a failed earlier launch must not be reported here
   int rc = check_device(cb);
   if (rc != E8_OK) return rc;
-  if (N < 0 || !valid_k(K) || !valid_bpw(bpw) || !(scale > 0.0f) || !std::isfinite(scale))
+  if (N < 0 || !valid_k(K) || !e8::valid_nh(K, nh) || !valid_bpw(bpw) ||
+      !e8::valid_scale(scale))
     return E8_EINVAL;
   if ((bpw == 2) != (idx2 == nullptr)) return E8_EINVAL;
   if (N == 0) return E8_OK;
@@ -315,34 +325,48 @@ int e8_encode(const e8_codebook* cb, const float* W, int64_t N, int64_t K, int b
     return E8_EINVAL;
   const size_t need = e8_workspace_bytes(E8_OP_ENCODE, 0, N, K, bpw);
   if (!workspace || !aligned16(workspace) || ws_bytes < need) return E8_EWORKSPACE;
-  const int64_t nh = e8::hadamard_block(K);
+  const int64_t nb = e8::resolve_nh(K, nh);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint32_t* count = reinterpret_cast<uint32_t*>(ws);
   e8::WorkItem* items = reinterpret_cast<e8::WorkItem*>(ws + 256);
   const uint64_t cap = (uint64_t)N * (uint64_t)(K / 8);
-  cudaError_t e = e8::launch_encode(dev_view(cb), W, N, K, bpw, rht_seed, gamma_of(scale, nh),
+  cudaError_t e = e8::launch_encode(dev_view(cb), W, N, K, bpw, rht_seed, gamma_of(scale, nb),
                                     idx1, idx2, items, count, cap, nullptr, 1, cb->sm_count,
-                                    (cudaStream_t)stream);
+                                    (cudaStream_t)stream, nb);
+  return cuda_status(e);
+}
+
+int e8_encode(const e8_codebook* cb, const float* W, int64_t N, int64_t K, int bpw,
+              uint64_t rht_seed, float scale, uint16_t* idx1, void* idx2, void* workspace,
+              size_t ws_bytes, void* stream) {
+  return e8_encode_nh(cb, W, N, K, 0, bpw, rht_seed, scale, idx1, idx2, workspace, ws_bytes,
+                      stream);
+}
+
+int e8_decode_to_bf16_nh(const e8_codebook* cb, const uint16_t* idx1, const void* idx2,
+                         int64_t N, int64_t K, int64_t nh, int bpw, uint64_t rht_seed,
+                         float scale, uint16_t* W_dec, void* stream) {
+  (void)cudaGetLastError();  // a failed earlier launch must not be reported here
+  int rc = check_device(cb);
+  if (rc != E8_OK) return rc;
+  if (N < 0 || !valid_k(K) || !e8::valid_nh(K, nh) || !valid_bpw(bpw) ||
+      !e8::valid_scale(scale))
+    return E8_EINVAL;
+  if ((bpw == 2) != (idx2 == nullptr)) return E8_EINVAL;
+  if (N == 0) return E8_OK;
+  if (!idx1 || !W_dec || !aligned16(idx1) || !aligned16(W_dec) || (idx2 && !aligned16(idx2)))
+    return E8_EINVAL;
+  const int64_t nb = e8::resolve_nh(K, nh);
+  cudaError_t e = e8::launch_decode(dev_view(cb), idx1, idx2, N, K, bpw, rht_seed,
+                                    alpha_of(scale, nb, bpw), W_dec, cb->sm_count,
+                                    (cudaStream_t)stream, nb);
   return cuda_status(e);
 }
 
 int e8_decode_to_bf16(const e8_codebook* cb, const uint16_t* idx1, const void* idx2, int64_t N,
                       int64_t K, int bpw, uint64_t rht_seed, float scale, uint16_t* W_dec,
                       void* stream) {
-  (void)cudaGetLastError();  // a failed earlier launch must not be reported here
-  int rc = check_device(cb);
-  if (rc != E8_OK) return rc;
-  if (N < 0 || !valid_k(K) || !valid_bpw(bpw) || !(scale > 0.0f) || !std::isfinite(scale))
-    return E8_EINVAL;
-  if ((bpw == 2) != (idx2 == nullptr)) return E8_EINVAL;
-  if (N == 0) return E8_OK;
-  if (!idx1 || !W_dec || !aligned16(idx1) || !aligned16(W_dec) || (idx2 && !aligned16(idx2)))
-    return E8_EINVAL;
-  const int64_t nh = e8::hadamard_block(K);
-  cudaError_t e = e8::launch_decode(dev_view(cb), idx1, idx2, N, K, bpw, rht_seed,
-                                    alpha_of(scale, nh, bpw), W_dec, cb->sm_count,
-                                    (cudaStream_t)stream);
-  return cuda_status(e);
+  return e8_decode_to_bf16_nh(cb, idx1, idx2, N, K, 0, bpw, rht_seed, scale, W_dec, stream);
 }
 
 int e8_act_rht(const uint16_t* X, int64_t M, int64_t K, uint64_t rht_seed, uint16_t* Xt,
@@ -354,14 +378,14 @@ int e8_act_rht(const uint16_t* X, int64_t M, int64_t K, uint64_t rht_seed, uint1
   return cuda_status(e8::launch_act_rht(X, M, K, rht_seed, Xt, rows, (cudaStream_t)stream));
 }
 
-int e8_gemm(const e8_codebook* cb, const uint16_t* X, int64_t M, const uint16_t* idx1,
-            const void* idx2, int64_t N, int64_t K, int bpw, uint64_t rht_seed, float scale,
-            float* Y, int mode, void* workspace, size_t ws_bytes, void* stream) {
+int e8_gemm_nh(const e8_codebook* cb, const uint16_t* X, int64_t M, const uint16_t* idx1,
+               const void* idx2, int64_t N, int64_t K, int64_t nh, int bpw, uint64_t rht_seed,
+               float scale, float* Y, int mode, void* workspace, size_t ws_bytes, void* stream) {
   (void)cudaGetLastError();  // a failed earlier launch must not be reported here
   int rc = check_device(cb);
   if (rc != E8_OK) return rc;
-  if (M < 0 || N < 0 || !valid_k(K) || !valid_bpw(bpw) || !(scale > 0.0f) ||
-      !std::isfinite(scale))
+  if (M < 0 || N < 0 || !valid_k(K) || !e8::valid_nh(K, nh) || !valid_bpw(bpw) ||
+      !e8::valid_scale(scale))
     return E8_EINVAL;
   if ((bpw == 2) != (idx2 == nullptr)) return E8_EINVAL;
   if (mode == E8_GEMM_AUTO) mode = e8_gemm_auto_mode(M, N, K, bpw);
@@ -373,26 +397,33 @@ int e8_gemm(const e8_codebook* cb, const uint16_t* X, int64_t M, const uint16_t*
   if (!X || !idx1 || !Y || !aligned16(X) || !aligned16(idx1) || !aligned16(Y) ||
       (idx2 && !aligned16(idx2)))
     return E8_EINVAL;
-  const size_t need = e8_workspace_bytes(mode, M, N, K, bpw);
+  const size_t need = e8_workspace_bytes_nh(mode, M, N, K, nh, bpw);
   if (!workspace || !aligned16(workspace) || ws_bytes < need) return E8_EWORKSPACE;
   cudaStream_t st = (cudaStream_t)stream;
-  const int64_t nh = e8::hadamard_block(K);
-  const float alpha = alpha_of(scale, nh, bpw);
+  const int64_t nb = e8::resolve_nh(K, nh);
+  const float alpha = alpha_of(scale, nb, bpw);
   const e8::DeviceCodebook d = dev_view(cb);
   cudaError_t e;
   if (act) {
     e = e8::run_act_gemm(cb, X, M, idx1, idx2, N, K, bpw, rht_seed, alpha, Y,
-                         mode == E8_GEMM_ACT_RHT_SMEM ? 1 : 0, workspace, st);
+                         mode == E8_GEMM_ACT_RHT_SMEM ? 1 : 0, workspace, st, nb);
     return cuda_status(e);
   }
   uint16_t* Wd = static_cast<uint16_t*>(workspace);
-  e = e8::launch_decode(d, idx1, idx2, N, K, bpw, rht_seed, alpha, Wd, cb->sm_count, st);
+  e = e8::launch_decode(d, idx1, idx2, N, K, bpw, rht_seed, alpha, Wd, cb->sm_count, st, nb);
   if (e != cudaSuccess) return E8_ECUDA;
   if (mode == E8_GEMM_SIMT)
     e = e8::launch_simt_gemm(X, M, Wd, N, K, Y, st);
   else
     e = e8::launch_dense_gemm(X, M, Wd, N, K, Y, cb->status, cb->sm_count, st);
   return cuda_status(e);
+}
+
+int e8_gemm(const e8_codebook* cb, const uint16_t* X, int64_t M, const uint16_t* idx1,
+            const void* idx2, int64_t N, int64_t K, int bpw, uint64_t rht_seed, float scale,
+            float* Y, int mode, void* workspace, size_t ws_bytes, void* stream) {
+  return e8_gemm_nh(cb, X, M, idx1, idx2, N, K, 0, bpw, rht_seed, scale, Y, mode, workspace,
+                    ws_bytes, stream);
 }
 
 size_t e8_gemm_host_workspace_bytes(int mode, int64_t M, int64_t N, int64_t K, int bpw) {

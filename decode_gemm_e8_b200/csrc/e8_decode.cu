@@ -361,13 +361,13 @@ static int decode_fast_plan(int64_t K, int* mask_off, int* bar_off, size_t* smem
 
 cudaError_t launch_decode(const DeviceCodebook& cb, const uint16_t* idx1, const void* idx2,
                           int64_t N, int64_t K, int bpw, uint64_t seed, float alpha,
-                          uint16_t* Wdec, int sm_count, cudaStream_t st) {
+                          uint16_t* Wdec, int sm_count, cudaStream_t st, int64_t nh_arg) {
   {
     const cudaError_t e =
-        launch_decode_tc(cb, idx1, idx2, N, K, bpw, seed, alpha, Wdec, sm_count, st);
+        launch_decode_tc(cb, idx1, idx2, N, K, bpw, seed, alpha, Wdec, sm_count, st, nh_arg);
     if (e != cudaErrorNotSupported) return e;
   }
-  const int64_t nh = hadamard_block(K);
+  const int64_t nh = resolve_nh(K, nh_arg);
   if ((K % 128) == 0 && nh >= 256 && nh <= 4096 && K <= 32768 && N > 0) {
     DecodeFastParams f;
     size_t smem = 0;
@@ -398,7 +398,7 @@ cudaError_t launch_decode(const DeviceCodebook& cb, const uint16_t* idx1, const 
   p.idx2 = idx2;
   p.N = N;
   p.K = K;
-  p.nh = (int)hadamard_block(K);
+  p.nh = (int)nh;
   p.elems_per_cta = p.nh < 2048 ? 2048 : p.nh;
   p.bpw = bpw;
   p.seed = seed;

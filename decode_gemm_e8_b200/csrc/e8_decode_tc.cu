@@ -514,8 +514,8 @@ static cudaError_t launch_decode_tc_t(const DecodeTcParams& p, const CUtensorMap
 // Shapes served: n_h in {1024, 2048, 4096}, N K a multiple of 8192 with
 // N K / 64 rows addressable by the store, 16-byte aligned buffers.
 bool decode_tc_eligible(int64_t N, int64_t K, const void* idx1, const void* idx2,
-                        const void* out) {
-  const int64_t nh = hadamard_block(K);
+                        const void* out, int64_t nh_arg) {
+  const int64_t nh = resolve_nh(K, nh_arg);
   auto al = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
   return N > 0 && (nh == 1024 || nh == 2048 || nh == 4096) && ((N * K) % dtc::SLAB) == 0 &&
          K <= ((int64_t)1 << 30) && N * K / 64 < ((int64_t)1 << 31) && al(idx1) &&
@@ -524,8 +524,8 @@ bool decode_tc_eligible(int64_t N, int64_t K, const void* idx1, const void* idx2
 
 cudaError_t launch_decode_tc(const DeviceCodebook& cb, const uint16_t* idx1, const void* idx2,
                              int64_t N, int64_t K, int bpw, uint64_t seed, float alpha,
-                             uint16_t* Wdec, int sm_count, cudaStream_t st) {
-  if (!decode_tc_eligible(N, K, idx1, bpw > 2 ? idx2 : nullptr, Wdec))
+                             uint16_t* Wdec, int sm_count, cudaStream_t st, int64_t nh_arg) {
+  if (!decode_tc_eligible(N, K, idx1, bpw > 2 ? idx2 : nullptr, Wdec, nh_arg))
     return cudaErrorNotSupported;
   CUtensorMap tm;
   if (!make_tmap_2d(&tm, Wdec, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)(N * K / 64), 64,
@@ -536,7 +536,7 @@ cudaError_t launch_decode_tc(const DeviceCodebook& cb, const uint16_t* idx1, con
   p.idx2 = idx2;
   p.slabs = N * K / dtc::SLAB;
   p.K = (int)K;
-  const int64_t nh = hadamard_block(K);
+  const int64_t nh = resolve_nh(K, nh_arg);
   p.log2R = 0;
   while ((int64_t(64) << p.log2R) < nh) ++p.log2R;
   p.seed = seed;

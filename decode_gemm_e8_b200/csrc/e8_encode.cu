@@ -430,12 +430,12 @@ int encode_elems_per_cta(int nh) { return nh < 2048 ? 2048 : nh; }
 cudaError_t launch_encode(const DeviceCodebook& cb, const float* W, int64_t N, int64_t K, int bpw,
                           uint64_t seed, float gamma, uint16_t* idx1, void* idx2,
                           WorkItem* work, uint32_t* work_count, uint64_t work_cap, float* U,
-                          int do_quantise, int sm_count, cudaStream_t st) {
+                          int do_quantise, int sm_count, cudaStream_t st, int64_t nh) {
   EncodeParams p;
   p.W = W;
   p.N = N;
   p.K = K;
-  p.nh = (int)hadamard_block(K);
+  p.nh = (int)resolve_nh(K, nh);
   p.elems_per_cta = encode_elems_per_cta(p.nh);
   p.bpw = bpw;
   p.seed = seed;

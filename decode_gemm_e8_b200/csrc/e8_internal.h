@@ -36,6 +36,12 @@ inline bool valid_scale(float s) { return s > 0.0f && std::isfinite(s); }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 // Shapes of the activation-side GEMM (E8_GEMM_ACT_RHT and _SMEM).
 inline bool act_shape_ok(int64_t M, int64_t K) { return M <= 64 && (K % 128) == 0; }
+// Hadamard block: 0 selects the default (the largest power of two dividing K);
+// an explicit block is a power of two in [8, 32768] that divides K.
+inline bool valid_nh(int64_t K, int64_t nh) {
+  return nh == 0 || (nh >= 8 && nh <= kMaxNh && (nh & (nh - 1)) == 0 && (K % nh) == 0);
+}
+inline int64_t resolve_nh(int64_t K, int64_t nh) { return nh ? nh : hadamard_block(K); }
 // Integer multiplier of the group vectors: z = m (c1 + beta c2).
 inline int m_of(int bpw) { return bpw == 2 ? 2 : (bpw == 3 ? 4 : 8); }
 // Decode constant alpha = fl32(scale / (m sqrt(n_h))), computed in binary64.
@@ -71,7 +77,7 @@ int encode_elems_per_cta(int nh);
 cudaError_t launch_encode(const DeviceCodebook& cb, const float* W, int64_t N, int64_t K, int bpw,
                           uint64_t seed, float gamma, uint16_t* idx1, void* idx2,
                           WorkItem* work, uint32_t* work_count, uint64_t work_cap, float* U,
-                          int do_quantise, int sm_count, cudaStream_t st);
+                          int do_quantise, int sm_count, cudaStream_t st, int64_t nh = 0);
 cudaError_t launch_encode_leader(const DeviceCodebook& cb, const WorkItem* in,
                                  const uint32_t* in_count, uint64_t cap, WorkItem* out,
                                  uint32_t* out_count, int bpw, uint16_t* idx1, void* idx2,
@@ -79,21 +85,21 @@ cudaError_t launch_encode_leader(const DeviceCodebook& cb, const WorkItem* in,
 
 cudaError_t launch_decode(const DeviceCodebook& cb, const uint16_t* idx1, const void* idx2,
                           int64_t N, int64_t K, int bpw, uint64_t seed, float alpha,
-                          uint16_t* Wdec, int sm_count, cudaStream_t st);
+                          uint16_t* Wdec, int sm_count, cudaStream_t st, int64_t nh = 0);
 // Tensor-core decoder (n_h = 1024, 2048, 4096; N K a multiple of 8192;
 // 16-byte aligned buffers); same contract and bit-identical result as
 // launch_decode.  Returns cudaErrorNotSupported, launching nothing, for other
 // shapes.
 bool decode_tc_eligible(int64_t N, int64_t K, const void* idx1, const void* idx2,
-                        const void* out);
+                        const void* out, int64_t nh = 0);
 cudaError_t launch_decode_tc(const DeviceCodebook& cb, const uint16_t* idx1, const void* idx2,
                              int64_t N, int64_t K, int bpw, uint64_t seed, float alpha,
-                             uint16_t* Wdec, int sm_count, cudaStream_t st);
+                             uint16_t* Wdec, int sm_count, cudaStream_t st, int64_t nh = 0);
 
 // X [M][K] bf16 -> Xt [rows][K] bf16: rows [0, M) hi parts, [M, 2M) lo parts of
 // FWHT(D x), rows [2M, rows) zero.
 cudaError_t launch_act_rht(const uint16_t* X, int64_t M, int64_t K, uint64_t seed, uint16_t* Xt,
-                           int64_t rows, cudaStream_t st, int pdl = 0);
+                           int64_t rows, cudaStream_t st, int pdl = 0, int64_t nh = 0);
 
 // Fused decode + GEMM with the transform moved onto the activations:
 // Y[m][n] = alpha * sum_k Xt[m][k] Z[n][k] (hi + lo rows), Z decoded on chip.
@@ -156,7 +162,7 @@ cudaError_t launch_gemm_q8_group(const DeviceCodebook& cb, const Q8Item* items, 
 // that launch_act_gemm_q8 accumulates into), after the preceding kernel ends.
 cudaError_t launch_act_q8(const uint16_t* X, int64_t M, int64_t K, uint64_t seed, int8_t* Xq,
                           float* scales, int32_t* colsum, int64_t rows, cudaStream_t st,
-                          int pdl, float* Yz = nullptr, int64_t yz_elems = 0);
+                          int pdl, float* Yz = nullptr, int64_t yz_elems = 0, int64_t nh = 0);
 // One output set of the grouped transform: X transformed with `seed` into
 // Xq / scales / colsum, and Yz[0, yz_elems) zeroed (Yz may be null).
 struct ActQ8Out {
@@ -169,7 +175,8 @@ struct ActQ8Out {
 };
 // The same transform for up to kMaxGroup seeds in one launch.
 cudaError_t launch_act_q8_group(const uint16_t* X, int64_t M, int64_t K, const ActQ8Out* outs,
-                                int count, int64_t rows, cudaStream_t st, int pdl);
+                                int count, int64_t rows, cudaStream_t st, int pdl,
+                                int64_t nh = 0);
 
 // Layout of the int8 activation buffer: Xq [rows][K] int8, then the per-token
 // steps (fp32 [M]) and the sums of every row over every 128-column unit
@@ -187,18 +194,19 @@ inline Q8Layout q8_layout(int64_t M, int64_t K, int64_t rows) {
 }
 // Shapes served by the int8 path: up to 32 tokens, K a multiple of 256 whose
 // Hadamard block lies in 256..4096, K <= 32768.
-inline bool q8_eligible(int64_t M, int64_t K) {
-  const int64_t nh = K & (-K);
-  return M >= 1 && M <= 32 && (K % 256) == 0 && nh >= 256 && nh <= 4096 && K <= 32768;
+inline bool q8_eligible(int64_t M, int64_t K, int64_t nh = 0) {
+  if (nh == 0) nh = K & (-K);
+  return M >= 1 && M <= 32 && (K % 256) == 0 && (K % nh) == 0 && nh >= 256 && nh <= 4096 &&
+         K <= 32768;
 }
 
 // Activation-side GEMM (E8_GEMM_ACT_RHT / _SMEM) on caller-provided scratch of
 // act_scratch_bytes() bytes: the transform and the fused kernel.
-size_t act_scratch_bytes(int64_t M, int64_t K, int smem_variant);
+size_t act_scratch_bytes(int64_t M, int64_t K, int smem_variant, int64_t nh = 0);
 cudaError_t run_act_gemm(const e8_codebook* cb, const uint16_t* X, int64_t M,
                          const uint16_t* idx1, const void* idx2, int64_t N, int64_t K, int bpw,
                          uint64_t seed, float alpha, float* Y, int smem_variant, void* scratch,
-                         cudaStream_t st);
+                         cudaStream_t st, int64_t nh = 0);
 
 // Dense Y[M][N] fp32 = X[M][K] bf16 * W[N][K]^T bf16 on tcgen05.
 cudaError_t launch_dense_gemm(const uint16_t* X, int64_t M, const uint16_t* W, int64_t N,

@@ -167,6 +167,33 @@ int e8_gemm(const e8_codebook* cb, const uint16_t* X, int64_t M, const uint16_t*
 int e8_act_rht_q8(const uint16_t* X, int64_t M, int64_t K, uint64_t rht_seed, void* buf,
                   void* stream);
 
+/* Explicit Hadamard block ("How it works", item 2: the transform is a
+ * randomized Hadamard transform of the input dimension; the page does not fix
+ * its block size).  The calls without a suffix use the default block, the
+ * largest power of two dividing K.  These take the block n_h explicitly: a
+ * power of two with 8 <= n_h <= 32768 that divides K (n_h = 0 selects the
+ * default), for instance n_h = 128 or 256 for every K, so that every K tile of
+ * 128 or 256 columns is transformed on its own.  Everything else -- signs,
+ * gamma = fl32(1 / (scale sqrt(n_h))), alpha = fl32(scale / (m sqrt(n_h))),
+ * the roundings, the codebooks -- is as above with n_h in place of the
+ * default block; codes written with one block must be decoded and multiplied
+ * with the same block.  Arguments, results and errors as the calls without the
+ * suffix (E8_EINVAL also for an invalid n_h). */
+int e8_rht_forward_nh(const e8_codebook* cb, const float* W, int64_t N, int64_t K, int64_t n_h,
+                      uint64_t rht_seed, float scale, float* U, void* stream);
+int e8_encode_nh(const e8_codebook* cb, const float* W, int64_t N, int64_t K, int64_t n_h,
+                 int bpw, uint64_t rht_seed, float scale, uint16_t* idx1, void* idx2,
+                 void* workspace, size_t ws_bytes, void* stream);
+int e8_decode_to_bf16_nh(const e8_codebook* cb, const uint16_t* idx1, const void* idx2,
+                         int64_t N, int64_t K, int64_t n_h, int bpw, uint64_t rht_seed,
+                         float scale, uint16_t* W_dec, void* stream);
+/* E8_GEMM_ACT_RHT with n_h < 256 takes the bf16 activation path (the int8 one
+ * needs 256 <= n_h <= 4096); the workspace is e8_workspace_bytes_nh's. */
+int e8_gemm_nh(const e8_codebook* cb, const uint16_t* X, int64_t M, const uint16_t* idx1,
+               const void* idx2, int64_t N, int64_t K, int64_t n_h, int bpw, uint64_t rht_seed,
+               float scale, float* Y, int mode, void* workspace, size_t ws_bytes, void* stream);
+size_t e8_workspace_bytes_nh(int op, int64_t M, int64_t N, int64_t K, int64_t n_h, int bpw);
+
 /* Size in bytes of the e8_act_rht_q8 buffer (0 if the shape is not served). */
 size_t e8_act_q8_bytes(int64_t M, int64_t K);
 

@@ -197,3 +197,19 @@ def test_grouped_call_refuses_bad_arguments_before_any_cuda_call(lib):
     # nothing to do: no CUDA call either
     assert call(M=0) == e8.E8_OK
     assert call(arr=items(3, {0: dict(N=0), 1: dict(N=0), 2: dict(N=0)})) == e8.E8_OK
+
+
+def test_explicit_block_workspace_sizes(lib):
+    N, K = 4096, 4096
+    # n_h = 256: the int8 activation path, as for the default block
+    assert e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT, 16, N, K, 4, nh=256) == \
+        e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT, 16, N, K, 4)
+    # n_h = 128: the bf16 activation path (hi and lo rows of K bf16)
+    assert e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT, 16, N, K, 4, nh=128) == 32 * K * 2
+    # n_h = 0 is the default block; invalid blocks give 0
+    assert e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT, 16, N, K, 4, nh=0) == \
+        e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT, 16, N, K, 4)
+    for nh in (4, 96, 8192 * 2, 65536):
+        assert e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT, 16, N, K, 4, nh=nh) == 0
+    assert e8.e8_workspace_bytes(e8.E8_GEMM_DECODED_W, 64, N, 3072, 4, nh=2048) == 0
+    assert e8.e8_workspace_bytes(e8.E8_GEMM_DECODED_W, 64, N, 3072, 4, nh=1024) == N * 3072 * 2
