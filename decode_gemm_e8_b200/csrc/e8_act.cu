@@ -265,10 +265,7 @@ namespace e8 {
 // row is written as two int8 pieces
 //   q0 = rint(x / s_m),  q1 = rint((x - q0 s_m) * 128 / s_m),  |q1| <= 64,
 // so x = s_m (q0 + q1 / 128) + e with |e| <= s_m / 256.  Piece rows are
-// interleaved (row 2m = q0, row 2m + 1 = q1); colsum[u][row] = the sum of
-// Xq[row][k] over the 128 positions k of unit u lets every partial product of
-// the GEMM remove the +128 bias of its unsigned weight operand over its own
-// K range, exactly.
+// interleaved (row 2m = q0, row 2m + 1 = q1).
 // Kept small (32 registers, at most 16 KB of shared memory) so that a CTA can
 // share an SM with a CTA of the GEMM that follows it; the transform runs
 // before the wait for the preceding kernel, and only the stores wait for it.
@@ -279,7 +276,6 @@ struct ActQ8Group {
   uint64_t seed[kMaxGroup];
   int8_t* Xq[kMaxGroup];
   float* scales[kMaxGroup];
-  int32_t* colsum[kMaxGroup];
   float* Yz[kMaxGroup];
   int64_t yz_elems[kMaxGroup];
 };
@@ -315,7 +311,6 @@ __global__ void __launch_bounds__(512, 4) k_act_q8(const uint16_t* __restrict__ 
   const uint64_t seed = pick_group(grp.seed, g);
   int8_t* __restrict__ Xq = pick_group(grp.Xq, g);
   float* __restrict__ scales = pick_group(grp.scales, g);
-  int32_t* __restrict__ colsum = pick_group(grp.colsum, g);
   float* __restrict__ Yz = pick_group(grp.Yz, g);
   const int64_t yz_elems = pick_group(grp.yz_elems, g);
   const int kb = c << 12;
@@ -435,7 +430,6 @@ __global__ void __launch_bounds__(512, 4) k_act_q8(const uint16_t* __restrict__ 
   const float amax = s_amax;
   const float step = amax > 0.0f ? amax / 127.0f : 1.0f;
   const float inv = 1.0f / step;
-  int sum0 = 0, sum1 = 0;
   uint2 e0 = make_uint2(0u, 0u), e1 = make_uint2(0u, 0u);   // this thread's bytes
   if (8 * t < C) {
     const float4 xa = *reinterpret_cast<const float4*>(chunk + 8 * t);
@@ -448,25 +442,20 @@ __global__ void __launch_bounds__(512, 4) k_act_q8(const uint16_t* __restrict__ 
       const float r = xs[i] - a * step;
       const float b = fminf(fmaxf(rintf(r * inv * 128.0f), -127.0f), 127.0f);
       const int ia = (int)a, ib = (int)b;
-      sum0 += ia;
-      sum1 += ib;
       p0[i >> 2] |= (uint32_t)(ia & 0xFF) << (8 * (i & 3));
       p1[i >> 2] |= (uint32_t)(ib & 0xFF) << (8 * (i & 3));
     }
     e0 = make_uint2(p0[0], p0[1]);
     e1 = make_uint2(p1[0], p1[1]);
   }
-  // piece sums of every 128-position unit: the 16 threads of a half-warp hold
-  // one unit (positions 128 (t / 16) .. + 127 of the chunk); lanes 0 and 16
-  // end with the sums
-#pragma unroll
-  for (int off = 8; off > 0; off >>= 1) {
-    sum0 += __shfl_xor_sync(0xffffffffu, sum0, off);
-    sum1 += __shfl_xor_sync(0xffffffffu, sum1, off);
-  }
   // the stores wait for the preceding kernel, which may still read Xq, the
-  // steps, the sums and Y
+  // steps and Y
   grid_dep_wait();
+  if (8 * t < C) {
+    *reinterpret_cast<uint2*>(Xq + (size_t)(2 * m) * K + kb + 8 * t) = e0;
+    *reinterpret_cast<uint2*>(Xq + (size_t)(2 * m + 1) * K + kb + 8 * t) = e1;
+  }
+  if (c == 0 && t == 0) scales[m] = step;
   if (Yz) {
     // the output that the following GEMM accumulates into starts at zero
     const int64_t nb = per_set;
@@ -480,23 +469,11 @@ __global__ void __launch_bounds__(512, 4) k_act_q8(const uint16_t* __restrict__ 
       }
     }
   }
-  // padding rows 2M .. rows-1: zero bytes, zero sums
-  const bool unit_lead = (t & 15) == 0 && 8 * t < C;
-  const size_t unit = (size_t)((kb >> 7) + (t >> 4));     // this half-warp's unit of the row
+  // padding rows 2M .. rows-1: zero bytes
   for (int pr = 2 * M + m; pr < rows; pr += M) {
     for (int k = 16 * t; k < C; k += 16 * 512)
       *reinterpret_cast<uint4*>(Xq + (size_t)pr * K + kb + k) = make_uint4(0u, 0u, 0u, 0u);
-    if (unit_lead) colsum[unit * rows + pr] = 0;
   }
-  if (8 * t < C) {
-    *reinterpret_cast<uint2*>(Xq + (size_t)(2 * m) * K + kb + 8 * t) = e0;
-    *reinterpret_cast<uint2*>(Xq + (size_t)(2 * m + 1) * K + kb + 8 * t) = e1;
-  }
-  if (unit_lead) {
-    colsum[unit * rows + 2 * m] = sum0;
-    colsum[unit * rows + 2 * m + 1] = sum1;
-  }
-  if (c == 0 && t == 0) scales[m] = step;
 }
 
 cudaError_t launch_act_q8_group(const uint16_t* X, int64_t M, int64_t K, const ActQ8Out* outs,
@@ -512,7 +489,6 @@ cudaError_t launch_act_q8_group(const uint16_t* X, int64_t M, int64_t K, const A
     grp.seed[g] = outs[g].seed;
     grp.Xq[g] = outs[g].Xq;
     grp.scales[g] = outs[g].scales;
-    grp.colsum[g] = outs[g].colsum;
     grp.Yz[g] = outs[g].Yz;
     grp.yz_elems[g] = outs[g].Yz ? outs[g].yz_elems : 0;
   }
@@ -542,13 +518,12 @@ cudaError_t launch_act_q8_group(const uint16_t* X, int64_t M, int64_t K, const A
 }
 
 cudaError_t launch_act_q8(const uint16_t* X, int64_t M, int64_t K, uint64_t seed, int8_t* Xq,
-                          float* scales, int32_t* colsum, int64_t rows, cudaStream_t st,
-                          int pdl, float* Yz, int64_t yz_elems, int64_t nh) {
+                          float* scales, int64_t rows, cudaStream_t st, int pdl, float* Yz,
+                          int64_t yz_elems, int64_t nh) {
   ActQ8Out o;
   o.seed = seed;
   o.Xq = Xq;
   o.scales = scales;
-  o.colsum = colsum;
   o.Yz = Yz;
   o.yz_elems = yz_elems;
   return launch_act_q8_group(X, M, K, &o, 1, rows, st, pdl, nh);

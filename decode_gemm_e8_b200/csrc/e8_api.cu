@@ -72,7 +72,6 @@ cudaError_t run_act_gemm(const e8_codebook* cb, const uint16_t* X, int64_t M,
     ActQ8Args a;
     a.Xq = reinterpret_cast<int8_t*>(buf);
     a.scales = reinterpret_cast<float*>(buf + l.scales_off);
-    a.colsum = reinterpret_cast<int32_t*>(buf + l.colsum_off);
     a.M = M;
     a.N = N;
     a.K = K;
@@ -85,8 +84,7 @@ cudaError_t run_act_gemm(const e8_codebook* cb, const uint16_t* X, int64_t M,
     a.pdl = 1;          // the fused kernel's prologue overlaps the transform
     a.early_codes = 1;  // which writes only the activation buffer
     cudaError_t e = launch_act_q8(X, M, K, seed, reinterpret_cast<int8_t*>(buf),
-                                  reinterpret_cast<float*>(buf + l.scales_off),
-                                  reinterpret_cast<int32_t*>(buf + l.colsum_off), rows, st, 1, Y,
+                                  reinterpret_cast<float*>(buf + l.scales_off), rows, st, 1, Y,
                                   M * N, nh);
     if (e != cudaSuccess) return e;
     return launch_act_gemm_q8(d, a, cb->sm_count, st);
@@ -488,8 +486,7 @@ int e8_act_rht_q8(const uint16_t* X, int64_t M, int64_t K, uint64_t rht_seed, vo
   const e8::Q8Layout l = e8::q8_layout(M, K, rows);
   uint8_t* b = static_cast<uint8_t*>(buf);
   return cuda_status(e8::launch_act_q8(X, M, K, rht_seed, reinterpret_cast<int8_t*>(b),
-                                       reinterpret_cast<float*>(b + l.scales_off),
-                                       reinterpret_cast<int32_t*>(b + l.colsum_off), rows,
+                                       reinterpret_cast<float*>(b + l.scales_off), rows,
                                        (cudaStream_t)stream, 0));
 }
 
@@ -520,7 +517,6 @@ int e8_gemm_xt(const e8_codebook* cb, const void* xq, int64_t M, const uint16_t*
   e8::ActQ8Args a;
   a.Xq = reinterpret_cast<const int8_t*>(b);
   a.scales = reinterpret_cast<const float*>(b + l.scales_off);
-  a.colsum = reinterpret_cast<const int32_t*>(b + l.colsum_off);
   a.M = M;
   a.N = N;
   a.K = K;
@@ -584,7 +580,6 @@ int e8_gemm_grouped(const e8_codebook* cb, const uint16_t* X, int64_t M, int64_t
     outs[n].seed = it.rht_seed;
     outs[n].Xq = reinterpret_cast<int8_t*>(buf);
     outs[n].scales = reinterpret_cast<float*>(buf + l.scales_off);
-    outs[n].colsum = reinterpret_cast<int32_t*>(buf + l.colsum_off);
     outs[n].Yz = it.Y;   // zeroed by the transform, accumulated into by the GEMM
     outs[n].yz_elems = M * it.N;
     its[n].idx1 = it.idx1;
@@ -593,7 +588,6 @@ int e8_gemm_grouped(const e8_codebook* cb, const uint16_t* X, int64_t M, int64_t
     its[n].alpha = alpha_of(it.scale, nh, bpw);
     its[n].Xq = outs[n].Xq;
     its[n].scales = outs[n].scales;
-    its[n].colsum = outs[n].colsum;
     its[n].Y = it.Y;
     ++n;
   }

@@ -8,11 +8,12 @@
 // (rows 2m and 2m + 1 of Xq, written by k_act_q8) with a per-token step s_m:
 //   xt_m = s_m (q0_m + q1_m / 128).
 // The weight operand is z + 128 as unsigned bytes, decoded on chip straight
-// into tensor memory; tcgen05.mma kind::i8 accumulates exactly in int32 and
-// the epilogue removes the +128 bias with the sums of the Xq rows over the
-// K units that the partial product covers (cs, from the transform's per-unit
-// sums), exactly in int32, before anything is rounded:
-//   y[m][n] = alpha s_m ((D[n][2m] - 128 cs[2m]) + (D[n][2m+1] - 128 cs[2m+1]) / 128).
+// into tensor memory; tcgen05.mma kind::i8 accumulates exactly in int32.  The
+// +128 bias is removed by the tensor cores too: every K step is followed by a
+// second product of the same Xq tile with a constant signed operand of -128,
+// accumulating -128 sum_k Xq into the same accumulator, so D = Xq . z exactly
+// and no partial sum carries the bias:
+//   y[m][n] = alpha s_m (D[n][2m] + D[n][2m+1] / 128).
 //
 // Work split (stream-K): the (128-row tile, 128-wide K unit) pairs are laid out
 // tile by tile and every CTA of a one-per-SM grid takes a contiguous run of
@@ -69,8 +70,12 @@ constexpr uint32_t A_COLS = KU / 4;       // 4 int8 weights per TMEM column
 constexpr int MAX_STAGES = 8;
 static_assert(MAX_STAGES % DEC_GROUPS == 0 && MAX_STAGES % 2 == 0,
               "each operand stage serves one decoder group and one issuer");
-// per matrix: alpha times the per-token steps [32]; then the segments' piece sums [3][64]
-constexpr int AUX_BYTES = 128 * kMaxGroup + 768;
+constexpr int AUX_BYTES = 128 * kMaxGroup;   // per matrix: alpha times the per-token steps [32]
+// The constant -128 operand (128 rows x 32 bytes, every byte 0x80 read as
+// signed): up to 16 tokens it sits in tensor-memory columns that the
+// accumulators of buffer 0 leave unused; above, in this shared-memory tile.
+constexpr int CONST_A_BYTES = 4096;
+constexpr uint32_t CONST_A_COL = 32;
 constexpr int BAR_BYTES = 512;
 // shared memory left free on the SM for a CTA of the activation transform
 // (K = 4096: 16 KB), so that it can run next to this kernel's CTA
@@ -84,7 +89,8 @@ constexpr int CORESIDENT_RESERVE = 18 * 1024;
 // and row sums, and the barriers.  Offsets below are relative to that
 // boundary.  The decoded operands live in a ring of sa tensor-memory stages.
 struct SkPlan {
-  int sa, sx, sc, b_bytes, code_bytes, i2_bytes, code_off, y_off, aux_off, bar_off, total;
+  int sa, sx, sc, b_bytes, code_bytes, i2_bytes, code_off, y_off, aux_off, const_off, bar_off,
+      total;
   uint32_t tmem_cols;
 };
 
@@ -95,7 +101,7 @@ __host__ __device__ inline SkPlan sk_plan(int rows_b, int bpw) {
   p.i2_bytes = bpw == 2 ? 0 : (bpw == 3 ? ROWS * GROUPS : ROWS * GROUPS * 2);
   p.code_bytes = I1_BYTES + p.i2_bytes;                     // multiple of 1 KB
   const int y_bytes = (rows_b <= 32 ? 16 : 32) * ROWS * 4;
-  const int budget = kMaxDynSmem - TABLE_BYTES - 1024 - AUX_BYTES - BAR_BYTES -
+  const int budget = kMaxDynSmem - TABLE_BYTES - 1024 - AUX_BYTES - CONST_A_BYTES - BAR_BYTES -
                      CORESIDENT_RESERVE - y_bytes;
   p.sa = MAX_STAGES;                                        // 4 x 64 + 8 x 32 TMEM columns
   // Xq tiles are requested after the transform kernel ends and take ~1 us to
@@ -114,7 +120,8 @@ __host__ __device__ inline SkPlan sk_plan(int rows_b, int bpw) {
   p.code_off = p.sx * p.b_bytes;
   p.y_off = p.code_off + p.sc * p.code_bytes;
   p.aux_off = p.y_off + y_bytes;
-  p.bar_off = p.aux_off + AUX_BYTES;
+  p.const_off = p.aux_off + AUX_BYTES;      // multiple of 512 bytes
+  p.bar_off = p.const_off + CONST_A_BYTES;
   p.total = TABLE_BYTES + 1024 + p.bar_off + BAR_BYTES;
   p.tmem_cols = 512u;
   return p;
@@ -141,7 +148,6 @@ struct SkMat {
   float alpha;
   int use_tma_y;         // Y by bulk reduce-add (else fp32 atomics)
   const float* tok_scale;
-  const int32_t* colsum;
   float* Y;
 };
 struct SkGroup {
@@ -177,6 +183,27 @@ __device__ __forceinline__ void sk_mma_i8(uint32_t d_tmem, uint32_t a_tmem, uint
 // both operands K-major.
 __host__ __device__ constexpr uint32_t sk_idesc(uint32_t M, uint32_t N) {
   return (2u << 4) | (0u << 7) | (1u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+// The same with a signed A operand (the constant -128 bias product).
+__host__ __device__ constexpr uint32_t sk_idesc_sa(uint32_t M, uint32_t N) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+
+// kind::i8 with both operands from shared memory (descriptors).
+__device__ __forceinline__ void sk_mma_i8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void sk_tmem_st8(uint32_t taddr, uint32_t v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr),
+      "r"(v)
+      : "memory");
 }
 
 __device__ __forceinline__ void sk_tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
@@ -246,8 +273,7 @@ __global__ void __maxnreg__(64)
   uint64_t* drain = acc_full + 5;                 // [2] one per issuer
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 7);
   volatile uint32_t* abort_flag = tmem_slot + 1;
-  float* s_sc = reinterpret_cast<float*>(smem + plan.aux_off);                          // [G][32]
-  int32_t* s_cs = reinterpret_cast<int32_t*>(smem + plan.aux_off + 128 * kMaxGroup);    // [3][64]
+  float* s_sc = reinterpret_cast<float*>(smem + plan.aux_off);   // [G][32]
   float* s_y = reinterpret_cast<float*>(smem + plan.y_off);                // [M][128]
   uint8_t* xq_ring = smem;
   uint8_t* code_ring = smem + plan.code_off;
@@ -288,6 +314,24 @@ __global__ void __maxnreg__(64)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const uint32_t tmem_a = tmem_base + ACC_TOTAL;
+  // the constant -128 operand: with up to 16 tokens (CW == 32) columns 32..39
+  // of accumulator buffer 0, which its MMAs (N <= 32) never write; else a
+  // shared-memory tile (K-major, no swizzle: every byte is the same)
+  const uint32_t const_a_tmem = tmem_base + CONST_A_COL;
+  if (CW == 32) {
+    if (warp >= 2 && warp < 6) {   // one warp per TMEM lane quarter
+      sk_tmem_st8(const_a_tmem + ((uint32_t)((warp & 3) * 32) << 16), 0x80808080u);
+      tmem_st_wait();
+    }
+  } else {
+    uint4* ca = reinterpret_cast<uint4*>(smem + plan.const_off);
+    for (int i = threadIdx.x; i < CONST_A_BYTES / 16; i += THREADS)
+      ca[i] = make_uint4(0x80808080u, 0x80808080u, 0x80808080u, 0x80808080u);
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
   const int nseg = nu > 0 ? (u_begin + nu - 1) / kunits - first_tile + 1 : 0;
   const int ku_first = u_begin - first_tile * kunits;   // K unit of the run's first unit
   // the next kernel of the stream may be launched now: it waits for this grid
@@ -382,7 +426,9 @@ __global__ void __maxnreg__(64)
     // or a decoder will reuse it.
     const int par = warp == 1 ? 0 : 1;
     const uint32_t idesc = sk_idesc(ROWS, (uint32_t)rows_b);
+    const uint32_t idesc_bias = sk_idesc_sa(ROWS, (uint32_t)rows_b);
     const uint64_t bd0 = smem_desc(smem_u32(xq_ring), 16, 1024, 2);
+    const uint64_t const_desc = smem_desc(smem_u32(smem + plan.const_off), 128, 256, 0);
     const uint32_t stage16 = (uint32_t)plan.b_bytes >> 4;
     int s = par, sxi = par % SX;   // operand and Xq stages of the issuer's unit
     uint32_t ph = 0;
@@ -416,9 +462,15 @@ __global__ void __maxnreg__(64)
         const uint64_t bds = bd0 + (uint64_t)((uint32_t)sxi * stage16);
         if (elect_one()) {
 #pragma unroll
-          for (int j = 0; j < KU / 32; ++j)
+          for (int j = 0; j < KU / 32; ++j) {
             sk_mma_i8(d, a0 + (uint32_t)(j * 8), bds + (uint64_t)(j * 2), idesc,
                       (i == i0 && j == 0) ? 0u : 1u);
+            // minus 128 times the same Xq columns: removes the weight bias
+            if (CW == 32)
+              sk_mma_i8(d, const_a_tmem, bds + (uint64_t)(j * 2), idesc_bias, 1u);
+            else
+              sk_mma_i8_ss(d, const_desc, bds + (uint64_t)(j * 2), idesc_bias, 1u);
+          }
           // the stage is reused by unit i + SX (Xq) and unit i + SA (operand)
           if (i + SX < nu) mma_commit(&a_empty[s]);
         }
@@ -558,46 +610,14 @@ __global__ void __maxnreg__(64)
     const int q = warp & 3;
     const int r = q * 32 + lane;
     const bool issuer = warp == EPI_WARP0 && lane == 0;
-    grid_dep_wait();   // steps, unit sums and the zeroed Y come from the transform
+    grid_dep_wait();   // steps and the zeroed Y come from the transform
     if (warp == EPI_WARP0) {
       for (int j = 0; j < grp.count; ++j) {
         const SkMat& mt = grp.mat[j];
         s_sc[32 * j + lane] = lane < M ? mt.alpha * __ldg(mt.tok_scale + lane) : 0.0f;
       }
     }
-    // Sums of the Xq rows over the K units [ku_lo, ku_hi) of segment sg: the
-    // bias its partial product carries.  Warp EPI_WARP0 computes those of the
-    // next segment while the current one is still being decoded, into a ring
-    // of three buffers (one being read, one being written, one that slow
-    // warps may still read for the previous segment until the barrier).
-    auto seg_sums = [&](int sg) {
-      const int slo = sg == 0 ? 0 : kunits - ku_first + (sg - 1) * kunits;
-      const int slen = kunits - (sg == 0 ? ku_first : 0);
-      const int shi = slo + slen < nu ? slo + slen : nu;
-      const int tl = first_tile + sg;
-      const int32_t* src = grp.mat[sk_mat_of(grp, tl)].colsum;
-      const int ku_lo = u_begin + slo - tl * kunits, ku_hi = u_begin + shi - tl * kunits;
-      int a0 = 0, a1 = 0;
-      for (int ku = ku_lo; ku < ku_hi; ku += 8) {
-        int v0[8], v1[8];   // eight independent loads in flight
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const bool in = ku + j < ku_hi;
-          const int32_t* p = src + (size_t)(ku + j) * rows_b;
-          v0[j] = in && lane < rows_b ? __ldg(p + lane) : 0;
-          v1[j] = in && 32 + lane < rows_b ? __ldg(p + 32 + lane) : 0;
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          a0 += v0[j];
-          a1 += v1[j];
-        }
-      }
-      int32_t* dst = s_cs + 64 * (sg % 3);
-      dst[lane] = a0;
-      dst[32 + lane] = a1;
-    };
-    if (warp == EPI_WARP0 && nseg > 0) seg_sums(0);
+    asm volatile("bar.sync 1, 128;" ::: "memory");   // the steps
     // every epilogue thread runs the same sequence of named barriers, also
     // after a failed wait (it then only skips the work)
     bool ok = true;
@@ -611,11 +631,6 @@ __global__ void __maxnreg__(64)
       const bool has1 = hi - lo >= 2 || (lo & 1) == 1;
       const int tile = first_tile + seg;
       const int mj = sk_mat_of(grp, tile);
-      if (warp == EPI_WARP0 && seg + 1 < nseg) seg_sums(seg + 1);
-      // the barrier publishes the sums of this segment (written one segment
-      // earlier) and the steps
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      const int32_t* cs = s_cs + 64 * (seg % 3);
       lo = hi;
       ok = ok && mbar_wait_sleep(&acc_full[b], (uint32_t)(seg >> 1) & 1u, abort_flag, status,
                                  kDevTimeoutMma);
@@ -625,7 +640,6 @@ __global__ void __maxnreg__(64)
       const int use_tma_y = grp.mat[mj].use_tma_y;
       const float* sc = s_sc + 32 * mj;
       const int n = (tile - grp.mat[mj].tile0) * ROWS + r;
-      constexpr int corr = 128;
       const uint32_t lane_off = (uint32_t)(q * 32) << 16;
       const uint32_t t0a = tmem_base + (uint32_t)b * ACC_COLS + lane_off;         // parity 0
       const uint32_t t1a = tmem_base + (uint32_t)(2 + b) * ACC_COLS + lane_off;   // parity 1
@@ -646,24 +660,22 @@ __global__ void __maxnreg__(64)
           dv[j] = x0 + x1;
         }
         if (use_tma_y) {
-          // tokens past M have zero steps and unit sums: staged as zeros (the
+          // tokens past M have zero steps: staged as zeros (the
           // bulk reduce covers only M rows), no branch in the loop
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const int m = (c0 >> 1) + j;
-            const int d0 = (int)dv[2 * j] - corr * cs[2 * m];
-            const int d1 = (int)dv[2 * j + 1] - corr * cs[2 * m + 1];
-            s_y[m * ROWS + r] = sc[m] * ((float)d0 + (float)d1 * (1.0f / 128.0f));
+            s_y[m * ROWS + r] = sc[m] * ((float)(int)dv[2 * j] + (float)(int)dv[2 * j + 1] *
+                                                                     (1.0f / 128.0f));
           }
         } else if (n < N) {
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const int m = (c0 >> 1) + j;
-            const int d0 = (int)dv[2 * j] - corr * cs[2 * m];
-            const int d1 = (int)dv[2 * j + 1] - corr * cs[2 * m + 1];
             if (m < M)
               red_add_f32(Y + (size_t)m * N + n,
-                          sc[m] * ((float)d0 + (float)d1 * (1.0f / 128.0f)));
+                          sc[m] * ((float)(int)dv[2 * j] + (float)(int)dv[2 * j + 1] *
+                                                               (1.0f / 128.0f)));
           }
         }
       }
@@ -742,7 +754,6 @@ static cudaError_t launch_gemm_q8(const DeviceCodebook& cb, const Q8Item* items,
     mt.alpha = a.alpha;
     mt.use_tma_y = use_tma_y;
     mt.tok_scale = a.scales;
-    mt.colsum = a.colsum;
     mt.Y = a.Y;
     tiles += (a.N + ROWS - 1) / ROWS;
   }
@@ -796,7 +807,6 @@ cudaError_t launch_act_gemm_q8(const DeviceCodebook& cb, const ActQ8Args& a, int
   it.alpha = a.alpha;
   it.Xq = a.Xq;
   it.scales = a.scales;
-  it.colsum = a.colsum;
   it.Y = a.Y;
   return launch_gemm_q8_group(cb, &it, 1, a.M, a.K, a.rows_b, a.bpw, a.pdl, a.early_codes,
                               sm_count, st);

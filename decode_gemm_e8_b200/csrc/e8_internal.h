@@ -126,7 +126,6 @@ cudaError_t launch_act_gemm(const DeviceCodebook& cb, const ActGemmArgs& a, int 
 struct ActQ8Args {
   const int8_t* Xq;
   const float* scales;   // [M]
-  const int32_t* colsum; // [K / 128][rows_b]
   int64_t M, N, K;
   int rows_b;
   const uint16_t* idx1;
@@ -152,7 +151,6 @@ struct Q8Item {
   float alpha;
   const int8_t* Xq;       // [rows_b][K], token m: rows 2m, 2m + 1
   const float* scales;    // [M]
-  const int32_t* colsum;  // [K / 128][rows_b]
   float* Y;               // [M][N], zero when the kernel starts
 };
 cudaError_t launch_gemm_q8_group(const DeviceCodebook& cb, const Q8Item* items, int count,
@@ -161,15 +159,14 @@ cudaError_t launch_gemm_q8_group(const DeviceCodebook& cb, const Q8Item* items, 
 // When Yz is not null the kernel also zeroes Yz[0, yz_elems) (the fp32 output
 // that launch_act_gemm_q8 accumulates into), after the preceding kernel ends.
 cudaError_t launch_act_q8(const uint16_t* X, int64_t M, int64_t K, uint64_t seed, int8_t* Xq,
-                          float* scales, int32_t* colsum, int64_t rows, cudaStream_t st,
-                          int pdl, float* Yz = nullptr, int64_t yz_elems = 0, int64_t nh = 0);
+                          float* scales, int64_t rows, cudaStream_t st, int pdl,
+                          float* Yz = nullptr, int64_t yz_elems = 0, int64_t nh = 0);
 // One output set of the grouped transform: X transformed with `seed` into
-// Xq / scales / colsum, and Yz[0, yz_elems) zeroed (Yz may be null).
+// Xq / scales, and Yz[0, yz_elems) zeroed (Yz may be null).
 struct ActQ8Out {
   uint64_t seed;
   int8_t* Xq;
   float* scales;
-  int32_t* colsum;
   float* Yz;
   int64_t yz_elems;
 };
@@ -179,17 +176,15 @@ cudaError_t launch_act_q8_group(const uint16_t* X, int64_t M, int64_t K, const A
                                 int64_t nh = 0);
 
 // Layout of the int8 activation buffer: Xq [rows][K] int8, then the per-token
-// steps (fp32 [M]) and the sums of every row over every 128-column unit
-// (int32 [K / 128][rows]), each part starting on a 256-byte boundary.
+// steps (fp32 [M]), each part starting on a 256-byte boundary.
 struct Q8Layout {
-  size_t scales_off, colsum_off, total;
+  size_t scales_off, total;
 };
 inline Q8Layout q8_layout(int64_t M, int64_t K, int64_t rows) {
   auto r256 = [](size_t x) { return (x + 255) & ~size_t(255); };
   Q8Layout l;
   l.scales_off = r256((size_t)rows * (size_t)K);
-  l.colsum_off = l.scales_off + r256((size_t)M * 4);
-  l.total = l.colsum_off + r256((size_t)rows * (size_t)(K / 128) * 4);
+  l.total = l.scales_off + r256((size_t)M * 4);
   return l;
 }
 // Shapes served by the int8 path: up to 32 tokens, K a multiple of 256 whose

@@ -159,9 +159,7 @@ int e8_gemm(const e8_codebook* cb, const uint16_t* X, int64_t M, const uint16_t*
  *     q1 of token m, where xt = FWHT(D x_m) per Hadamard block,
  *     s_m = max|xt| / 127, q0 = rint(xt / s_m), q1 = rint((xt - q0 s_m) 128 / s_m),
  *     so xt = s_m (q0 + q1 / 128) within s_m / 256; padding rows are zero;
- *   then s_m (fp32 [M]) and the sums of every Xq row over every unit of 128
- *     columns (int32 [K / 128][rows], unit-major), each part starting on a
- *     256-byte boundary after the previous one.
+ *   then s_m (fp32 [M]), starting on a 256-byte boundary after Xq.
  * Shapes: 1 <= M <= 32, K a multiple of 256 whose Hadamard block is 256..4096,
  * K <= 32768 (else E8_EINVAL). */
 int e8_act_rht_q8(const uint16_t* X, int64_t M, int64_t K, uint64_t rht_seed, void* buf,

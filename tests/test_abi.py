@@ -48,13 +48,11 @@ def test_workspace_sizes(lib):
     # fast path, then what the class search leaves open)
     assert e8.e8_workspace_bytes(e8.E8_OP_ENCODE, 0, N, K, 4) == 256 + 2 * 48 * N * K // 8
     assert e8.e8_workspace_bytes(e8.E8_GEMM_DECODED_W, 4096, N, K, 3) == N * K * 2
-    # int8 pieces for 16 tokens: 32 rows of K bytes, 16 steps, then the sums of
-    # the 32 rows over each of the K / 128 units
-    units = K // 128
-    assert e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT, 16, N, K, 4) == 32 * K + 256 + 32 * units * 4
-    assert e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT, 1, N, K, 4) == 16 * K + 256 + 16 * units * 4
-    assert e8.e8_workspace_bytes(e8.E8_GEMM_AUTO, 16, N, K, 4) == 32 * K + 256 + 32 * units * 4
-    assert e8.e8_act_q8_bytes(16, K) == 32 * K + 256 + 32 * units * 4
+    # int8 pieces for 16 tokens: 32 rows of K bytes, then 16 steps
+    assert e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT, 16, N, K, 4) == 32 * K + 256
+    assert e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT, 1, N, K, 4) == 16 * K + 256
+    assert e8.e8_workspace_bytes(e8.E8_GEMM_AUTO, 16, N, K, 4) == 32 * K + 256
+    assert e8.e8_act_q8_bytes(16, K) == 32 * K + 256
     # bf16 hi and lo rows where the int8 path does not apply (more than 32 tokens)
     assert e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT, 40, N, K, 4) == 80 * K * 2
     assert e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT_SMEM, 16, N, K, 4) == 32 * K * 2
@@ -141,12 +139,11 @@ def test_missing_library_fails_loudly(tmp_path):
 
 
 def test_grouped_workspace_sizes(lib):
-    # one int8 activation buffer per item: 2M rows (padded to 16) of K bytes,
-    # the per-token steps and the row sums, each on 256 bytes
+    # one int8 activation buffer per item: 2M rows (padded to 16) of K bytes
+    # and the per-token steps, each on 256 bytes
     one = e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT, 16, 4096, 4096, 4)
     assert e8.e8_gemm_grouped_workspace_bytes(16, 4096, 4, 3) == 3 * one
-    assert e8.e8_gemm_grouped_workspace_bytes(5, 14336, 2, 4) == \
-        4 * (16 * 14336 + 256 + 16 * (14336 // 128) * 4)
+    assert e8.e8_gemm_grouped_workspace_bytes(5, 14336, 2, 4) == 4 * (16 * 14336 + 256)
     # invalid: no items, too many, more than 32 tokens, K outside the int8 path
     assert e8.e8_gemm_grouped_workspace_bytes(16, 4096, 4, 0) == 0
     assert e8.e8_gemm_grouped_workspace_bytes(16, 4096, 4, e8.E8_GROUP_MAX + 1) == 0

@@ -261,18 +261,14 @@ def test_gemm_xt_matches_gemm_and_graph_capture(gcb):
 @pytest.mark.parametrize("M,K", [(16, 4096), (3, 3072), (32, 256), (1, 12288), (5, 14336),
                                  (7, 4352), (2, 20480), (3, 30720), (32, 14336)])
 def test_act_rht_q8_pieces(gcb, M, K):
-    # xt = s_m (q0 + q1 / 128) within s_m / 256, s_m = max|xt| / 127, and the
-    # sums of every row over every 128-column unit (unit-major)
+    # xt = s_m (q0 + q1 / 128) within s_m / 256, s_m = max|xt| / 127
     X = synth.activations_bf16(M, K, 40 + M)
     buf = gu.to_np(e8.e8_act_rht_q8(gu.bf16_dev(X), 17))
     rows = e8.e8_gemm_xt_rows(M)
     assert len(buf) >= e8.e8_act_q8_bytes(M, K)
     xq = buf[:rows * K].view(np.int8).reshape(rows, K).astype(np.int64)
     off_s = (rows * K + 255) // 256 * 256
-    off_c = off_s + (M * 4 + 255) // 256 * 256
     sc = buf[off_s:off_s + 4 * M].view(np.float32).astype(np.float64)
-    units = K // 128
-    cs = buf[off_c:off_c + 4 * rows * units].view(np.int32).reshape(units, rows)
     x = synth.bf16_bits_to_f32(X).astype(np.float64)
     d = orc.signs(17, K).astype(np.float64)
     from tests import indep
@@ -284,5 +280,4 @@ def test_act_rht_q8_pieces(gcb, M, K):
     rec = sc[:, None] * (xq[0:2 * M:2] + xq[1:2 * M:2] / 128.0)
     assert np.all(np.abs(rec - ref) <= sc[:, None] / 256 * 1.01 + 1e-6)
     assert np.all(np.abs(xq[1:2 * M:2]) <= 64)
-    assert np.array_equal(cs, xq.reshape(rows, units, 128).sum(2).T)
     assert not xq[2 * M:].any()
