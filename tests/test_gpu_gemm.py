@@ -281,3 +281,22 @@ def test_act_rht_q8_pieces(gcb, M, K):
     assert np.all(np.abs(rec - ref) <= sc[:, None] / 256 * 1.01 + 1e-6)
     assert np.all(np.abs(xq[1:2 * M:2]) <= 64)
     assert not xq[2 * M:].any()
+
+
+@pytest.mark.parametrize("M,N,K,bpw", [(300, 520, 1000, 4), (1024, 768, 4096, 3), (260, 260, 256, 2),
+                                       (512, 1280, 3072, 4)])
+def test_gemm_prefill_ragged_two_sm_tiles(gcb, M, N, K, bpw):
+    # the prefill product on 256 x 256 tiles computed by CTA pairs: ragged M and
+    # N (partial tiles on both sides of the pair) and a K that is not a multiple
+    # of the 64-deep step (1000); decoded-weight bar 1e-4
+    W = synth.gaussian_weights(N, K, 0.02, M + N)
+    s = synth.suggest_scale(W, bpw)
+    rs = 31
+    i1, i2 = _layer_codes(gcb, W, bpw, rs, s)
+    X = synth.activations_bf16(M, K, N)
+    Y = gu.to_np(e8.e8_gemm(gcb, gu.bf16_dev(X), i1, i2, N, K, bpw, rs, s,
+                            mode=e8.E8_GEMM_DECODED_W))
+    wd = orc.decode(gu.to_np(i1), None if i2 is None else gu.to_np(i2), N, K, bpw, rs, s)
+    err = gu.rel_fro(Y, orc.gemm(X, wd))
+    assert err < BAR_DECODED, (M, N, K, err)
+    assert e8.e8_sync_status(gcb) == e8.E8_OK
