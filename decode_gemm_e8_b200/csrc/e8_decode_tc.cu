@@ -167,6 +167,14 @@ __device__ __forceinline__ void load_codes(const DecodeTcParams& p, uint8_t* dst
     bulk_load(dst + 2048, static_cast<const uint8_t*>(p.idx2) + slab * (int64_t)i2b, i2b, bar);
 }
 
+// L2 prefetch of one slab's index words (no shared memory, no completion).
+template <int BPW>
+__device__ __forceinline__ void prefetch_codes_l2(const DecodeTcParams& p, int64_t slab) {
+  constexpr uint32_t i2b = BPW == 4 ? 2048u : (BPW == 3 ? 1024u : 0u);
+  bulk_prefetch_l2(p.idx1 + slab * dtc::GROUPS, 2048u);
+  if (BPW > 2) bulk_prefetch_l2(static_cast<const uint8_t*>(p.idx2) + slab * (int64_t)i2b, i2b);
+}
+
 template <int BPW>
 __global__ void __launch_bounds__(dtc::THREADS, 1)
     k_decode_tc(const DecodeTcParams p, const __grid_constant__ CUtensorMap tmOut) {
@@ -279,6 +287,10 @@ __global__ void __launch_bounds__(dtc::THREADS, 1)
         load_codes<BPW>(p, codes + s * CODE_BYTES, &code_full[s],
                         (int64_t)blockIdx.x + i * gridDim.x);
         ++issued;
+        // the ring holds two slabs, less than the latency of a copy from
+        // HBM; bring the index words of slabs i + 3 and i + 4 into L2 now
+        for (int64_t f = i + 3; f < i + 5 && f < nsl; ++f)
+          prefetch_codes_l2<BPW>(p, (int64_t)blockIdx.x + f * gridDim.x);
         if (++s == CSTAGES) {
           s = 0;
           ph ^= 1u;
