@@ -100,8 +100,10 @@ struct DeviceCodebook {
 };
 
 // Codebook index of the lattice vector v (doubled coordinates), or -1 if v is
-// not one of the 65536 entries.
-__device__ __forceinline__ int rank_vector(const DeviceCodebook& cb, const int* v) {
+// not one of the 65536 entries; hkeys / hvals: the hash of the positive
+// representatives.
+__device__ __forceinline__ int rank_vector(const uint32_t* hkeys, const uint32_t* hvals,
+                                           const int* v) {
   int first = 0;
   for (int j = 0; j < 8; ++j) {
     if (v[j] != 0) { first = v[j]; break; }
@@ -115,9 +117,9 @@ __device__ __forceinline__ int rank_vector(const DeviceCodebook& cb, const int* 
   uint32_t key = pack_vec(w);
   uint32_t s = hash_slot(key);
   for (int probe = 0; probe < kHashSlots; ++probe) {
-    uint32_t k = __ldg(cb.hkeys + s);
+    uint32_t k = __ldg(hkeys + s);
     if (k == key) {
-      int q = (int)__ldg(cb.hvals + s);
+      int q = (int)__ldg(hvals + s);
       int idx = first > 0 ? 2 * q + 1 : 2 * q + 2;
       return idx < kCbSize ? idx : -1;
     }
@@ -125,6 +127,10 @@ __device__ __forceinline__ int rank_vector(const DeviceCodebook& cb, const int* 
     s = (s + 1) & (kHashSlots - 1);
   }
   return -1;
+}
+
+__device__ __forceinline__ int rank_vector(const DeviceCodebook& cb, const int* v) {
+  return rank_vector(cb.hkeys, cb.hvals, v);
 }
 
 }  // namespace e8

@@ -296,72 +296,156 @@ __device__ int exact_cmp(const float (&u)[8], const int (&Za)[8], const int (&Zb
   return exact_sign_sum(t, 9);
 }
 
-// binary64 |u - (base + v_c) / den|^2 with explicit roundings (no contraction),
-// so that both passes below compute bit-identical values; Z receives base + v_c.
-__device__ __forceinline__ double approx_d2(const DeviceCodebook& cb, const float (&u)[8],
-                                            const int (&base)[8], int c, double inv_den,
-                                            int (&Z)[8]) {
-  const int8_t* v = cb.vecs + 8 * c;
-  double s = 0.0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    Z[i] = base[i] + v[i];
-    double x = __dsub_rn((double)u[i], __dmul_rn((double)Z[i], inv_den));
-    s = __dadd_rn(s, __dmul_rn(x, x));
-  }
-  return s;
-}
-
-// Exact argmin of |u - (base + v_c)/den|^2 by one warp over the candidates c =
-// list[0..n) (or c in [0, n) when list is null), plus `extra` when >= 0;
-// smallest index on ties.  All lanes return the same index.
-__device__ int warp_exact_argmin(const DeviceCodebook& cb, const float (&u)[8],
-                                 const int (&base)[8], int den, int n, const int32_t* list,
-                                 int extra) {
+// Exact argmin of |u - (base + v_c)/den|^2 by one warp over the listed
+// norm-12 points (all of squared norm 12, doubled 48) plus `extra` when >= 0;
+// smallest index on ties.  On the list |base + v|^2 - 2 den <u, base + v>
+// differs from -2 <den u - base, v> by a constant, so each lane ranks its
+// candidates by the fp32 score <T, v>, T = den u - base, read from the
+// shared-memory copy sl of the list (eight fp32 coordinates per point), and
+// compares two candidates exactly whenever their scores are within tol of
+// each other: every decision of the lane scan and of the warp tournament is
+// then the exact one, so the winner is the exact argmin.
+// Bound: t_k = fl32(T_k) within 2^-24 |T_k|; the fused chain of eight
+// products with |v_k| <= 6 adds at most 8 roundings of 2^-24 6 S, S = sum
+// |t_k|; a score is within 54 2^-24 S (1 + 2^-20) < 2^-18 S of <T, v>, the
+// difference of two within 2^-17 S; tol = 2^-15 (S + 1) covers it.
+__device__ int warp_list_argmin(const DeviceCodebook& cb, const float4* sl, const float (&u)[8],
+                                const int (&base)[8], int den, int extra) {
   const int lane = threadIdx.x & 31;
-  const double inv_den = 1.0 / den;
-  const int total = n + (extra >= 0 ? 1 : 0);
-  auto cand = [&](int i) { return i < n ? (list ? (int)__ldg(list + i) : i) : extra; };
-  double dmin = INFINITY;
-  int Z[8];
-  for (int i = lane; i < total; i += 32)
-    dmin = fmin(dmin, approx_d2(cb, u, base, cand(i), inv_den, Z));
+  float t[8];
+  float S = 0.0f;
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) dmin = fmin(dmin, __shfl_xor_sync(0xffffffffu, dmin, off));
-  const double lim = dmin * (1.0 + 0x1p-40);
-  // lane-local exact winner among the short list, then a warp tournament
-  int best = -1;
-  int Zw[8];
-  for (int i = lane; i < total; i += 32) {
-    const int c = cand(i);
-    double s = approx_d2(cb, u, base, c, inv_den, Z);
-    if (!(s <= lim)) continue;
-    int cmp = best < 0 ? 1 : exact_cmp(u, Zw, Z, den);
-    if (cmp > 0 || (cmp == 0 && c < best)) {
-      best = c;
+  for (int k = 0; k < 8; ++k) {
+    t[k] = __fsub_rn(__fmul_rn((float)den, u[k]), (float)base[k]);
+    S += fabsf(t[k]);
+  }
+  const float tol = 0x1p-15f * (S * 1.0001f + 1.0f);
+  auto z_of = [&](int c, int (&Z)[8]) {
 #pragma unroll
-      for (int k = 0; k < 8; ++k) Zw[k] = Z[k];
+    for (int k = 0; k < 8; ++k) Z[k] = base[k] + (int)cb.vecs[8 * c + k];
+  };
+  // true when candidate list[j] (score sj) beats list[i] (score si)
+  auto beats = [&](int j, float sj, int i, float si) -> bool {
+    if (i < 0) return j >= 0;
+    if (j < 0) return false;
+    if (sj > si + tol) return true;
+    if (sj < si - tol) return false;
+    const int cj = __ldg(cb.clist + j), ci = __ldg(cb.clist + i);
+    int Zi[8], Zj[8];
+    z_of(ci, Zi);
+    z_of(cj, Zj);
+    const int cmp = exact_cmp(u, Zi, Zj, den);
+    return cmp > 0 || (cmp == 0 && cj < ci);
+  };
+  float bs = -INFINITY;
+  int bi = -1;
+  for (int i = lane; i < cb.clist_len; i += 32) {
+    const float4 a = sl[2 * i], b = sl[2 * i + 1];
+    float sc = __fmul_rn(t[0], a.x);
+    sc = __fmaf_rn(t[1], a.y, sc);
+    sc = __fmaf_rn(t[2], a.z, sc);
+    sc = __fmaf_rn(t[3], a.w, sc);
+    sc = __fmaf_rn(t[4], b.x, sc);
+    sc = __fmaf_rn(t[5], b.y, sc);
+    sc = __fmaf_rn(t[6], b.z, sc);
+    sc = __fmaf_rn(t[7], b.w, sc);
+    if (beats(i, sc, bi, bs)) {
+      bi = i;
+      bs = sc;
     }
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) {
-    int other = __shfl_xor_sync(0xffffffffu, best, off);
-    if (other >= 0) {
-      if (best < 0) {
-        best = other;
-      } else if (other != best) {
-        int Zo[8], Zb[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          Zo[i] = base[i] + cb.vecs[8 * other + i];
-          Zb[i] = base[i] + cb.vecs[8 * best + i];
-        }
-        int s = exact_cmp(u, Zb, Zo, den);
-        if (s > 0 || (s == 0 && other < best)) best = other;
-      }
+    const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+    const float os = __shfl_xor_sync(0xffffffffu, bs, off);
+    if (beats(oi, os, bi, bs)) {
+      bi = oi;
+      bs = os;
+    }
+  }
+  int best = bi < 0 ? -1 : __ldg(cb.clist + bi);
+  if (extra >= 0) {
+    if (best < 0) {
+      best = extra;
+    } else {
+      int Zb[8], Ze[8];
+      z_of(best, Zb);
+      z_of(extra, Ze);
+      const int cmp = exact_cmp(u, Zb, Ze, den);
+      if (cmp > 0 || (cmp == 0 && extra < best)) best = extra;
     }
   }
   return best < 0 ? 0 : best;
+}
+
+// Exact argmin of |u - (base + v_c)/den|^2 by one warp over c = 0 .. n - 1,
+// smallest index on ties.  Each lane ranks its candidates by the fp32 score
+// q_c - 2 <T, v_c>, q_c = |v_c|^2 (exact), T = den u - base, which differs
+// from den^2 |u - (base + v_c)/den|^2 by a constant; two scores within tol
+// of each other are compared exactly.  Bound: <T, v> is within 2^-18 S of
+// its value (as in warp_list_argmin, S = sum |t_k|), the subtraction adds
+// 2^-24 (48 + 12 S), so a score is within 2^-17 S + 2^-19 and a difference
+// within 2^-16 S + 2^-18; tol = 2^-14 (S + 1).
+__device__ int warp_full_argmin(const DeviceCodebook& cb, const float (&u)[8],
+                                const int (&base)[8], int den, int n) {
+  const int lane = threadIdx.x & 31;
+  float t[8];
+  float S = 0.0f;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    t[k] = __fsub_rn(__fmul_rn((float)den, u[k]), (float)base[k]);
+    S += fabsf(t[k]);
+  }
+  const float tol = 0x1p-14f * (S * 1.0001f + 1.0f);
+  auto z_of = [&](int c, int (&Z)[8]) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) Z[k] = base[k] + (int)cb.vecs[8 * c + k];
+  };
+  // true when candidate cj (score sj) beats ci (score si)
+  auto beats = [&](int cj, float sj, int ci, float si) -> bool {
+    if (ci < 0) return cj >= 0;
+    if (cj < 0) return false;
+    if (sj < si - tol) return true;
+    if (sj > si + tol) return false;
+    int Zi[8], Zj[8];
+    z_of(ci, Zi);
+    z_of(cj, Zj);
+    const int cmp = exact_cmp(u, Zi, Zj, den);
+    return cmp > 0 || (cmp == 0 && cj < ci);
+  };
+  const uint2* vv = reinterpret_cast<const uint2*>(cb.vecs);
+  float bs = INFINITY;
+  int bc = -1;
+  for (int c = lane; c < n; c += 32) {
+    const uint2 w = __ldg(vv + c);
+    float v[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      v[k] = (float)(int8_t)(w.x >> (8 * k));
+      v[k + 4] = (float)(int8_t)(w.y >> (8 * k));
+    }
+    float q = 0.0f, d = 0.0f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      q = __fmaf_rn(v[k], v[k], q);
+      d = __fmaf_rn(t[k], v[k], d);
+    }
+    const float sc = __fsub_rn(q, 2.0f * d);
+    if (beats(c, sc, bc, bs)) {
+      bc = c;
+      bs = sc;
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const int oc = __shfl_xor_sync(0xffffffffu, bc, off);
+    const float os = __shfl_xor_sync(0xffffffffu, bs, off);
+    if (beats(oc, os, bc, bs)) {
+      bc = oc;
+      bs = os;
+    }
+  }
+  return bc < 0 ? 0 : bc;
 }
 
 // One warp per work item: exact brute force over the whole candidate set, or
@@ -372,6 +456,14 @@ __global__ void __launch_bounds__(256) k_encode_slow(const WorkItem* in, const u
                                                      uint32_t* out_count, int bpw,
                                                      uint16_t* idx1, void* idx2,
                                                      DeviceCodebook cb) {
+  // the listed norm-12 points as fp32 coordinates (exact small integers)
+  extern __shared__ float4 s_list[];
+  for (int i = threadIdx.x; i < cb.clist_len; i += blockDim.x) {
+    const int8_t* v = cb.vecs + 8 * __ldg(cb.clist + i);
+    s_list[2 * i] = make_float4(v[0], v[1], v[2], v[3]);
+    s_list[2 * i + 1] = make_float4(v[4], v[5], v[6], v[7]);
+  }
+  __syncthreads();
   const uint64_t n = (uint64_t)min((unsigned long long)*in_count, (unsigned long long)cap);
   const uint64_t warp = ((uint64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const uint64_t nwarps = ((uint64_t)gridDim.x * blockDim.x) >> 5;
@@ -386,8 +478,8 @@ __global__ void __launch_bounds__(256) k_encode_slow(const WorkItem* in, const u
     if (mask & kWorkStage1) {
       int zero[8] = {0, 0, 0, 0, 0, 0, 0, 0};
       const int i1 = (mask & kWorkStage1List)
-                         ? warp_exact_argmin(cb, u, zero, 2, cb.clist_len, cb.clist, (int)it.cand)
-                         : warp_exact_argmin(cb, u, zero, 2, kCbSize, nullptr, -1);
+                         ? warp_list_argmin(cb, s_list, u, zero, 2, (int)it.cand)
+                         : warp_full_argmin(cb, u, zero, 2, kCbSize);
       if (lane == 0) {
         idx1[g] = (uint16_t)i1;
         if (bpw > 2) {
@@ -413,9 +505,8 @@ __global__ void __launch_bounds__(256) k_encode_slow(const WorkItem* in, const u
 #pragma unroll
       for (int i = 0; i < 8; ++i) base[i] = (m / 2) * (int)cb.vecs[8 * i1 + i];
       const int i2 = (mask & kWorkStage2List)
-                         ? warp_exact_argmin(cb, u, base, m, cb.clist_len, cb.clist, (int)it.cand)
-                         : warp_exact_argmin(cb, u, base, m, bpw == 3 ? 256 : kCbSize, nullptr,
-                                             -1);
+                         ? warp_list_argmin(cb, s_list, u, base, m, (int)it.cand)
+                         : warp_full_argmin(cb, u, base, m, bpw == 3 ? 256 : kCbSize);
       if (lane == 0) {
         if (bpw == 3) reinterpret_cast<uint8_t*>(idx2)[g] = (uint8_t)i2;
         else reinterpret_cast<uint16_t*>(idx2)[g] = (uint16_t)i2;
@@ -464,17 +555,19 @@ cudaError_t launch_encode(const DeviceCodebook& cb, const float* W, int64_t N, i
   // brute force takes a second round
   WorkItem* r1 = work;
   WorkItem* r2 = work + work_cap;
+  const size_t slow_smem = (size_t)(cb.clist_len > 0 ? cb.clist_len : 0) * 2 * sizeof(float4);
+  if ((e = ensure_smem_limit(k_encode_slow, kMaxDynSmem)) != cudaSuccess) return e;
   e = launch_encode_leader(cb, r1, work_count, work_cap, r2, work_count + 1, bpw, idx1, idx2,
                            sm_count, st);
   if (e != cudaSuccess) return e;
-  k_encode_slow<<<sm_count * 4, 256, 0, st>>>(r2, work_count + 1, work_cap, r1, work_count + 2,
+  k_encode_slow<<<sm_count * 4, 256, slow_smem, st>>>(r2, work_count + 1, work_cap, r1, work_count + 2,
                                               bpw, idx1, idx2, cb);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (bpw == 2) return cudaSuccess;
   e = launch_encode_leader(cb, r1, work_count + 2, work_cap, r2, work_count + 3, bpw, idx1, idx2,
                            sm_count, st);
   if (e != cudaSuccess) return e;
-  k_encode_slow<<<sm_count * 4, 256, 0, st>>>(r2, work_count + 3, work_cap, nullptr, nullptr, bpw,
+  k_encode_slow<<<sm_count * 4, 256, slow_smem, st>>>(r2, work_count + 3, work_cap, nullptr, nullptr, bpw,
                                               idx1, idx2, cb);
   return cudaGetLastError();
 }

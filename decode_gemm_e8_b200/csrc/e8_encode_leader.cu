@@ -168,11 +168,25 @@ struct Best {
 
 enum { kLsOk = 0, kLsNeedC = 1, kLsFallback = 2 };
 
+// The tables the class search reads, passed by value so that the searches
+// below can stay out of line: one copy of their code serves both stages and
+// every call site (the kernel is bound by instruction fetch and divergence
+// when each call site inlines its own copy).
+struct LsTabs {
+  const uint32_t* hkeys;
+  const uint32_t* hvals;
+  const int8_t* vecs;
+};
+
+__device__ __noinline__ int ls_rank(const LsTabs& tb, const int (&v)[8]) {
+  return rank_vector(tb.hkeys, tb.hvals, v);
+}
+
 // Nearest point of the whole codebook to T (doubled coordinates, binary64,
 // exactly the target).  kLsOk: *idx is the answer.  kLsNeedC: the answer is
 // *idx unless a point of the x1 = 0, |x2| = 2 part of the norm-12 shell is
 // nearer.  kLsFallback: undecided.
-__device__ int leader_search(const DeviceCodebook& cb, const double (&t)[8], int* idx) {
+__device__ __noinline__ int leader_search(const LsTabs tb, const double (&t)[8], int* idx) {
   using namespace ls;
   double b[8];
   int p[8];
@@ -202,7 +216,7 @@ __device__ int leader_search(const DeviceCodebook& cb, const double (&t)[8], int
   {
     int V[8];
     class8_best(kFullCls[bestcls], t, b, p, nneg, V);
-    const int r = rank_vector(cb, V);
+    const int r = ls_rank(tb, V);
     if (r < 0) return kLsFallback;  // full shells are always members
     best.offer(bscore, r);
   }
@@ -222,7 +236,7 @@ __device__ int leader_search(const DeviceCodebook& cb, const double (&t)[8], int
   bool need_c = false;
   int V[8];
   class8_best(kS12Cls[c12], t, b, p, nneg, V);
-  int r12 = rank_vector(cb, V);
+  int r12 = ls_rank(tb, V);
   if (r12 >= 0) {
     best.offer(s12, r12);
     best.shadow(s12b);
@@ -255,7 +269,7 @@ __device__ int leader_search(const DeviceCodebook& cb, const double (&t)[8], int
       W[1] = part == 0 ? 0 : s1 * (part == 1 ? 2 : 4);
 #pragma unroll
       for (int k = 0; k < 6; ++k) W[p6[k]] = sgn_of(t[p6[k]]) * (int)cl.l[k];
-      const int r = rank_vector(cb, W);
+      const int r = ls_rank(tb, W);
       if (part < 2) {
         if (r < 0) return kLsFallback;  // these parts are kept whole
         best.offer(sb, r);
@@ -278,7 +292,7 @@ __device__ int leader_search(const DeviceCodebook& cb, const double (&t)[8], int
 
 // Nearest of the first 256 codebook entries (origin, the 240 points of norm 2,
 // 15 points of norm 4) to T (doubled coordinates).
-__device__ int c28_search(const DeviceCodebook& cb, const double (&t)[8], int* idx) {
+__device__ __noinline__ int c28_search(const LsTabs tb, const double (&t)[8], int* idx) {
   using namespace ls;
   double b[8];
   int p[8];
@@ -296,12 +310,12 @@ __device__ int c28_search(const DeviceCodebook& cb, const double (&t)[8], int* i
   for (int c = 0; c < 2; ++c) {  // the two classes of norm 2 (doubled 8)
     int V[8];
     const double s = class8_best(kFullCls[c], t, b, p, nneg, V);
-    const int r = rank_vector(cb, V);
+    const int r = ls_rank(tb, V);
     if (r < 0 || r >= 241) return kLsFallback;
     best.offer(__dsub_rn(8.0, 2.0 * s), r);
   }
   for (int i = 241; i < 256; ++i) {
-    const int8_t* v = cb.vecs + 8 * i;
+    const int8_t* v = tb.vecs + 8 * i;
     double s = 0.0;
 #pragma unroll
     for (int k = 0; k < 8; ++k) s = __dadd_rn(s, __dmul_rn((double)v[k], t[k]));
@@ -330,12 +344,14 @@ __device__ __forceinline__ void push_item(WorkItem* list, uint32_t* count, uint6
 }
 
 // One thread per work item: class search for the undecided stages; what stays
-// undecided goes to `out` for the warp brute force.
+// undecided goes to `out` for the warp brute force.  Both stages go through
+// one call site of the (out-of-line) search.
 __global__ void __launch_bounds__(256) k_encode_leader(const WorkItem* in, const uint32_t* in_count,
                                                        uint64_t cap, WorkItem* out,
                                                        uint32_t* out_count, int bpw,
                                                        uint16_t* idx1, void* idx2,
                                                        DeviceCodebook cb) {
+  const LsTabs tb{cb.hkeys, cb.hvals, cb.vecs};
   const uint64_t n = (uint64_t)min((unsigned long long)*in_count, (unsigned long long)cap);
   const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
   for (uint64_t w = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; w < n; w += stride) {
@@ -345,39 +361,43 @@ __global__ void __launch_bounds__(256) k_encode_leader(const WorkItem* in, const
     for (int i = 0; i < 8; ++i) u[i] = it.u[i];
     const int64_t g = it.group;
     const uint32_t mask = it.mask;
-    int i1 = -1;
-    if (mask & kWorkStage1) {
+    if (!(mask & kWorkStage1) && (bpw == 2 || !(mask & kWorkStage2))) continue;
+    // stage 1 target 2u; stage 2 target (2u - V1) / beta (doubled coordinates)
+    int stage = (mask & kWorkStage1) ? 1 : 2;
+    int i1 = stage == 1 ? -1 : (int)idx1[g];
+    for (;;) {
       double t[8];
+      if (stage == 1) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) t[i] = 2.0 * (double)u[i];
+        for (int i = 0; i < 8; ++i) t[i] = 2.0 * (double)u[i];
+      } else {
+        const int8_t* v1 = cb.vecs + 8 * i1;
+        const double k = bpw == 3 ? 2.0 : 4.0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) t[i] = k * __dsub_rn(2.0 * (double)u[i], (double)v1[i]);
+      }
       int r = 0;
-      const int st = leader_search(cb, t, &r);
+      const int st = (stage == 2 && bpw == 3) ? c28_search(tb, t, &r) : leader_search(tb, t, &r);
       if (st != kLsOk) {
-        const uint32_t m2 = bpw > 2 ? kWorkStage2 : 0u;
-        push_item(out, out_count, cap, cb.status, u, g,
-                  kWorkStage1 | m2 | (st == kLsNeedC ? kWorkStage1List : 0u), (uint32_t)r);
+        uint32_t m;
+        if (stage == 1)
+          m = kWorkStage1 | (bpw > 2 ? kWorkStage2 : 0u) | (st == kLsNeedC ? kWorkStage1List : 0u);
+        else
+          m = kWorkStage2 | (st == kLsNeedC ? kWorkStage2List : 0u);
+        push_item(out, out_count, cap, cb.status, u, g, m, (uint32_t)r);
+        break;
+      }
+      if (stage == 1) {
+        idx1[g] = (uint16_t)r;
+        if (bpw == 2) break;
+        i1 = r;
+        stage = 2;
         continue;
       }
-      i1 = r;
-      idx1[g] = (uint16_t)i1;
+      if (bpw == 3) reinterpret_cast<uint8_t*>(idx2)[g] = (uint8_t)r;
+      else reinterpret_cast<uint16_t*>(idx2)[g] = (uint16_t)r;
+      break;
     }
-    if (bpw == 2 || !(mask & (kWorkStage1 | kWorkStage2))) continue;
-    if (i1 < 0) i1 = idx1[g];
-    // stage 2 target in doubled coordinates: (2u - V1) / beta
-    const int8_t* v1 = cb.vecs + 8 * i1;
-    const double k = bpw == 3 ? 2.0 : 4.0;
-    double t[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) t[i] = k * __dsub_rn(2.0 * (double)u[i], (double)v1[i]);
-    int r = 0;
-    const int st = bpw == 3 ? c28_search(cb, t, &r) : leader_search(cb, t, &r);
-    if (st != kLsOk) {
-      push_item(out, out_count, cap, cb.status, u, g,
-                kWorkStage2 | (st == kLsNeedC ? kWorkStage2List : 0u), (uint32_t)r);
-      continue;
-    }
-    if (bpw == 3) reinterpret_cast<uint8_t*>(idx2)[g] = (uint8_t)r;
-    else reinterpret_cast<uint16_t*>(idx2)[g] = (uint16_t)r;
   }
 }
 
