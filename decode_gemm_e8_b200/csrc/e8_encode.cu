@@ -385,8 +385,10 @@ __device__ int warp_list_argmin(const DeviceCodebook& cb, const float4* sl, cons
 // of each other are compared exactly.  Bound: <T, v> is within 2^-18 S of
 // its value (as in warp_list_argmin, S = sum |t_k|), the subtraction adds
 // 2^-24 (48 + 12 S), so a score is within 2^-17 S + 2^-19 and a difference
-// within 2^-16 S + 2^-18; tol = 2^-14 (S + 1).
-__device__ int warp_full_argmin(const DeviceCodebook& cb, const float (&u)[8],
+// within 2^-16 S + 2^-18; tol = 2^-14 (S + 1).  Out of line: few items take
+// it, and its eight loads in flight would crowd the registers of the list
+// search beside it.
+__device__ __noinline__ int warp_full_argmin(const DeviceCodebook& cb, const float (&u)[8],
                                 const int (&base)[8], int den, int n) {
   const int lane = threadIdx.x & 31;
   float t[8];
@@ -413,27 +415,38 @@ __device__ int warp_full_argmin(const DeviceCodebook& cb, const float (&u)[8],
     const int cmp = exact_cmp(u, Zi, Zj, den);
     return cmp > 0 || (cmp == 0 && cj < ci);
   };
+  // eight candidates per lane and step, their loads issued together (a lone
+  // warp scans up to 65536 entries: one load at a time would leave it bound
+  // by the L2 latency)
   const uint2* vv = reinterpret_cast<const uint2*>(cb.vecs);
   float bs = INFINITY;
   int bc = -1;
-  for (int c = lane; c < n; c += 32) {
-    const uint2 w = __ldg(vv + c);
-    float v[8];
+  for (int c0 = lane; c0 < n; c0 += 32 * 8) {
+    uint2 w[8];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      v[k] = (float)(int8_t)(w.x >> (8 * k));
-      v[k + 4] = (float)(int8_t)(w.y >> (8 * k));
-    }
-    float q = 0.0f, d = 0.0f;
+    for (int j = 0; j < 8; ++j)
+      w[j] = c0 + 32 * j < n ? __ldg(vv + c0 + 32 * j) : make_uint2(0u, 0u);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      q = __fmaf_rn(v[k], v[k], q);
-      d = __fmaf_rn(t[k], v[k], d);
-    }
-    const float sc = __fsub_rn(q, 2.0f * d);
-    if (beats(c, sc, bc, bs)) {
-      bc = c;
-      bs = sc;
+    for (int j = 0; j < 8; ++j) {
+      const int c = c0 + 32 * j;
+      if (c >= n) break;
+      float v[8];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        v[k] = (float)(int8_t)(w[j].x >> (8 * k));
+        v[k + 4] = (float)(int8_t)(w[j].y >> (8 * k));
+      }
+      float q = 0.0f, d = 0.0f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        q = __fmaf_rn(v[k], v[k], q);
+        d = __fmaf_rn(t[k], v[k], d);
+      }
+      const float sc = __fsub_rn(q, 2.0f * d);
+      if (beats(c, sc, bc, bs)) {
+        bc = c;
+        bs = sc;
+      }
     }
   }
 #pragma unroll
@@ -451,7 +464,7 @@ __device__ int warp_full_argmin(const DeviceCodebook& cb, const float (&u)[8],
 // One warp per work item: exact brute force over the whole candidate set, or
 // over the listed norm-12 points plus the item's best other candidate.  A
 // stage 1 settled here sends its stage 2 back (to `out`) for the class search.
-__global__ void __launch_bounds__(256) k_encode_slow(const WorkItem* in, const uint32_t* in_count,
+__global__ void __launch_bounds__(256, 4) k_encode_slow(const WorkItem* in, const uint32_t* in_count,
                                                      uint64_t cap, WorkItem* out,
                                                      uint32_t* out_count, int bpw,
                                                      uint16_t* idx1, void* idx2,
@@ -556,7 +569,7 @@ cudaError_t launch_encode(const DeviceCodebook& cb, const float* W, int64_t N, i
   WorkItem* r1 = work;
   WorkItem* r2 = work + work_cap;
   const size_t slow_smem = (size_t)(cb.clist_len > 0 ? cb.clist_len : 0) * 2 * sizeof(float4);
-  if ((e = ensure_smem_limit(k_encode_slow, kMaxDynSmem)) != cudaSuccess) return e;
+  if ((e = ensure_smem_limit(k_encode_slow, kMaxDynSmem, true)) != cudaSuccess) return e;
   e = launch_encode_leader(cb, r1, work_count, work_cap, r2, work_count + 1, bpw, idx1, idx2,
                            sm_count, st);
   if (e != cudaSuccess) return e;

@@ -345,8 +345,10 @@ __device__ __forceinline__ void push_item(WorkItem* list, uint32_t* count, uint6
 
 // One thread per work item: class search for the undecided stages; what stays
 // undecided goes to `out` for the warp brute force.  Both stages go through
-// one call site of the (out-of-line) search.
-__global__ void __launch_bounds__(256) k_encode_leader(const WorkItem* in, const uint32_t* in_count,
+// one call site of the (out-of-line) search.  Four blocks per SM (64
+// registers): the search is latency-bound and gains more from warps in
+// flight than it loses to the few spilled values.
+__global__ void __launch_bounds__(256, 4) k_encode_leader(const WorkItem* in, const uint32_t* in_count,
                                                        uint64_t cap, WorkItem* out,
                                                        uint32_t* out_count, int bpw,
                                                        uint16_t* idx1, void* idx2,
