@@ -456,8 +456,14 @@ def _profile_other(e8, synth, dev, mode):
         W = synth.gaussian_weights(lay.N, lay.K, lay.std, lay.w_seed)
         s = synth.suggest_scale(W, lay.bpw)
         Wd = torch.from_numpy(W).to(dev)
+        ws = torch.empty(e8.e8_workspace_bytes(e8.E8_OP_ENCODE, 0, lay.N, lay.K, lay.bpw),
+                         dtype=torch.uint8, device=dev)
         for _ in range(2):
-            e8.e8_encode(cb, Wd, lay.bpw, lay.rht_seed, s)
+            e8.e8_encode(cb, Wd, lay.bpw, lay.rht_seed, s, workspace=ws)
+            cnt = ws[:16].view(torch.int32).cpu().tolist()
+            print("encode %dx%d at %d bpw: %d groups; fast path left %d open, brute force "
+                  "took %d, second round %d / %d" % (lay.N, lay.K, lay.bpw, lay.N * lay.K // 8,
+                                                     cnt[0], cnt[1], cnt[2], cnt[3]))
     else:
         M, N, K, bpw = 16, 14336, 4096, 4
         codes = [_random_codes(torch, dev, N, K, bpw, gen) for _ in range(3)]
@@ -675,9 +681,12 @@ def _other_rows(e8, synth, cb, Wd, W, codes, X, N, K, bpw, rs, s, dev, stream, a
     ms = _time_graphs(enc, n_enc, 2, stream)
     t = ms / 1e3 / n_enc
     byt = N * K * (4 + bpw / 8)
+    cnt = wsb[:16].view(torch.int32).cpu().tolist()   # documented counters of e8_encode
     rows["encode"] = {"weights_per_s": N * K / t, "ms": t * 1e3, "GB_s": byt / t / 1e9,
                       "hbm_frac": round(byt / t / 1e9 / peaks["hbm_gbs"], 4),
-                      "bytes_per_weight": 4 + bpw / 8}
+                      "bytes_per_weight": 4 + bpw / 8, "groups": N * K // 8,
+                      "groups_class_search": cnt[0], "groups_brute_force": cnt[1],
+                      "groups_second_round": [cnt[2], cnt[3]]}
     # four outputs (134 MB) so that the written weights leave the L2 cache
     outs = [torch.empty((N, K), dtype=torch.bfloat16, device=dev) for _ in range(4)]
 

@@ -107,7 +107,13 @@ int e8_rht_forward(const e8_codebook* cb, const float* W, int64_t N, int64_t K,
  * global scale.  Every index equals the exact nearest codebook point of the
  * transformed, scaled group (smallest index on ties); groups with a
  * non-finite coordinate get index 0.  workspace: at least
- * e8_workspace_bytes(E8_OP_ENCODE, 0, N, K, bpw) bytes, contents ignored. */
+ * e8_workspace_bytes(E8_OP_ENCODE, 0, N, K, bpw) bytes, contents ignored.
+ * When the call has completed on the stream, the first four uint32 words of
+ * the workspace hold diagnostic counts of groups: [0] left open by the
+ * Conway-Sloane fast path (one class search per open stage follows), [1]
+ * left for the exact brute force after it, [2] stage-2 searches of groups
+ * whose stage 1 the brute force settled, [3] of those, left for a second
+ * brute force. */
 int e8_encode(const e8_codebook* cb, const float* W, int64_t N, int64_t K, int bpw,
               uint64_t rht_seed, float scale, uint16_t* idx1, void* idx2, void* workspace,
               size_t ws_bytes, void* stream);
