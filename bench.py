@@ -210,7 +210,7 @@ def run_ours(args):
     if args.profile == "decode":
         _profile_decode(e8, dev)
         return
-    if args.profile in ("dense_up", "dense_out", "encode", "gemm_mlp"):
+    if args.profile in ("dense_up", "dense_out", "encode", "gemm_mlp", "ep_decode"):
         _profile_other(e8, synth, dev, args.profile)
         return
     peaks = _peaks()
@@ -438,7 +438,9 @@ def _profile_other(e8, synth, dev, mode):
       dense_out  the same for the DiT out projection (3072 x 3072, 4 bpw)
       encode     two encodes of the 4096 x 4096 Llama layer at 4 bpw
       gemm_mlp   three small-batch products (16 tokens) of a 14336 x 4096
-                 matrix at 4 bpw on pre-transformed activations (k_gemm_q8)"""
+                 matrix at 4 bpw on pre-transformed activations (k_gemm_q8)
+      ep_decode  the entropy-coded variant: three decodes of a 14336 x 4096
+                 Gaussian matrix at delta 0.075 (about 4 bpp)"""
     import torch
     gen = torch.Generator(device=dev)
     gen.manual_seed(7)
@@ -451,6 +453,12 @@ def _profile_other(e8, synth, dev, mode):
                          dtype=torch.uint8, device=dev)
         for _ in range(2):
             e8.e8_gemm(cb, X, c1, c2, N, K, bpw, 1, 0.02, mode=e8.E8_GEMM_DECODED_W, workspace=ws)
+    elif mode == "ep_decode":
+        W = torch.from_numpy(synth.gaussian_weights(14336, 4096, 0.02, 4)).to(dev)
+        m = e8.e8_ep_encode(cb, W, 0.075)
+        out = torch.empty((14336, 4096), dtype=torch.bfloat16, device=dev)
+        for _ in range(3):
+            e8.e8_ep_decode_to_bf16(cb, m, out=out)
     elif mode == "encode":
         lay = synth.workloads()[WORKLOAD].layers[0]
         W = synth.gaussian_weights(lay.N, lay.K, lay.std, lay.w_seed)
@@ -529,6 +537,50 @@ def _prefill_rows(e8, synth, cb, dev, stream, peaks):
                                    "bound": "tensor" if flop / (peaks["bf16_tflops"] * 1e12) >=
                                    byt / (peaks["hbm_gbs"] * 1e9) else "hbm"}
         del codes, X, Y, ws
+    return rows
+
+
+def _ep_rows(e8, synth, cb, dev, stream, peaks):
+    """Entropy-coded variant at a 4 bpp target on the DiT out projection
+    (3072 x 3072, Student-t with outlier columns) and the MLP up-projection
+    (14336 x 4096, Gaussian): the step the rate search picks, the actual rate
+    with metadata, the decode to bf16 (stream read + 2 bytes written per
+    weight) and the prefill GEMM on 4096 tokens (decode included)."""
+    import torch
+    rows = {}
+    for name, N, K, W in (("dit_3072_out", 3072, 3072, synth.student_t_outlier_weights(3072, 3072, 7)),
+                          ("mlp_up_14336", 14336, 4096,
+                           synth.gaussian_weights(14336, 4096, 0.015, 4))):
+        Wd = torch.from_numpy(W).to(dev)
+        d = e8.e8_ep_choose_delta(cb, Wd, 4.0)
+        m = e8.e8_ep_encode(cb, Wd, d)
+        outs = [torch.empty((N, K), dtype=torch.bfloat16, device=dev) for _ in range(4)]
+
+        def dec(i, m=m, outs=outs):
+            e8.e8_ep_decode_to_bf16(cb, m, out=outs[i % 4], stream=stream)
+
+        n = 20
+        t = _time_graphs(dec, n, 4, stream) / 1e3 / n
+        byt = m.total_words * 2 + N * K * 2
+        M = 4096
+        X = torch.from_numpy(synth.activations_bf16(M, K, 11).view(np.int16)).to(dev).view(
+            torch.bfloat16)
+        Y = torch.empty((M, N), dtype=torch.float32, device=dev)
+        ws = torch.empty(e8.load_library().e8_ep_gemm_workspace_bytes(M, N, K), dtype=torch.uint8,
+                         device=dev)
+
+        def gem(i, m=m, X=X, Y=Y, ws=ws):
+            e8.e8_ep_gemm(cb, X, m, Y=Y, workspace=ws, stream=stream)
+
+        tg = _time_graphs(gem, 10, 3, stream) / 1e3 / 10
+        flop = 2.0 * M * N * K
+        rows["ep_" + name + "_4bpp"] = {
+            "delta": d, "actual_bpp": round(m.actual_bpp(), 4),
+            "decode_us": round(t * 1e6, 1), "decode_GB_s": round(byt / t / 1e9, 1),
+            "decode_hbm_frac": round(byt / t / 1e9 / peaks["hbm_gbs"], 4),
+            "prefill_TFLOP_s": round(flop / tg / 1e12, 1), "prefill_us": round(tg * 1e6, 1),
+            "prefill_frac": round(flop / tg / 1e12 / peaks["bf16_tflops"], 4)}
+        del Wd, m, outs, X, Y, ws
     return rows
 
 
@@ -701,6 +753,7 @@ def _other_rows(e8, synth, cb, Wd, W, codes, X, N, K, bpw, rs, s, dev, stream, a
                               "hbm_frac": round(byt / t / 1e9 / peaks["hbm_gbs"], 4),
                               "bytes_per_weight": 2 + bpw / 8}
     rows.update(_prefill_rows(e8, synth, cb, dev, stream, peaks))
+    rows.update(_ep_rows(e8, synth, cb, dev, stream, peaks))
     rows.update(_decode_sweep_rows(e8, synth, cb, dev, stream, peaks))
     rows.update(_layer_chain_rows(e8, synth, cb, dev, stream, peaks))
     for Mx in (1, 4):
@@ -801,7 +854,8 @@ def main():
     ap.add_argument("--no-load", action="store_true",
                     help="skip the load phase that precedes the timed region (clock record)")
     ap.add_argument("--profile", nargs="?", const="gemm",
-                    choices=["gemm", "decode", "dense_up", "dense_out", "encode", "gemm_mlp"],
+                    choices=["gemm", "decode", "dense_up", "dense_out", "encode", "gemm_mlp",
+                             "ep_decode"],
                     help="small runs for ncu captures, then exit: 8 eager steps of the "
                          "headline call (gemm), 3 bf16 decodes of a 14336 x 4096 matrix "
                          "(decode), prefill GEMMs (dense_up, dense_out), two encodes "

@@ -20,7 +20,9 @@ import os
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "_lib", "libe8.so")
 
-E8_OK, E8_EINVAL, E8_EWORKSPACE, E8_EDEVICE, E8_ECUDA, E8_ETIMEOUT, E8_ENOMEM = range(7)
+E8_OK, E8_EINVAL, E8_EWORKSPACE, E8_EDEVICE, E8_ECUDA, E8_ETIMEOUT, E8_ENOMEM, E8_EDATA = range(8)
+E8_EP_BLOCK_GROUPS = 64
+E8_EP_TABLE_WORDS = 770
 E8_GEMM_AUTO, E8_GEMM_ACT_RHT, E8_GEMM_DECODED_W, E8_GEMM_ACT_RHT_SMEM, E8_GEMM_SIMT = range(5)
 E8_OP_ENCODE = 100
 
@@ -34,7 +36,10 @@ EXPORTED = ("e8_codebook_build", "e8_codebook_free", "e8_codebook_export", "e8_r
             "e8_workspace_bytes_nh",
             "e8_gemm_host_workspace_bytes", "e8_gemm_auto_mode",
             "e8_workspace_bytes", "e8_sync_status", "e8_debug_wait_timeout", "e8_status_str",
-            "e8_version")
+            "e8_version",
+            "e8_ep_num_blocks", "e8_ep_max_words", "e8_ep_actual_bpp",
+            "e8_ep_encode_workspace_bytes", "e8_ep_gemm_workspace_bytes", "e8_ep_encode",
+            "e8_ep_estimate_bpp", "e8_ep_choose_delta", "e8_ep_decode_to_bf16", "e8_ep_gemm")
 
 _lib = None
 
@@ -90,6 +95,19 @@ def load_library(path: str = LIB_PATH):
         "e8_debug_wait_timeout": ([P, c.c_int, P], c.c_int),
         "e8_status_str": ([c.c_int], c.c_char_p),
         "e8_version": ([], c.c_int),
+        "e8_ep_num_blocks": ([I64, I64], I64),
+        "e8_ep_max_words": ([I64, I64], I64),
+        "e8_ep_actual_bpp": ([I64, I64, I64], c.c_double),
+        "e8_ep_encode_workspace_bytes": ([I64, I64], c.c_size_t),
+        "e8_ep_gemm_workspace_bytes": ([I64, I64, I64], c.c_size_t),
+        "e8_ep_encode": ([P, P, I64, I64, c.c_float, P, I64, P, P, P, c.POINTER(c.c_int64), P,
+                          c.c_size_t, P], c.c_int),
+        "e8_ep_estimate_bpp": ([P, P, I64, I64, c.c_float, c.POINTER(c.c_double), P, c.c_size_t,
+                                P], c.c_int),
+        "e8_ep_choose_delta": ([P, P, I64, I64, c.c_double, c.POINTER(c.c_float), P, c.c_size_t,
+                                P], c.c_int),
+        "e8_ep_decode_to_bf16": ([P, P, I64, P, P, P, I64, I64, P, P], c.c_int),
+        "e8_ep_gemm": ([P, P, I64, P, I64, P, P, P, I64, I64, P, P, c.c_size_t, P], c.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -416,3 +434,92 @@ def e8_gemm_grouped(cb: Codebook, X, items, K: int, bpw: int, workspace=None, st
                                           _ptr(workspace), workspace.numel(), _stream(stream)),
            "e8_gemm_grouped")
     return outs
+
+
+# ------------------------------------------------------ entropy-coded variant --
+class EpMatrix:
+    """Compressed form of one matrix (e8_ep_encode): stream words, block
+    offsets, row scales t, frequency tables (all on the device)."""
+
+    def __init__(self, N, K, delta, words, offsets, t, tables, total_words):
+        self.N, self.K, self.delta = N, K, delta
+        self.words, self.offsets, self.t, self.tables = words, offsets, t, tables
+        self.total_words = total_words
+
+    def actual_bpp(self) -> float:
+        return float(load_library().e8_ep_actual_bpp(self.N, self.K, self.total_words))
+
+
+def _ep_ws(N, K, dev, workspace):
+    return _workspace(load_library().e8_ep_encode_workspace_bytes(N, K), dev, workspace)
+
+
+def e8_ep_encode(cb: Codebook, W, delta: float, workspace=None, stream=None) -> EpMatrix:
+    """W fp32 [N, K] (CUDA) at step delta -> EpMatrix (synchronous)."""
+    import torch
+    N, K = W.shape
+    lib = load_library()
+    dev = W.device
+    nmax = max(int(lib.e8_ep_max_words(N, K)), 1)
+    nb = max(int(lib.e8_ep_num_blocks(N, K)), 0)
+    words = torch.empty(nmax, dtype=torch.uint16, device=dev)
+    offsets = torch.empty(nb + 1, dtype=torch.int32, device=dev)
+    t = torch.empty(max(N, 1), dtype=torch.float32, device=dev)
+    tables = torch.empty(E8_EP_TABLE_WORDS, dtype=torch.uint16, device=dev)
+    total = ctypes.c_int64(0)
+    ws = _ep_ws(N, K, dev, workspace)
+    rc = lib.e8_ep_encode(cb.handle, _ptr(W), N, K, float(delta), _ptr(words), nmax,
+                          _ptr(offsets), _ptr(t), _ptr(tables), ctypes.byref(total), _ptr(ws),
+                          ws.numel(), _stream(stream))
+    _check(rc, "e8_ep_encode")
+    return EpMatrix(N, K, float(delta), words[:max(total.value, 1)], offsets, t[:N], tables,
+                    total.value)
+
+
+def e8_ep_estimate_bpp(cb: Codebook, W, delta: float, workspace=None, stream=None) -> float:
+    N, K = W.shape
+    out = ctypes.c_double(0.0)
+    ws = _ep_ws(N, K, W.device, workspace)
+    rc = load_library().e8_ep_estimate_bpp(cb.handle, _ptr(W), N, K, float(delta),
+                                           ctypes.byref(out), _ptr(ws), ws.numel(), _stream(stream))
+    _check(rc, "e8_ep_estimate_bpp")
+    return out.value
+
+
+def e8_ep_choose_delta(cb: Codebook, W, target_bpp: float, workspace=None, stream=None) -> float:
+    N, K = W.shape
+    out = ctypes.c_float(0.0)
+    ws = _ep_ws(N, K, W.device, workspace)
+    rc = load_library().e8_ep_choose_delta(cb.handle, _ptr(W), N, K, float(target_bpp),
+                                           ctypes.byref(out), _ptr(ws), ws.numel(), _stream(stream))
+    _check(rc, "e8_ep_choose_delta")
+    return out.value
+
+
+def e8_ep_decode_to_bf16(cb: Codebook, m: EpMatrix, out=None, stream=None):
+    """bf16 [N, K] weights of an EpMatrix."""
+    import torch
+    if out is None:
+        out = torch.empty((m.N, m.K), dtype=torch.bfloat16, device=m.words.device)
+    rc = load_library().e8_ep_decode_to_bf16(cb.handle, _ptr(m.words), m.words.numel(),
+                                             _ptr(m.offsets),
+                                             _ptr(m.t), _ptr(m.tables), m.N, m.K, _ptr(out),
+                                             _stream(stream))
+    _check(rc, "e8_ep_decode_to_bf16")
+    return out
+
+
+def e8_ep_gemm(cb: Codebook, X, m: EpMatrix, Y=None, workspace=None, stream=None):
+    """Y fp32 [M, N] = X bf16 [M, K] times the decoded weights, transposed."""
+    import torch
+    M = X.shape[0]
+    lib = load_library()
+    if Y is None:
+        Y = torch.empty((M, m.N), dtype=torch.float32, device=X.device)
+    ws = _workspace(lib.e8_ep_gemm_workspace_bytes(M, m.N, m.K), X.device, workspace)
+    rc = lib.e8_ep_gemm(cb.handle, _ptr(X), M, _ptr(m.words), m.words.numel(), _ptr(m.offsets),
+                        _ptr(m.t),
+                        _ptr(m.tables), m.N, m.K, _ptr(Y), _ptr(ws), ws.numel(), _stream(stream))
+    _check(rc, "e8_ep_gemm")
+    return Y
+

@@ -168,6 +168,7 @@ const char* e8_status_str(int s) {
     case E8_ECUDA: return "CUDA error";
     case E8_ETIMEOUT: return "device wait timed out";
     case E8_ENOMEM: return "out of device memory";
+    case E8_EDATA: return "malformed compressed stream";
     default: return "unknown status";
   }
 }
@@ -612,6 +613,8 @@ int e8_sync_status(const e8_codebook* cb, void* stream) {
   if (s & (e8::kDevTimeoutFull | e8::kDevTimeoutEmpty | e8::kDevTimeoutMma | e8::kDevTimeoutCluster))
     return E8_ETIMEOUT;
   if (s & e8::kDevWorklistOverflow) return E8_EWORKSPACE;
+  if (s & e8::kDevBadStream) return E8_EDATA;
+  if (s & e8::kDevBadInput) return E8_EINVAL;
   return E8_OK;
 }
 

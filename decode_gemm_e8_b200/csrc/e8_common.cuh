@@ -25,6 +25,7 @@ enum : uint32_t {
   kDevTimeoutCluster = 1u << 3,  // a cluster peer never arrived
   kDevWorklistOverflow = 1u << 4,
   kDevBadInput = 1u << 5,
+  kDevBadStream = 1u << 6,       // an entropy-coded stream did not decode exactly
 };
 
 // Give up on a wait after this many nanoseconds of %globaltimer.

@@ -203,6 +203,23 @@ cudaError_t run_act_gemm(const e8_codebook* cb, const uint16_t* X, int64_t M,
                          uint64_t seed, float alpha, float* Y, int smem_variant, void* scratch,
                          cudaStream_t st, int64_t nh = 0);
 
+// Entropy-coded E8 variant (e8_ep.cu).
+constexpr int kEpBlockGroups = 64;    // groups of 8 weights per independently decodable block
+constexpr int kEpTableWords = 770;    // frequency tables: c, m|0, m|1, q|0, q|1
+int64_t ep_num_blocks(int64_t N, int64_t K);
+int64_t ep_max_words(int64_t N, int64_t K);
+size_t ep_encode_workspace_bytes(int64_t N, int64_t K);
+// 0 ok, 1 CUDA error, 2 frequency normalisation impossible, 3 stream longer
+// than max_words.  Synchronises the stream.
+int ep_encode(const float* W, int64_t N, int64_t K, float delta, uint16_t* words,
+              int64_t max_words, uint32_t* offsets, float* t, uint16_t* tables, void* ws,
+              uint32_t* status, int sm_count, cudaStream_t st, int64_t* total_words);
+int ep_estimate_bpp(const float* W, int64_t N, int64_t K, float delta, void* ws,
+                    uint32_t* status, int sm_count, cudaStream_t st, double* bpp);
+cudaError_t launch_ep_decode(const uint16_t* words, int64_t n_words, const uint32_t* offsets,
+                             const float* t, const uint16_t* tables, int64_t N, int64_t K,
+                             uint16_t* out, uint32_t* status, int sm_count, cudaStream_t st);
+
 // Dense Y[M][N] fp32 = X[M][K] bf16 * W[N][K]^T bf16 on tcgen05.
 cudaError_t launch_dense_gemm(const uint16_t* X, int64_t M, const uint16_t* W, int64_t N,
                               int64_t K, float* Y, uint32_t* status, int sm_count,

@@ -68,6 +68,7 @@ extern "C" {
 #define E8_ECUDA 4       /* a CUDA runtime or driver call failed */
 #define E8_ETIMEOUT 5    /* a kernel gave up on a bounded wait (reported by e8_sync_status) */
 #define E8_ENOMEM 6      /* device allocation failed (e8_codebook_build only) */
+#define E8_EDATA 7       /* an entropy-coded stream did not decode exactly (e8_sync_status) */
 
 /* GEMM modes (e8_gemm `mode`, and `op` of e8_workspace_bytes). */
 #define E8_GEMM_AUTO 0          /* ACT_RHT for M <= 64 and K % 128 == 0, else DECODED_W */
@@ -307,9 +308,87 @@ size_t e8_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int bpw);
 
 /* Synchronises `stream`, then reads and clears the codebook's device status
  * word.  Returns E8_ETIMEOUT if a kernel gave up on a bounded wait since the
- * last call, E8_EWORKSPACE on an encoder work-list overflow, E8_ECUDA if the
- * stream reported an error, else E8_OK. */
+ * last call, E8_EWORKSPACE on an encoder work-list overflow, E8_EDATA if an
+ * entropy-coded stream did not decode exactly, E8_EINVAL if an entropy-coded
+ * encode met a weight outside the quantiser's range (non-finite), E8_ECUDA if
+ * the stream reported an error, else E8_OK. */
 int e8_sync_status(const e8_codebook* cb, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Entropy-coded E8 variant (page "Transformers Proposes EntroPack Integration
+ * for Configurable Non-Integer-Bit-Rate Weight Compression", second paragraph:
+ * per-row normalised E8 lattice quantisation, a conditional probability model,
+ * entropy coding into independently decodable blocks, fused symbol decoding and
+ * weight reconstruction on the GPU; third paragraph: the actual rate counts
+ * the metadata).  The page fixes no detail; this library's format:
+ *   - row scale t_n = fl32(max_k |w_nk| * delta) (0 when below FLT_MIN), for a
+ *     global step delta >= 1/120; u = fl32(w * fl32(1 / t_n)) per group of 8;
+ *   - V = the E8 point of u in doubled coordinates chosen by Conway & Sloane's
+ *     algorithm in fp32 with fixed tie rules (whole lattice, no codebook);
+ *   - decoded weight w' = bf16_rne(fl32(V * fl32(t_n / 2)));
+ *   - per group 9 symbols: coset c, seven m_i = (V_i - c) / 2, q = floor(m_7 / 2),
+ *     coded by rANS (32-bit state, 16-bit words, 12-bit frequencies) with the
+ *     models P(c), P(m | c), P(q | c) counted over the matrix;
+ *   - the groups of the row-major matrix in blocks of E8_EP_BLOCK_GROUPS, each
+ *     block its own stream of 16-bit words from offsets[b] to offsets[b + 1];
+ *   - tables: E8_EP_TABLE_WORDS uint16 frequencies (c[2], m|0[256], m|1[256],
+ *     q|0[128], q|1[128]), each model summing to 4096;
+ *   - actual bits per weight = (16 words + 32 (blocks + 1) + 32 N
+ *     + 16 E8_EP_TABLE_WORDS + 32) / (N K).
+ * Shapes: K >= 8, K % 8 == 0, N K / 8 <= 2^31.  The codebook handle only
+ * selects the device and carries the status word. */
+#define E8_EP_BLOCK_GROUPS 64
+#define E8_EP_TABLE_WORDS 770
+
+/* Blocks of an N x K matrix (ceil(N K / 8 / 64)) and the most stream words an
+ * encode can produce (9 per group + 2 per block); -1 for an invalid shape. */
+int64_t e8_ep_num_blocks(int64_t N, int64_t K);
+int64_t e8_ep_max_words(int64_t N, int64_t K);
+
+/* Actual bits per weight of an encoded matrix, metadata included (formula
+ * above); -1 for an invalid shape or N = 0. */
+double e8_ep_actual_bpp(int64_t N, int64_t K, int64_t total_words);
+
+/* Workspace bytes of e8_ep_encode / e8_ep_estimate_bpp / e8_ep_choose_delta
+ * (symbols, block sizes, row scales, histogram), and of e8_ep_gemm (the
+ * decoded bf16 weights); 0 for an invalid shape. */
+size_t e8_ep_encode_workspace_bytes(int64_t N, int64_t K);
+size_t e8_ep_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/* Encoder: W fp32 [N][K] (finite) at step delta -> words uint16
+ * [max_words >= the stream], offsets uint32 [blocks + 1], t fp32 [N], tables
+ * uint16 [E8_EP_TABLE_WORDS]; *total_words (host) = offsets[blocks].
+ * Synchronous (it reads the histogram and the block sizes back to the host).
+ * E8_EWORKSPACE if max_words is too small or the workspace is. */
+int e8_ep_encode(const e8_codebook* cb, const float* W, int64_t N, int64_t K, float delta,
+                 uint16_t* words, int64_t max_words, uint32_t* offsets, float* t,
+                 uint16_t* tables, int64_t* total_words, void* workspace, size_t ws_bytes,
+                 void* stream);
+
+/* Estimated bits per weight at step delta, metadata included (the model's
+ * ideal code lengths plus 32 bits of final state per block); synchronous.
+ * e8_ep_choose_delta: the smallest step in [1/120, 16] (bisection on log
+ * delta) whose estimate is at most target_bpp; synchronous. */
+int e8_ep_estimate_bpp(const e8_codebook* cb, const float* W, int64_t N, int64_t K, float delta,
+                       double* bpp, void* workspace, size_t ws_bytes, void* stream);
+int e8_ep_choose_delta(const e8_codebook* cb, const float* W, int64_t N, int64_t K,
+                       double target_bpp, float* delta, void* workspace, size_t ws_bytes,
+                       void* stream);
+
+/* Decoder: the compressed form -> bf16 weights out [N][K] (16-byte aligned),
+ * one thread per block.  n_words: length of `words` (no read goes past it).
+ * A block whose offsets leave [0, n_words], whose stream runs past its end or
+ * does not return to the initial state sets E8_EDATA (read by
+ * e8_sync_status); its weights are then unspecified. */
+int e8_ep_decode_to_bf16(const e8_codebook* cb, const uint16_t* words, int64_t n_words,
+                         const uint32_t* offsets, const float* t, const uint16_t* tables,
+                         int64_t N, int64_t K, uint16_t* out, void* stream);
+
+/* Y fp32 [M][N] = X bf16 [M][K] * W'^T: the decoder into the workspace
+ * (e8_ep_gemm_workspace_bytes), then the dense tcgen05 GEMM of E8_GEMM_DECODED_W. */
+int e8_ep_gemm(const e8_codebook* cb, const uint16_t* X, int64_t M, const uint16_t* words,
+               int64_t n_words, const uint32_t* offsets, const float* t, const uint16_t* tables,
+               int64_t N, int64_t K, float* Y, void* workspace, size_t ws_bytes, void* stream);
 
 /* Failure-detection check (diagnostic): launches one thread that waits on a
  * barrier nothing ever signals, gives up after wait_ms (1..5000) milliseconds
