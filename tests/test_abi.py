@@ -210,3 +210,33 @@ def test_explicit_block_workspace_sizes(lib):
         assert e8.e8_workspace_bytes(e8.E8_GEMM_ACT_RHT, 16, N, K, 4, nh=nh) == 0
     assert e8.e8_workspace_bytes(e8.E8_GEMM_DECODED_W, 64, N, 3072, 4, nh=2048) == 0
     assert e8.e8_workspace_bytes(e8.E8_GEMM_DECODED_W, 64, N, 3072, 4, nh=1024) == N * 3072 * 2
+
+
+def test_entropy_coded_sizes_and_rate(lib):
+    # host-only queries of the entropy-coded variant: blocks of 64 groups, at
+    # most 9 words per group plus 2 per block, the rate formula of the oracle
+    from oracle import ep_oracle as ep
+    assert lib.e8_ep_num_blocks(4096, 4096) == 4096 * 512 // 64
+    assert lib.e8_ep_num_blocks(7, 1000) == (7 * 125 + 63) // 64
+    assert lib.e8_ep_max_words(7, 1000) == 9 * 875 + 2 * 14
+    for bad in ((4, 12), (4, 0), (-1, 64)):
+        assert lib.e8_ep_num_blocks(*bad) == -1
+        assert lib.e8_ep_encode_workspace_bytes(*bad) == 0
+        assert lib.e8_ep_gemm_workspace_bytes(16, *bad) == 0
+    assert lib.e8_ep_gemm_workspace_bytes(16, 3072, 3072) == 3072 * 3072 * 2
+    for N, K, words in ((24, 256, 1234), (3072, 3072, 2_300_000), (1, 8, 2)):
+        nb = lib.e8_ep_num_blocks(N, K)
+        enc = {"N": N, "K": K, "offsets": [0] * nb + [words]}
+        assert lib.e8_ep_actual_bpp(N, K, words) == pytest.approx(ep.actual_bpp(enc), rel=1e-12)
+    assert lib.e8_ep_actual_bpp(0, 64, 0) == -1.0
+
+
+def test_entropy_coded_refusals_need_no_gpu(lib):
+    import ctypes
+    tw = ctypes.c_int64(5)
+    # no codebook handle: refused before any device work
+    assert lib.e8_ep_encode(None, None, 4, 64, 0.05, None, 0, None, None, None,
+                            ctypes.byref(tw), None, 0, None) == e8.E8_EINVAL
+    assert lib.e8_ep_decode_to_bf16(None, None, 0, None, None, None, 4, 64, None,
+                                    None) == e8.E8_EINVAL
+    assert e8.status_str(e8.E8_EDATA) == "malformed compressed stream"
