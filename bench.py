@@ -210,7 +210,7 @@ def run_ours(args):
     if args.profile == "decode":
         _profile_decode(e8, dev)
         return
-    if args.profile in ("dense_up", "dense_out", "encode", "gemm_mlp", "ep_decode"):
+    if args.profile in ("dense_up", "dense_out", "encode", "gemm_mlp", "ep_decode", "grouped"):
         _profile_other(e8, synth, dev, args.profile)
         return
     peaks = _peaks()
@@ -440,7 +440,10 @@ def _profile_other(e8, synth, dev, mode):
       gemm_mlp   three small-batch products (16 tokens) of a 14336 x 4096
                  matrix at 4 bpw on pre-transformed activations (k_gemm_q8)
       ep_decode  the entropy-coded variant: three decodes of a 14336 x 4096
-                 Gaussian matrix at delta 0.075 (about 4 bpp)"""
+                 Gaussian matrix at delta 0.075 (about 4 bpp)
+      grouped    three grouped small-batch calls (e8_gemm_grouped) of the q, k,
+                 v projections of a Llama-3-8B layer (4096, 1024, 1024 rows x
+                 4096, 4 bpw, 16 tokens): one transform and one GEMM launch each"""
     import torch
     gen = torch.Generator(device=dev)
     gen.manual_seed(7)
@@ -453,6 +456,17 @@ def _profile_other(e8, synth, dev, mode):
                          dtype=torch.uint8, device=dev)
         for _ in range(2):
             e8.e8_gemm(cb, X, c1, c2, N, K, bpw, 1, 0.02, mode=e8.E8_GEMM_DECODED_W, workspace=ws)
+    elif mode == "grouped":
+        K, bpw, M = 4096, 4, 16
+        items = []
+        for j, N in enumerate((4096, 1024, 1024)):
+            c1, c2 = _random_codes(torch, dev, N, K, bpw, gen)
+            items.append((c1, c2, N, 100 + j, 0.02))
+        X = torch.randn((M, K), generator=gen, device=dev).to(torch.bfloat16)
+        ws = torch.empty(e8.e8_gemm_grouped_workspace_bytes(M, K, bpw, len(items)),
+                         dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            e8.e8_gemm_grouped(cb, X, items, K, bpw, workspace=ws)
     elif mode == "ep_decode":
         W = torch.from_numpy(synth.gaussian_weights(14336, 4096, 0.02, 4)).to(dev)
         m = e8.e8_ep_encode(cb, W, 0.075)
@@ -855,7 +869,7 @@ def main():
                     help="skip the load phase that precedes the timed region (clock record)")
     ap.add_argument("--profile", nargs="?", const="gemm",
                     choices=["gemm", "decode", "dense_up", "dense_out", "encode", "gemm_mlp",
-                             "ep_decode"],
+                             "ep_decode", "grouped"],
                     help="small runs for ncu captures, then exit: 8 eager steps of the "
                          "headline call (gemm), 3 bf16 decodes of a 14336 x 4096 matrix "
                          "(decode), prefill GEMMs (dense_up, dense_out), two encodes "
