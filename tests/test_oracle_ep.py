@@ -200,3 +200,23 @@ def test_symbol_bounds_at_the_smallest_step():
     assert S[:, 8].min() >= -64 and S[:, 8].max() <= 63
     with pytest.raises(ValueError):
         ep.quantise(W, 1 / 121)
+
+
+@pytest.mark.parametrize("scale", [0.4, 0.9])
+def test_nearest_e8_agrees_with_the_codebook_brute_force(scale):
+    # inside the full shells (squared norm <= 10) the nearest lattice point is
+    # the nearest codebook point, which the main oracle finds by an exact
+    # brute force over all 65536 entries (a separate implementation)
+    from oracle import oracle as orc
+    rng = np.random.default_rng(int(scale * 100))
+    U = (rng.standard_normal((2000, 8)) * scale).astype(np.float32)
+    V = ep.nearest_e8(U)
+    keep = (V.astype(np.int64) ** 2).sum(axis=1) <= 40   # doubled: squared norm <= 10
+    i1, _ = orc.nearest_groups(U[keep], 2)
+    C = orc.codebook().astype(np.int32)
+    W = C[i1.astype(np.int64)]
+    diff = np.any(W != V[keep], axis=1)
+    for u, a, b in zip(U[keep][diff], V[keep][diff], W[diff]):
+        # a different choice only on an exact tie of the two distances
+        assert orc.cmp_dist(u, a, b, 2) == 0
+    assert keep.sum() > 1500
